@@ -1,0 +1,387 @@
+"""Pins of the fp64 oracle against things other than itself: closed forms,
+invariants, brute force on tiny inputs, library routines (torch fp64) and
+hand-written fixtures in tests/golden/.  CPU only."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import synth
+from oracle import vit_ref as R
+from oracle import run as orun
+from tests import torch_fp64_layer
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+# ------------------------------------------------------------------ LayerNorm
+def test_layernorm_matches_torch():
+    x = rng(1).standard_normal((7, 33)) * 3 + 1.5
+    g = 1 + 0.1 * rng(2).standard_normal(33)
+    b = 0.1 * rng(3).standard_normal(33)
+    ref = F.layer_norm(torch.tensor(x), (33,), torch.tensor(g), torch.tensor(b), 1e-6).numpy()
+    np.testing.assert_allclose(R.layernorm(x, g, b, 1e-6), ref, rtol=0, atol=1e-13)
+
+
+def test_layernorm_moments_closed_form():
+    # gamma = 1, beta = 0: per-row mean 0, biased variance v / (v + eps)
+    x = rng(4).standard_normal((5, 1152)) * 2.0 - 0.7
+    eps = 1e-2      # large eps so a dropped or misplaced eps is visible
+    y = R.layernorm(x, np.ones(1152), np.zeros(1152), eps)
+    v = x.var(axis=1)          # numpy var is the biased variance
+    np.testing.assert_allclose(y.mean(axis=1), 0, atol=1e-13)
+    np.testing.assert_allclose((y ** 2).mean(axis=1), v / (v + eps), rtol=1e-12)
+
+
+def test_layernorm_affine_and_constant_row():
+    x = np.tile(np.array([[2.5]]), (1, 8))            # constant row: x - mean = 0
+    g = np.arange(8.0)
+    b = np.linspace(-1, 1, 8)
+    np.testing.assert_array_equal(R.layernorm(x, g, b), np.broadcast_to(b, (1, 8)))
+    x = np.array([[1.0, -1.0]])                         # mean 0, var 1
+    y = R.layernorm(x, np.array([2.0, 3.0]), np.array([0.5, -0.5]), eps=0.0)
+    np.testing.assert_allclose(y, [[2.5, -3.5]], atol=1e-15)
+
+
+# ------------------------------------------------------------------ GEMM
+def test_linear_brute_force():
+    x = rng(5).standard_normal((3, 4))
+    w = rng(6).standard_normal((5, 4))
+    b = rng(7).standard_normal(5)
+    y = R.linear(x, w, b)
+    for i in range(3):
+        for j in range(5):
+            acc = b[j]
+            for k in range(4):
+                acc += x[i, k] * w[j, k]
+            assert abs(y[i, j] - acc) < 1e-13
+
+
+def test_linear_matches_torch():
+    x = rng(8).standard_normal((17, 40))
+    w = rng(9).standard_normal((23, 40))
+    b = rng(10).standard_normal(23)
+    ref = F.linear(torch.tensor(x), torch.tensor(w), torch.tensor(b)).numpy()
+    np.testing.assert_allclose(R.linear(x, w, b), ref, atol=1e-12)
+
+
+# ------------------------------------------------------------------ GELU
+def test_gelu_tanh_identities():
+    u = np.linspace(-6, 6, 1001)
+    g = R.gelu_tanh(u)
+    assert R.gelu_tanh(np.array([0.0]))[0] == 0.0
+    # 0.5u(1+tanh(a)) - (-0.5u)(1+tanh(-a)) = u exactly (tanh odd)
+    np.testing.assert_allclose(g - R.gelu_tanh(-u), u, atol=1e-14)
+    # the tanh form stays within 1e-3 of the exact erf form
+    exact = np.array([0.5 * t * (1 + math.erf(t / math.sqrt(2))) for t in u])
+    assert np.max(np.abs(g - exact)) < 1e-3
+    # large |u| limits: identity and zero
+    assert abs(R.gelu_tanh(np.array([30.0]))[0] - 30.0) < 1e-12
+    assert abs(R.gelu_tanh(np.array([-30.0]))[0]) < 1e-12
+
+
+def test_gelu_tanh_matches_torch():
+    u = rng(11).standard_normal(1000) * 4
+    ref = F.gelu(torch.tensor(u), approximate="tanh").numpy()
+    np.testing.assert_allclose(R.gelu_tanh(u), ref, atol=1e-14)
+
+
+# ------------------------------------------------------------------ RoPE
+def _golden_rope():
+    vals = []
+    with open(os.path.join(GOLDEN, "rope2d_d8_example.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            i, _expr, v = line.split()
+            vals.append((int(i), float(v)))
+    return np.array([v for _, v in sorted(vals)])
+
+
+def test_rope_golden_example():
+    x = np.arange(1.0, 9.0).reshape(1, 1, 8)
+    y = R.rope2d(x, np.array([[1, 2]]), theta=100.0)
+    np.testing.assert_allclose(y[0, 0], _golden_rope(), atol=1e-14)
+
+
+@pytest.mark.parametrize("d", [8, 64, 72, 128])
+def test_rope_each_coordinate_angle(d):
+    # unit vector in dim j of a half rotates into dim j + h/2 by angle p*w_j
+    theta = 10000.0
+    h = d // 2
+    for axis in (0, 1):
+        for j in range(h // 2):
+            e = np.zeros((1, 1, d))
+            e[0, 0, axis * h + j] = 1.0
+            pos = np.array([[3, 0]]) if axis == 0 else np.array([[0, 5]])
+            p = pos[0, axis]
+            ang = p * theta ** (-2.0 * j / h)
+            y = R.rope2d(e, pos, theta)[0, 0]
+            expect = np.zeros(d)
+            expect[axis * h + j] = math.cos(ang)
+            expect[axis * h + h // 2 + j] = math.sin(ang)
+            np.testing.assert_allclose(y, expect, atol=1e-14)
+
+
+def test_rope_identity_norm_composition():
+    d = 72
+    x = rng(12).standard_normal((6, 3, d))
+    np.testing.assert_array_equal(R.rope2d(x, np.zeros((6, 2), int)), x)
+    pos = rng(13).integers(0, 80, size=(6, 2))
+    y = R.rope2d(x, pos)
+    # norm preserved per rotated pair
+    h = d // 2
+    for lo in (0, h):
+        a0, b0 = x[..., lo:lo + h // 2], x[..., lo + h // 2:lo + h]
+        a1, b1 = y[..., lo:lo + h // 2], y[..., lo + h // 2:lo + h]
+        np.testing.assert_allclose(a0 ** 2 + b0 ** 2, a1 ** 2 + b1 ** 2, rtol=1e-12)
+    # R(a) R(b) = R(a + b)
+    p2 = rng(14).integers(-40, 40, size=(6, 2))
+    np.testing.assert_allclose(R.rope2d(R.rope2d(x, pos), p2), R.rope2d(x, pos + p2), atol=1e-11)
+
+
+def test_rope_relative_offset():
+    # <R(p) q, R(p') k> depends only on p' - p: shifting both by s is invisible
+    d = 72
+    q = rng(15).standard_normal((1, 1, d))
+    k = rng(16).standard_normal((1, 1, d))
+    p, pk = np.array([[3, 7]]), np.array([[11, 2]])
+    base = float(np.sum(R.rope2d(q, p) * R.rope2d(k, pk)))
+    for s in ([1, 0], [0, 1], [5, -9], [40, 33]):
+        s = np.array([s])
+        v = float(np.sum(R.rope2d(q, p + s) * R.rope2d(k, pk + s)))
+        assert abs(v - base) < 1e-11
+    # and equals <q, R(p' - p) k>
+    v = float(np.sum(q * R.rope2d(k, pk - p)))
+    assert abs(v - base) < 1e-11
+
+
+# ------------------------------------------------------------------ attention
+def _brute_attention(q, k, v, scale):
+    n, m = q.shape[0], k.shape[0]
+    out = np.zeros((n, v.shape[1]))
+    for i in range(n):
+        s = [sum(q[i, t] * k[j, t] for t in range(q.shape[1])) * scale for j in range(m)]
+        mx = max(s)
+        e = [math.exp(x - mx) for x in s]
+        z = sum(e)
+        for j in range(m):
+            out[i] += e[j] / z * v[j]
+    return out
+
+
+def test_attention_brute_force_tiny():
+    T, H, d = 8, 2, 4
+    q, k, v = (rng(s).standard_normal((T, H, d)) for s in (20, 21, 22))
+    o = R.attention(q, k, v, [0, T])
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h], _brute_attention(q[:, h], k[:, h], v[:, h], 0.5),
+                                   atol=1e-13)
+
+
+def test_attention_matches_torch_sdpa():
+    T, H, d = 37, 3, 72
+    q, k, v = (rng(s).standard_normal((T, H, d)) for s in (23, 24, 25))
+    ref = F.scaled_dot_product_attention(*(torch.tensor(t).transpose(0, 1) for t in (q, k, v)))
+    np.testing.assert_allclose(R.attention(q, k, v, [0, T]), ref.transpose(0, 1).numpy(),
+                               atol=1e-13)
+
+
+def test_attention_rows_sum_to_one():
+    # with V = identity the output rows are the softmax rows themselves
+    n, d = 6, 6
+    q = rng(26).standard_normal((n, 1, d)) * 3
+    k = rng(27).standard_normal((n, 1, d)) * 3
+    v = np.eye(n).reshape(n, 1, d)
+    p = R.attention(q, k, v, [0, n])[:, 0]
+    assert np.all(p >= 0)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-14)
+
+
+def test_attention_special_cases():
+    n, d = 9, 8
+    q = rng(28).standard_normal((n, 1, d))
+    v = rng(29).standard_normal((n, 1, d))
+    # all keys equal -> every output row is the mean of V
+    k = np.tile(rng(30).standard_normal((1, 1, d)), (n, 1, 1))
+    o = R.attention(q, k, v, [0, n])
+    np.testing.assert_allclose(o[:, 0], np.tile(v[:, 0].mean(0), (n, 1)), atol=1e-14)
+    # one dominant key -> its V row
+    k = np.zeros((n, 1, d))
+    k[4, 0, :] = 1.0
+    qd = np.full((n, 1, d), 200.0)
+    o = R.attention(qd, k, v, [0, n])
+    np.testing.assert_allclose(o[:, 0], np.tile(v[4, 0], (n, 1)), atol=1e-12)
+    # a scale argument multiplies the logits
+    k = rng(31).standard_normal((n, 1, d))
+    o1 = R.attention(q, k, v, [0, n], scale=0.7)
+    o2 = R.attention(q * 0.7 * math.sqrt(d), k, v, [0, n])
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+
+
+def test_attention_permutations():
+    n, H, d = 10, 2, 8
+    q, k, v = (rng(s).standard_normal((n, H, d)) for s in (32, 33, 34))
+    o = R.attention(q, k, v, [0, n])
+    perm = rng(35).permutation(n)
+    # permuting queries permutes outputs; permuting (K, V) jointly changes nothing
+    np.testing.assert_allclose(R.attention(q[perm], k, v, [0, n]), o[perm], atol=1e-13)
+    np.testing.assert_allclose(R.attention(q, k[perm], v[perm], [0, n]), o, atol=1e-13)
+
+
+def test_attention_varlen_is_block_diagonal():
+    lens = [5, 1, 7, 3]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, H, d = cu[-1], 2, 8
+    q, k, v = (rng(s).standard_normal((T, H, d)) for s in (36, 37, 38))
+    pos = rng(39).integers(0, 9, size=(T, 2))
+    o = R.attention(q, k, v, cu, pos)
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        np.testing.assert_allclose(o[a:b], R.attention(q[a:b], k[a:b], v[a:b], [0, b - a],
+                                                       pos[a:b]), atol=1e-13)
+    # reversing the segment order reverses the output blocks
+    order = list(range(len(lens)))[::-1]
+    idx = np.concatenate([np.arange(cu[s], cu[s + 1]) for s in order])
+    cu2 = np.concatenate([[0], np.cumsum([lens[s] for s in order])])
+    o2 = R.attention(q[idx], k[idx], v[idx], cu2, pos[idx])
+    np.testing.assert_allclose(o2, o[idx], atol=1e-13)
+
+
+def test_attention_prefix_is_concatenation():
+    lens, P, H, Hkv, d = [6, 4], 5, 4, 2, 8
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T = cu[-1]
+    q, k, v = (rng(s).standard_normal((T, H, d)) for s in (40, 41, 42))
+    pkv = rng(43).standard_normal((2, 2, P, Hkv, d))
+    pos = rng(44).integers(0, 5, size=(T, 2))
+    o = R.attention(q, k, v, cu, pos, pkv)
+    qr, kr = R.rope2d(q, pos), R.rope2d(k, pos)
+    for s in range(2):
+        a, b = cu[s], cu[s + 1]
+        for h in range(H):
+            ks = np.concatenate([pkv[s, 0, :, h // 2], kr[a:b, h]])
+            vs = np.concatenate([pkv[s, 1, :, h // 2], v[a:b, h]])
+            np.testing.assert_allclose(o[a:b, h], _brute_attention(qr[a:b, h], ks, vs,
+                                                                   1 / math.sqrt(d)), atol=1e-12)
+
+
+# ------------------------------------------------------------------ merge / positions
+def _golden_merge():
+    maps = {}
+    with open(os.path.join(GOLDEN, "merge_index_maps.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            grids, rest = line.split("|")
+            o, ins = rest.split(":")
+            maps.setdefault(grids.strip(), {})[int(o)] = [int(t) for t in ins.split()]
+    return maps
+
+
+def test_merge_golden_index_maps():
+    for key, m in _golden_merge().items():
+        grids = [tuple(int(a) for a in g.split("x")) for g in key.split(",")]
+        T = synth.grid_tokens(grids)
+        C = 3
+        x = np.arange(T * C).reshape(T, C)     # token t holds t*C .. t*C+C-1
+        y = R.spatial_merge_2x2(x, grids)
+        assert y.shape == (T // 4, 4 * C)
+        for o, ins in m.items():
+            expect = np.concatenate([x[t] for t in ins])
+            np.testing.assert_array_equal(y[o], expect)
+
+
+def test_merge_is_a_permutation():
+    grids = [(6, 8), (2, 2), (4, 10)]
+    T = synth.grid_tokens(grids)
+    C = 5
+    x = np.arange(T * C).reshape(T, C)
+    y = R.spatial_merge_2x2(x, grids)
+    flat = y.reshape(-1)
+    assert sorted(flat.tolist()) == list(range(T * C))        # bijection
+    inv = np.empty(T * C, dtype=np.int64)
+    inv[flat] = np.arange(T * C)
+    np.testing.assert_array_equal(flat[inv].reshape(T, C), x)    # inverse recovers x
+    with pytest.raises(ValueError):
+        R.spatial_merge_2x2(np.zeros((60 * 65, 1)), [(60, 65)])
+
+
+def test_positions_golden():
+    with open(os.path.join(GOLDEN, "positions_2x3_1x2.txt")) as f:
+        lines = [ln for ln in f if not ln.startswith("#")]
+    cu_exp = [int(t) for t in lines[0].split(":")[1].split()]
+    pos_exp = [tuple(int(a) for a in t.split(",")) for t in lines[1].split(":")[1].split()]
+    cu, pos = R.positions_from_grids([(2, 3), (1, 2)])
+    assert cu.tolist() == cu_exp
+    assert [tuple(p) for p in pos.tolist()] == pos_exp
+
+
+# ------------------------------------------------------------------ layer / stack
+def _small_layer_inputs(seed, T_grids, C=64, H=4, d=16, Fm=96, dtype="f32", P=0, attn_only=False):
+    wl = synth.Workload("t", seed, dtype, C, H, d, Fm, 2, tuple(T_grids),
+                        prefix_len=P, kv_heads=(H // 2 if P else 0), attn_only=attn_only)
+    return wl, synth.make_inputs(wl)
+
+
+@pytest.mark.parametrize("P,attn_only", [(0, False), (3, True)])
+def test_layer_matches_torch_restatement(P, attn_only):
+    wl, inp = _small_layer_inputs(50, [(3, 4), (2, 5)], P=P, attn_only=attn_only)
+    cu, pos = R.positions_from_grids(wl.grids)
+    w = orun.layer_f64(inp, 0)
+    x = synth.to_f64(inp.x, wl.dtype)
+    pkv = None if inp.prefix_kv is None else synth.to_f64(inp.prefix_kv, wl.dtype)
+    y = R.layer_forward(x, w, cu, pos, wl.heads, wl.head_dim, wl.ln_eps, wl.rope_theta, pkv,
+                        attn_only)
+    ref = torch_fp64_layer.layer(x, w, cu, pos, wl.heads, wl.head_dim, wl.ln_eps,
+                                 wl.rope_theta, pkv, attn_only)
+    np.testing.assert_allclose(y, ref, atol=1e-12)
+
+
+def test_encoder_is_layer_composition():
+    wl, inp = _small_layer_inputs(51, [(4, 4)])
+    y2 = orun.run_layers(inp)
+    y1 = orun.run_layers(inp, n_layers=1)
+    cu, pos = R.positions_from_grids(wl.grids)
+    np.testing.assert_allclose(
+        y2, R.layer_forward(y1, orun.layer_f64(inp, 1), cu, pos, wl.heads, wl.head_dim),
+        atol=1e-13)
+
+
+def test_c1_layer_matches_torch_restatement():
+    wl = synth.get("c1")
+    inp = synth.make_inputs(wl)
+    cu, pos = R.positions_from_grids(wl.grids)
+    w = orun.layer_f64(inp, 0)
+    x = synth.to_f64(inp.x, wl.dtype)
+    y = R.layer_forward(x, w, cu, pos, wl.heads, wl.head_dim)
+    ref = torch_fp64_layer.layer(x, w, cu, pos, wl.heads, wl.head_dim, 1e-6, 1e4)
+    np.testing.assert_allclose(y, ref, atol=1e-10)
+
+
+# ------------------------------------------------------------------ synth
+def test_bf16_rounding_matches_torch():
+    a = rng(60).standard_normal(100000) * 10.0 ** rng(61).integers(-6, 6, 100000)
+    bits = synth.round_bf16_bits(a)
+    ref = torch.tensor(a.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+    np.testing.assert_array_equal(bits, ref.view(np.uint16))
+    np.testing.assert_array_equal(synth.bf16_bits_to_f64(bits),
+                                  torch.tensor(a.astype(np.float32)).to(torch.bfloat16)
+                                  .to(torch.float64).numpy())
+
+
+def test_workload_flop_counts():
+    # per-layer algorithmic FLOP of the 3900-token layer, by hand:
+    # GEMM 2*T*C*(3C + C + 2F); attention 4*T^2*C
+    f = synth.get("c2").flops()
+    T, C, Fm = 3900, 1152, 4304
+    assert f["gemm"] == 27 * 2.0 * T * C * (4 * C + 2 * Fm)
+    assert f["attn"] == 27 * 4.0 * T * T * C
+    assert abs(f["total"] - 5.0987e12) / 5.0987e12 < 1e-4
