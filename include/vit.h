@@ -1,0 +1,212 @@
+/*
+ * vit.h -- C ABI of libvit, a B200 (sm_100a) implementation of the vision
+ * transformer encoder hot path of an OCR vision-language model:
+ *
+ *   27 x [ LayerNorm -> QKV GEMM + bias -> 2D RoPE -> bidirectional
+ *          multi-head attention -> output projection + bias + residual ->
+ *          LayerNorm -> fc1 + bias -> GELU(tanh) -> fc2 + bias + residual ]
+ *   followed by the 2x2 spatial merge.
+ *
+ * Source of the method: KLiteInfer README (PaddleOCR-VL 0.9B vision tower),
+ * intro bullet "多模态全流程自研" (SigLIP ViT, 27 layers, 2D RoPE, bidirectional
+ * attention, 2x2 spatial merge), section "精度与性能" (27 layers x 3900 tokens
+ * of batched GEMMs) and section "架构", paragraph "视觉算子" (row-major batched
+ * tokens; GEMM + bias, bidirectional attention, LayerNorm, 2D RoPE, 2x2
+ * spatial merge).  The prefix K/V segment follows the LightX2V NeoPP README,
+ * section "KV file layout" (online layout [layers, 2, seq, kv_heads, d]).
+ *
+ * Conventions (all entry points):
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller, unless the
+ *    parameter name ends in _host.  The library never allocates or frees
+ *    device memory, except one 16-byte status word per context (allocated
+ *    by vit_init, freed by vit_destroy).
+ *  - Activations are row-major [tokens, features] with contiguous rows.
+ *    Weights use the [out_features, in_features] row-major layout.
+ *  - Element type of every floating tensor = vit_config.dtype (fp32 or bf16).
+ *    bf16 runs tcgen05 tensor-core kernels with fp32 accumulation; fp32 runs
+ *    SIMT FFMA kernels (no TF32).
+ *  - Streams are passed as void* (a cudaStream_t; NULL = legacy stream).  All
+ *    work is enqueued asynchronously on that stream.
+ *  - All argument and shape checks happen before anything is launched; on an
+ *    error status nothing was launched and outputs are untouched.  A failed
+ *    launch returns VIT_ERR_CUDA.  Faults detected inside a kernel (a bounded
+ *    wait that ran out, an index out of range) set the context's device
+ *    status word, read by vit_get_last_device_status().
+ *  - Pointers passed to bf16 entry points must be 16-byte aligned, and row
+ *    pitches (features x element size) multiples of 16 bytes.
+ *  - A context may be used from several host threads and streams at once as
+ *    long as each concurrent call has its own workspace.
+ */
+#ifndef VIT_H_
+#define VIT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VIT_API __attribute__((visibility("default")))
+#else
+#define VIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VIT_OK = 0,
+  VIT_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum      */
+  VIT_ERR_SHAPE = 2,         /* inconsistent sizes (odd merge grid, T != sum) */
+  VIT_ERR_UNSUPPORTED = 3,   /* valid but not implemented (head_dim 96, non-sm_100 device) */
+  VIT_ERR_WORKSPACE = 4,     /* workspace missing or too small              */
+  VIT_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed        */
+  VIT_ERR_TIMEOUT = 6,       /* a kernel's bounded wait ran out (device status) */
+  VIT_ERR_DEVICE_BOUNDS = 7  /* a kernel's index check failed (device status) */
+} vit_status;
+
+typedef enum { VIT_F32 = 0, VIT_BF16 = 1 } vit_dtype;
+
+/* vit_config.flags */
+#define VIT_FLAG_NO_ROPE 0x1u   /* layers skip 2D RoPE                        */
+#define VIT_FLAG_NO_MLP  0x2u   /* layers stop after the attention residual   */
+
+typedef struct {
+  int hidden;        /* C = heads * head_dim                                 */
+  int heads;         /* H                                                    */
+  int head_dim;      /* d: 64 (fp32 only), 72 or 128                         */
+  int mlp;           /* F, MLP width (ignored with VIT_FLAG_NO_MLP)          */
+  float ln_eps;      /* LayerNorm epsilon (biased variance), e.g. 1e-6       */
+  float rope_theta;  /* 2D RoPE base, e.g. 10000                             */
+  vit_dtype dtype;
+  unsigned flags;
+} vit_config;
+
+/* One layer's parameters; all device pointers of cfg.dtype.
+ * w_qkv [3C, C] (output rows: Q heads 0..H-1, then K, then V; d each),
+ * w_o [C, C], w_fc1 [F, C], w_fc2 [C, F]; biases and LayerNorm vectors 1-D.
+ * The ln2 / fc pointers may be NULL with VIT_FLAG_NO_MLP. */
+typedef struct {
+  const void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o;
+  const void *ln2_g, *ln2_b, *w_fc1, *b_fc1, *w_fc2, *b_fc2;
+} vit_layer_weights;
+
+/* Packed variable-length sequences (images).  Tokens of sequence s are rows
+ * cu_seqlens[s] .. cu_seqlens[s+1]-1; attention never crosses sequences
+ * (block-diagonal mask).  pos_rc[t] = (row, col) of token t in its image
+ * grid (NULL: no RoPE).  prefix_kv, if not NULL, holds per sequence P keys
+ * and values used as given (no RoPE) in front of the sequence's own keys:
+ * layout [n_seqs, 2 (K then V), prefix_len, kv_heads, head_dim]; query head h
+ * reads prefix head h / (heads / kv_heads). */
+typedef struct {
+  int total_tokens;            /* T = cu_seqlens[n_seqs]                     */
+  int n_seqs;                  /* >= 1                                       */
+  int max_seqlen;              /* >= every sequence length                   */
+  const int32_t *cu_seqlens;   /* device [n_seqs + 1], cu_seqlens[0] = 0     */
+  const int32_t *pos_rc;       /* device [T, 2] or NULL                      */
+  const void *prefix_kv;       /* device, see above, or NULL                 */
+  int prefix_len;              /* P (0 when prefix_kv is NULL)               */
+  int kv_heads;                /* heads of prefix_kv (0 means = heads)       */
+} vit_seqs;
+
+typedef struct vit_ctx vit_ctx;
+
+/* Creates a context for one device.  Checks that the device is sm_100,
+ * validates cfg (hidden = heads*head_dim, head_dim in {64,72,128} with 64
+ * fp32-only, mlp > 0 unless VIT_FLAG_NO_MLP) and allocates the 16-byte
+ * device status word.  *out receives the context (NULL on error). */
+VIT_API vit_status vit_init(const vit_config *cfg, int device, vit_ctx **out);
+
+/* Frees the context and its status word.  NULL is ignored. */
+VIT_API void vit_destroy(vit_ctx *ctx);
+
+/* Bytes of device workspace vit_layer_forward / vit_encoder_forward need for
+ * total_tokens tokens (256-byte aligned base required). */
+VIT_API size_t vit_workspace_bytes(const vit_ctx *ctx, int total_tokens);
+
+/* One pre-LN encoder layer (reading: x1 = x + Wo Attn(RoPE(Wqkv LN1(x))) + bo;
+ * y = x1 + W2 GELU(W1 LN2(x1) + b1) + b2).  x, y: [T, C]; y may not alias x.
+ * With VIT_FLAG_NO_MLP y = x1 (DiT-style attention half-layer). */
+VIT_API vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w,
+                             const void *x, void *y, const vit_seqs *seqs,
+                             void *workspace, size_t ws_bytes, void *stream);
+
+/* The stack of n_layers layers; layers is a HOST array of n_layers weight
+ * structs (device pointers inside).  Intermediate activations live in the
+ * workspace; x is read only; y [T, C] receives the last layer's output. */
+VIT_API vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers,
+                               int n_layers, const void *x, void *y,
+                               const vit_seqs *seqs, void *workspace,
+                               size_t ws_bytes, void *stream);
+
+/* Bidirectional multi-head attention over packed sequences ("视觉算子":
+ * softmax(Q K^T * scale) V per head and sequence).  qkv [T, 3, H, d]
+ * (the QKV projection's output layout), o [T, H, d].  With seqs->pos_rc the
+ * kernel rotates Q and K by 2D RoPE as it loads them.  scale <= 0 selects
+ * 1/sqrt(d). */
+VIT_API vit_status vit_attention(vit_ctx *ctx, const void *qkv, void *o,
+                         const vit_seqs *seqs, float scale, void *stream);
+
+/* 2x2 spatial merge (intro bullet: Projector, 2x2 spatial merge).  Per image
+ * with grid (rows, cols), both even: output token (R, Q) = concat of input
+ * tokens (2R,2Q), (2R,2Q+1), (2R+1,2Q), (2R+1,2Q+1).  x [T, channels],
+ * y [T/4, 4*channels]; images packed in order.  grids_hw_host: HOST int32
+ * [n_images, 2] = (rows, cols).  Odd sides -> VIT_ERR_SHAPE.  Bit-exact. */
+VIT_API vit_status vit_spatial_merge_2x2(vit_ctx *ctx, const void *x, void *y,
+                                 const int32_t *grids_hw_host, int n_images,
+                                 int channels, void *stream);
+
+/* Writes cu_seqlens [n_images+1] and pos_rc [T, 2] (row-major tokens,
+ * positions restarting at (0,0) per image) for packed image grids given on
+ * the HOST ([n_images, 2] = rows, cols; n_images <= 1024). */
+VIT_API vit_status vit_positions_from_grids(vit_ctx *ctx, const int32_t *grids_hw_host,
+                                    int n_images, int32_t *cu_seqlens,
+                                    int32_t *pos_rc, void *stream);
+
+/* ---- single steps of the layer, exposed for step-level use and testing --- */
+
+/* LayerNorm over the last axis ("视觉算子": LayerNorm), biased variance,
+ * y = (x - mean)/sqrt(var + eps) * gamma + beta.  x, y [rows, cols];
+ * y may alias x. */
+VIT_API vit_status vit_layernorm(vit_ctx *ctx, const void *x, void *y,
+                         const void *gamma, const void *beta, int rows,
+                         int cols, float eps, void *stream);
+
+/* Epilogues of vit_linear */
+typedef enum {
+  VIT_EPI_BIAS = 0,           /* y = x W^T + b                               */
+  VIT_EPI_BIAS_GELU = 1,      /* y = GELU_tanh(x W^T + b)                    */
+  VIT_EPI_BIAS_RESIDUAL = 2   /* y = residual + x W^T + b (residual [M, N])  */
+} vit_epilogue;
+
+/* GEMM + bias with a fused epilogue ("视觉算子": GEMM + bias).  x [M, K],
+ * w [N, K], bias [N] (may be NULL), residual [M, N] for
+ * VIT_EPI_BIAS_RESIDUAL, y [M, N].  bf16: K and N multiples of 8. */
+VIT_API vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w,
+                      const void *bias, const void *residual, void *y, int M,
+                      int N, int K, vit_epilogue epi, void *stream);
+
+/* 2D RoPE in place on the Q and K parts of qkv [T, 3, H, d] (intro bullet
+ * "2D RoPE"): dims [0, d/2) rotate by row, [d/2, d) by column; within a
+ * half of width h, dim j pairs with j + h/2 at frequency
+ * theta^(-2j/h). */
+VIT_API vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc,
+                      int total_tokens, void *stream);
+
+/* ---- status ---- */
+
+/* Synchronises the device, reads the context's device status word, clears
+ * it and returns VIT_OK, VIT_ERR_TIMEOUT or VIT_ERR_DEVICE_BOUNDS (or
+ * VIT_ERR_CUDA when the device reports an error). */
+VIT_API vit_status vit_get_last_device_status(vit_ctx *ctx);
+
+/* Static string for a status code. */
+VIT_API const char *vit_status_string(vit_status s);
+
+/* Library version string, e.g. "libvit 0.1 sm_100a". */
+VIT_API const char *vit_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VIT_H_ */

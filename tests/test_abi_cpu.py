@@ -1,0 +1,79 @@
+"""Host-only checks of the C ABI library: it loads, exports every entry point
+declared in include/vit.h, and rejects bad arguments without touching a GPU.
+No compute call is made here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vit.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"VIT_API\s+[\w\s\*]+?\b(vit_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ("vit_init", "vit_destroy", "vit_workspace_bytes", "vit_layer_forward",
+                 "vit_encoder_forward", "vit_attention", "vit_spatial_merge_2x2",
+                 "vit_positions_from_grids", "vit_get_last_device_status", "vit_status_string"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol():
+    import vision_transformer_encoder_layernorm_b200 as vit
+    out = subprocess.run(["nm", "-D", "--defined-only", vit.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (vit_\w+)", out))
+    declared = set(header_functions())
+    assert declared <= exported, declared - exported
+    assert set(vit.ABI_FUNCTIONS) == declared
+
+
+def test_status_strings_and_version():
+    import vision_transformer_encoder_layernorm_b200 as vit
+    for code, name in vit.STATUS.items():
+        assert vit.lib.vit_status_string(code).decode() == name
+    assert vit.lib.vit_status_string(99).decode() == "VIT_ERR_UNKNOWN"
+    assert b"sm_100a" in vit.lib.vit_version()
+
+
+def test_null_arguments_rejected_without_gpu():
+    import vision_transformer_encoder_layernorm_b200 as vit
+    L = vit.lib
+    assert L.vit_init(None, 0, None) == 1
+    h = ctypes.c_void_p()
+    assert L.vit_init(None, 0, ctypes.byref(h)) == 1 and not h.value
+    bad = vit.VitConfig(100, 3, 72, 512, 1e-6, 1e4, vit.BF16, 0)    # 3*72 != 100
+    assert L.vit_init(ctypes.byref(bad), 0, ctypes.byref(h)) == 2
+    bad = vit.VitConfig(256, 4, 64, 1024, 1e-6, 1e4, vit.BF16, 0)   # d=64 is fp32-only
+    assert L.vit_init(ctypes.byref(bad), 0, ctypes.byref(h)) == 3
+    bad = vit.VitConfig(1152, 16, 72, 4304, 1e-6, 1e4, 7, 0)        # bad dtype
+    assert L.vit_init(ctypes.byref(bad), 0, ctypes.byref(h)) == 1
+    L.vit_destroy(None)
+    assert L.vit_workspace_bytes(None, 10) == 0
+    assert L.vit_layer_forward(None, None, None, None, None, None, 0, None) == 1
+    assert L.vit_encoder_forward(None, None, 1, None, None, None, None, 0, None) == 1
+    assert L.vit_attention(None, None, None, None, 0.0, None) == 1
+    assert L.vit_spatial_merge_2x2(None, None, None, None, 0, 0, None) == 1
+    assert L.vit_positions_from_grids(None, None, 0, None, None, None) == 1
+    assert L.vit_layernorm(None, None, None, None, None, 0, 0, 0.0, None) == 1
+    assert L.vit_linear(None, None, None, None, None, None, 0, 0, 0, 0, None) == 1
+    assert L.vit_rope2d(None, None, None, 0, None) == 1
+    assert L.vit_get_last_device_status(None) == 1
+
+
+def test_init_without_device_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    import vision_transformer_encoder_layernorm_b200 as vit
+    cfg = vit.VitConfig(1152, 16, 72, 4304, 1e-6, 1e4, vit.BF16, 0)
+    h = ctypes.c_void_p()
+    assert vit.lib.vit_init(ctypes.byref(cfg), 0, ctypes.byref(h)) == 5
+    assert not h.value

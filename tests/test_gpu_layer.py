@@ -1,0 +1,183 @@
+"""Layer- and stack-level parity of the CUDA path against the fp64 oracle on
+the seeded workloads, through the C ABI, plus boundary behaviour on a GPU
+(errors before any launch, outputs untouched)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import run as orun
+from oracle import vit_ref as R
+from tests.gpu_util import assert_close, context_for, from_dev, int_dev, layer_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+vit = pytest.importorskip("vision_transformer_encoder_layernorm_b200")
+
+
+def _device_run(wl, inputs, n_layers=None, merge=None):
+    """Runs the workload's stack (and merge) on the GPU; returns fp64 numpy."""
+    ctx = context_for(wl)
+    T, C = wl.tokens, wl.hidden
+    cu_r, pos_r = R.positions_from_grids(wl.grids)
+    cu = torch.empty(len(wl.grids) + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+    ctx.positions_from_grids(wl.grids, cu, pos)
+    x = to_dev(inputs.x, wl.dtype)
+    pkv = None if inputs.prefix_kv is None else to_dev(inputs.prefix_kv, wl.dtype)
+    sq = vit.seqs(T, len(wl.grids), int(max(h * w for h, w in wl.grids)), cu,
+                  pos if wl.rope else None, pkv, wl.prefix_len, wl.prefix_heads)
+    n = len(inputs.layers) if n_layers is None else n_layers
+    layers = [layer_dev(inputs, i) for i in range(n)]
+    ws = torch.empty(ctx.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(x)
+    ctx.encoder_forward(layers, x, y, sq, ws)
+    out = y
+    if merge if merge is not None else wl.merge:
+        out = torch.empty((T // 4, 4 * C), dtype=x.dtype, device="cuda")
+        ctx.spatial_merge_2x2(y, out, wl.grids, C)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    res = from_dev(out)
+    ctx.close()
+    return res
+
+
+def test_c0_fp32_layer_and_merge():
+    wl = synth.get("c0")
+    inp = synth.make_inputs(wl)
+    got = _device_run(wl, inp)
+    ref = orun.run_workload(inp)
+    assert got.shape == (64, 1024)
+    assert_close(got, ref, 1e-4, None, "c0 fp32")
+
+
+def test_c1_bf16_layer():
+    wl = synth.get("c1")
+    inp = synth.make_inputs(wl)
+    got = _device_run(wl, inp)
+    ref = orun.run_workload(inp)
+    assert_close(got, ref, 2e-2, 0.9999, "c1 layer")
+
+
+def test_small_stack_bf16():
+    # 4 layers, two images with ragged tiles, hidden 288 (4 x 72)
+    wl = synth.Workload("t", 7, "bf16", 288, 4, 72, 640, 4, ((13, 11), (6, 30)))
+    inp = synth.make_inputs(wl)
+    got = _device_run(wl, inp)
+    ref = orun.run_workload(inp)
+    assert_close(got, ref, 5e-2, 0.999, "small stack")
+
+
+def test_small_stack_d128_prefix_no_mlp():
+    wl = synth.Workload("t", 8, "bf16", 256, 2, 128, 0, 2, ((10, 20), (7, 9)),
+                        prefix_len=150, kv_heads=1, attn_only=True)
+    inp = synth.make_inputs(wl)
+    got = _device_run(wl, inp)
+    ref = orun.run_workload(inp)
+    assert_close(got, ref, 5e-2, 0.999, "attention-only stack")
+
+
+def test_encoder_one_layer_equals_layer_forward():
+    wl = synth.get("c1")
+    inp = synth.make_inputs(wl)
+    ctx = context_for(wl)
+    T = wl.tokens
+    cu = int_dev(R.positions_from_grids(wl.grids)[0])
+    pos = int_dev(R.positions_from_grids(wl.grids)[1])
+    sq = vit.seqs(T, 1, T, cu, pos)
+    x = to_dev(inp.x, wl.dtype)
+    ws = torch.empty(ctx.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    y1, y2 = torch.empty_like(x), torch.empty_like(x)
+    lw = layer_dev(inp, 0)
+    ctx.layer_forward(lw, x, y1, sq, ws)
+    ctx.encoder_forward([lw], x, y2, sq, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    ctx.close()
+
+
+@pytest.mark.slow
+def test_c4_attention_half_layer():
+    wl = synth.get("c4")
+    inp = synth.make_inputs(wl)
+    got = _device_run(wl, inp)
+    ref = orun.run_workload(inp)
+    assert_close(got, ref, 2e-2, 0.9999, "c4 attention half-layer")
+
+
+@pytest.mark.slow
+def test_c3_first_layer_full_size():
+    wl = synth.get("c3")
+    inp = synth.make_inputs(wl, layers=1)
+    got = _device_run(wl, inp, n_layers=1)
+    ref = orun.run_layers(inp, n_layers=1)
+    assert_close(got, ref, 2e-2, 0.9999, "c3 layer 0")
+
+
+@pytest.mark.slow
+def test_c2_full_stack_and_merge():
+    # the headline workload: 27 layers over 3900 tokens, then the 2x2 merge
+    wl = synth.get("c2")
+    inp = synth.make_inputs(wl)
+    got = _device_run(wl, inp)
+    ref = orun.run_workload(inp)
+    assert got.shape == (975, 4608)
+    assert_close(got, ref, 1.0, 0.999, "c2 27-layer stack + merge")
+
+
+# ------------------------------------------------------------------ boundary
+def test_boundary_errors_launch_nothing():
+    wl = synth.get("c1")
+    ctx = context_for(wl)
+    T, C = wl.tokens, wl.hidden
+    cu = int_dev(np.array([0, T]))
+    pos = int_dev(R.positions_from_grids(wl.grids)[1])
+    x = torch.zeros((T, C), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((T, C), 5.0, dtype=torch.bfloat16, device="cuda")
+    inp = synth.make_inputs(wl)
+    lw = layer_dev(inp, 0)
+    need = ctx.workspace_bytes(T)
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    sq = vit.seqs(T, 1, T, cu, pos)
+    cases = [
+        (lambda: ctx.layer_forward(lw, x, y, sq, small), 4),                      # workspace
+        (lambda: ctx.layer_forward(lw, x, x, sq, ws), 1),                         # aliasing
+        (lambda: ctx.layer_forward(lw, x, y, vit.seqs(T, 1, T + 1, cu, pos), ws), 2),
+        (lambda: ctx.layer_forward(lw, x, y, vit.seqs(T, 1, T, cu, None), ws), 1),  # no pos
+        (lambda: ctx.layer_forward(dict(lw, w_o=None), x, y, sq, ws), 1),
+        (lambda: ctx.attention(x[:, :3 * 8], y, vit.seqs(T, 1, T, cu, None, x, 4, 3)), 2),
+        (lambda: ctx.linear(x[:, :12], x[:12, :12], None, y), 3),               # K % 8
+    ]
+    for fn, code in cases:
+        with pytest.raises(vit.VitError) as e:
+            fn()
+        assert e.value.code == code
+    torch.cuda.synchronize()
+    assert torch.all(y == 5.0)
+    ctx.close()
+
+
+def test_unsupported_configs_rejected():
+    with pytest.raises(vit.VitError) as e:
+        vit.Context(96 * 4, 4, 96, 512, vit.BF16)
+    assert e.value.code == 3
+    with pytest.raises(vit.VitError) as e:
+        vit.Context(256, 4, 64, 1024, vit.BF16)
+    assert e.value.code == 3
+
+
+def test_empty_input_is_a_no_op():
+    wl = synth.get("c1")
+    ctx = context_for(wl)
+    x = torch.zeros((0, wl.hidden), dtype=torch.bfloat16, device="cuda")
+    cu = int_dev(np.array([0, 0]))
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    ctx.layer_forward(layer_dev(synth.make_inputs(wl), 0), x, torch.empty_like(x),
+                      vit.seqs(0, 1, 0, cu, cu), ws)
+    ctx.attention(torch.zeros((0, 3 * wl.hidden), dtype=torch.bfloat16, device="cuda"), x,
+                  vit.seqs(0, 1, 0, cu))
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    ctx.close()

@@ -1,0 +1,211 @@
+"""Python binding of libvit (include/vit.h): a B200 (sm_100a) implementation
+of the vision-transformer encoder hot path -- pre-LN layers of LayerNorm,
+QKV GEMM + bias, 2D RoPE, bidirectional varlen attention (optional prefix
+K/V), output projection + residual and a GELU-tanh MLP, then the 2x2 spatial
+merge.
+
+This module only marshals arguments: every step runs in the CUDA kernels of
+``libvit.so``.  There is no fallback; importing fails loudly when the library
+has not been built (``python -m vision_transformer_encoder_layernorm_b200.build``).
+Tensors are PyTorch tensors (device memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+__all__ = [
+    "lib", "LIB_PATH", "VitError", "VitConfig", "VitLayerWeights", "VitSeqs", "Context",
+    "F32", "BF16", "FLAG_NO_ROPE", "FLAG_NO_MLP", "EPI_BIAS", "EPI_BIAS_GELU",
+    "EPI_BIAS_RESIDUAL", "STATUS", "ABI_FUNCTIONS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvit.so")
+
+F32, BF16 = 0, 1
+FLAG_NO_ROPE, FLAG_NO_MLP = 0x1, 0x2
+EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_RESIDUAL = 0, 1, 2
+STATUS = {0: "VIT_OK", 1: "VIT_ERR_INVALID_ARG", 2: "VIT_ERR_SHAPE", 3: "VIT_ERR_UNSUPPORTED",
+          4: "VIT_ERR_WORKSPACE", 5: "VIT_ERR_CUDA", 6: "VIT_ERR_TIMEOUT",
+          7: "VIT_ERR_DEVICE_BOUNDS"}
+
+
+class VitError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} -> {STATUS.get(code, code)}")
+        self.code = code
+
+
+class VitConfig(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("mlp", ctypes.c_int), ("ln_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("dtype", ctypes.c_int), ("flags", ctypes.c_uint)]
+
+
+_WKEYS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
+          "ln2_g", "ln2_b", "w_fc1", "b_fc1", "w_fc2", "b_fc2")
+
+
+class VitLayerWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in _WKEYS]
+
+
+class VitSeqs(ctypes.Structure):
+    _fields_ = [("total_tokens", ctypes.c_int), ("n_seqs", ctypes.c_int),
+                ("max_seqlen", ctypes.c_int), ("cu_seqlens", ctypes.c_void_p),
+                ("pos_rc", ctypes.c_void_p), ("prefix_kv", ctypes.c_void_p),
+                ("prefix_len", ctypes.c_int), ("kv_heads", ctypes.c_int)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+# name -> (restype, argtypes); the exported C ABI of include/vit.h
+ABI_FUNCTIONS = {
+    "vit_init": (_I, [ctypes.POINTER(VitConfig), _I, ctypes.POINTER(_P)]),
+    "vit_destroy": (None, [_P]),
+    "vit_workspace_bytes": (ctypes.c_size_t, [_P, _I]),
+    "vit_layer_forward": (_I, [_P, ctypes.POINTER(VitLayerWeights), _P, _P,
+                               ctypes.POINTER(VitSeqs), _P, ctypes.c_size_t, _P]),
+    "vit_encoder_forward": (_I, [_P, ctypes.POINTER(VitLayerWeights), _I, _P, _P,
+                                 ctypes.POINTER(VitSeqs), _P, ctypes.c_size_t, _P]),
+    "vit_attention": (_I, [_P, _P, _P, ctypes.POINTER(VitSeqs), ctypes.c_float, _P]),
+    "vit_spatial_merge_2x2": (_I, [_P, _P, _P, ctypes.POINTER(ctypes.c_int32), _I, _I, _P]),
+    "vit_positions_from_grids": (_I, [_P, ctypes.POINTER(ctypes.c_int32), _I, _P, _P, _P]),
+    "vit_layernorm": (_I, [_P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P]),
+    "vit_linear": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "vit_rope2d": (_I, [_P, _P, _P, _I, _P]),
+    "vit_get_last_device_status": (_I, [_P]),
+    "vit_status_string": (ctypes.c_char_p, [_I]),
+    "vit_version": (ctypes.c_char_p, []),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m vision_transformer_encoder_layernorm_b200.build` (nvcc, sm_100a)")
+    h = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in ABI_FUNCTIONS.items():
+        fn = getattr(h, name)
+        fn.restype = res
+        fn.argtypes = args
+    return h
+
+
+lib = _load()
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise VitError(fn, code)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _grids_arr(grids: Sequence[Sequence[int]]):
+    flat = [int(v) for g in grids for v in g]
+    return (ctypes.c_int32 * len(flat))(*flat), len(grids)
+
+
+def layer_weights(d) -> VitLayerWeights:
+    """A VitLayerWeights from a mapping of the 12 parameter names to tensors
+    (missing or None entries become NULL)."""
+    return VitLayerWeights(*[_ptr(d.get(k)) for k in _WKEYS])
+
+
+def seqs(total_tokens: int, n_seqs: int, max_seqlen: int, cu_seqlens, pos_rc=None,
+         prefix_kv=None, prefix_len: int = 0, kv_heads: int = 0) -> VitSeqs:
+    return VitSeqs(total_tokens, n_seqs, max_seqlen, _ptr(cu_seqlens), _ptr(pos_rc),
+                   _ptr(prefix_kv), prefix_len if prefix_kv is not None else 0, kv_heads)
+
+
+class Context:
+    """Owns one ``vit_ctx``; each method is the C entry point of the same name
+    (without the ``vit_`` prefix) with tensors in place of pointers."""
+
+    def __init__(self, hidden, heads, head_dim, mlp, dtype=BF16, ln_eps=1e-6,
+                 rope_theta=10000.0, flags=0, device=0):
+        self.cfg = VitConfig(hidden, heads, head_dim, mlp, ln_eps, rope_theta, dtype, flags)
+        h = ctypes.c_void_p()
+        _check("vit_init", lib.vit_init(ctypes.byref(self.cfg), device, ctypes.byref(h)))
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.vit_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, total_tokens: int) -> int:
+        return lib.vit_workspace_bytes(self._h, total_tokens)
+
+    def layer_forward(self, weights, x, y, sq: VitSeqs, workspace, stream=None):
+        lw = layer_weights(weights) if not isinstance(weights, VitLayerWeights) else weights
+        _check("vit_layer_forward", lib.vit_layer_forward(
+            self._h, ctypes.byref(lw), _ptr(x), _ptr(y), ctypes.byref(sq), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream)))
+
+    def encoder_forward(self, layers, x, y, sq: VitSeqs, workspace, stream=None):
+        arr = (VitLayerWeights * len(layers))(
+            *[l if isinstance(l, VitLayerWeights) else layer_weights(l) for l in layers])
+        _check("vit_encoder_forward", lib.vit_encoder_forward(
+            self._h, arr, len(layers), _ptr(x), _ptr(y), ctypes.byref(sq), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream)))
+
+    def attention(self, qkv, o, sq: VitSeqs, scale: float = 0.0, stream=None):
+        _check("vit_attention", lib.vit_attention(self._h, _ptr(qkv), _ptr(o), ctypes.byref(sq),
+                                                  scale, _stream(stream)))
+
+    def spatial_merge_2x2(self, x, y, grids, channels: int, stream=None):
+        arr, n = _grids_arr(grids)
+        _check("vit_spatial_merge_2x2", lib.vit_spatial_merge_2x2(
+            self._h, _ptr(x), _ptr(y), arr, n, channels, _stream(stream)))
+
+    def positions_from_grids(self, grids, cu_seqlens, pos_rc, stream=None):
+        arr, n = _grids_arr(grids)
+        _check("vit_positions_from_grids", lib.vit_positions_from_grids(
+            self._h, arr, n, _ptr(cu_seqlens), _ptr(pos_rc), _stream(stream)))
+
+    def layernorm(self, x, y, gamma, beta, eps: float = 1e-6, stream=None):
+        rows, cols = x.shape
+        _check("vit_layernorm", lib.vit_layernorm(self._h, _ptr(x), _ptr(y), _ptr(gamma),
+                                                  _ptr(beta), rows, cols, eps, _stream(stream)))
+
+    def linear(self, x, w, bias, y, epi=EPI_BIAS, residual=None, stream=None):
+        M, K = x.shape
+        N = w.shape[0]
+        _check("vit_linear", lib.vit_linear(self._h, _ptr(x), _ptr(w), _ptr(bias), _ptr(residual),
+                                            _ptr(y), M, N, K, epi, _stream(stream)))
+
+    def rope2d(self, qkv, pos_rc, stream=None):
+        _check("vit_rope2d", lib.vit_rope2d(self._h, _ptr(qkv), _ptr(pos_rc), qkv.shape[0],
+                                            _stream(stream)))
+
+    def device_status(self) -> int:
+        return lib.vit_get_last_device_status(self._h)

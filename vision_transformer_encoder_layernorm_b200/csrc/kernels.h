@@ -1,0 +1,86 @@
+// kernels.h -- launchers of libvit's kernels (internal; the public ABI is
+// include/vit.h).  Every launcher enqueues on the given stream and returns
+// the launch status; argument validation happens in vit_api.cu.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace vit {
+
+constexpr int kF32 = 0;
+constexpr int kBF16 = 1;
+
+// Per-image table passed by value (__grid_constant__) to the merge and
+// positions kernels; a call covers at most kMaxImagesPerLaunch images.
+constexpr int kMaxImagesPerLaunch = 256;
+struct ImageEntry {
+  int rows, cols;
+  int base;  // first token of the image in the packed sequence
+};
+struct ImageTable {
+  ImageEntry img[kMaxImagesPerLaunch];
+};
+
+// Rotation frequencies divided by pi, wpi[j] = theta^(-2j/h) / pi for
+// j < d/4, h = d/2 (computed on the host in fp64).  Kernels evaluate the
+// rotation as sincospif(p * wpi[j]), whose argument reduction is exact.
+struct RopeFreqs {
+  float wpi[32];
+};
+
+// Sequence description shared by the attention kernels.
+struct SeqArgs {
+  int total_tokens, n_seqs, max_seqlen;
+  const int32_t *cu_seqlens;
+  const int32_t *pos;      // [T, 2] or null
+  const void *prefix_kv;   // [S, 2, P, Hkv, d] or null
+  int prefix_len, kv_heads;
+};
+
+cudaError_t launch_layernorm(int dtype, const void *x, void *y, const void *g, const void *b,
+                             int rows, int cols, float eps, cudaStream_t st);
+cudaError_t launch_merge2x2(const ImageTable &tab, int n_images, const void *x, void *y,
+                            size_t row_bytes, long long max_out_tokens, cudaStream_t st);
+cudaError_t launch_positions(const ImageTable &tab, int n_images, int cu_offset_index,
+                             int max_tokens, int32_t *cu, int32_t *pos, cudaStream_t st);
+cudaError_t launch_rope2d(int dtype, void *qkv, const int32_t *pos, int T, int H, int d,
+                          const RopeFreqs &fr, cudaStream_t st);
+
+// Epilogue codes (match vit_epilogue)
+constexpr int kEpiBias = 0;
+constexpr int kEpiGelu = 1;
+constexpr int kEpiResidual = 2;
+
+// SIMT GEMM (fp32 FFMA; fp32 or bf16 storage): y = epi(x w^T + b).
+cudaError_t launch_gemm_simt(int dtype, const void *x, const void *w, const void *b,
+                             const void *res, void *y, int M, int N, int K, int epi,
+                             cudaStream_t st);
+
+// SIMT attention (fp32 math; fp32 or bf16 storage).
+cudaError_t launch_attention_simt(int dtype, const void *qkv, void *o, const SeqArgs &s, int H,
+                                  int d, float scale, const RopeFreqs &fr, int *status,
+                                  cudaStream_t st);
+
+// tcgen05 GEMM, bf16 in / bf16 out, fp32 accumulation in TMEM.
+struct GemmPlan;
+cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
+                           int M, int N, int K, int epi, int num_sms, int *status,
+                           cudaStream_t st);
+
+// tcgen05 flash attention, bf16, head_dim 72 or 128.
+cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,
+                                float scale, const RopeFreqs &fr, int num_sms, int *status,
+                                cudaStream_t st);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once).
+CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
+                              uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
+                              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+}  // namespace vit

@@ -1,0 +1,432 @@
+// vit_api.cu -- the C ABI of include/vit.h: argument validation (always
+// before any launch), workspace carving, and the order of kernel launches for
+// one encoder layer and for the stack.
+//
+// Layer (pre-LN reading of the KLiteInfer README, "视觉算子" op list):
+//   h  = LN1(x)                      layernorm kernel
+//   qkv = h Wqkv^T + bqkv            GEMM (bias epilogue)
+//   qkv[Q,K] = RoPE2D(qkv[Q,K])      rope kernel, in place (workspace)
+//   a  = Attn(qkv)                   attention kernel (varlen, prefix)
+//   x1 = x + a Wo^T + bo             GEMM (bias + residual epilogue)
+//   h  = LN2(x1)                     layernorm kernel
+//   g  = GELU(h W1^T + b1)           GEMM (bias + GELU epilogue)
+//   y  = x1 + g W2^T + b2            GEMM (bias + residual epilogue)
+// bf16 runs the tcgen05 GEMM / attention kernels, fp32 the SIMT ones.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/vit.h"
+#include "kernels.h"
+
+struct vit_ctx {
+  vit_config cfg;
+  int device;
+  int num_sms;
+  int *d_status;  // 4 ints; [0] = first error code recorded by a kernel
+  vit::RopeFreqs fr;
+};
+
+namespace {
+
+using namespace vit;
+
+struct DeviceGuard {
+  int prev = -1;
+  bool changed = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+      changed = cudaSetDevice(dev) == cudaSuccess;
+    }
+  }
+  ~DeviceGuard() {
+    if (changed) cudaSetDevice(prev);
+  }
+};
+
+inline size_t esize(const vit_config &c) { return c.dtype == VIT_F32 ? 4 : 2; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+vit_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VIT_OK : VIT_ERR_CUDA; }
+
+vit_status check_seqs(const vit_ctx *ctx, const vit_seqs *s, bool allow_prefix) {
+  if (!s) return VIT_ERR_INVALID_ARG;
+  if (s->total_tokens < 0 || s->n_seqs < 1 || s->max_seqlen < 0) return VIT_ERR_INVALID_ARG;
+  if (s->total_tokens > 0 && (!s->cu_seqlens || s->max_seqlen < 1)) return VIT_ERR_INVALID_ARG;
+  if (s->max_seqlen > s->total_tokens) return VIT_ERR_SHAPE;
+  if (s->prefix_kv) {
+    if (!allow_prefix) return VIT_ERR_INVALID_ARG;
+    if (s->prefix_len <= 0) return VIT_ERR_SHAPE;
+    const int hkv = s->kv_heads > 0 ? s->kv_heads : ctx->cfg.heads;
+    if (hkv > ctx->cfg.heads || ctx->cfg.heads % hkv) return VIT_ERR_SHAPE;
+    if (ctx->cfg.dtype == VIT_BF16 && !aligned16(s->prefix_kv)) return VIT_ERR_INVALID_ARG;
+  } else if (s->prefix_len != 0) {
+    return VIT_ERR_INVALID_ARG;
+  }
+  return VIT_OK;
+}
+
+SeqArgs to_seq_args(const vit_seqs *s, bool with_pos) {
+  SeqArgs a;
+  a.total_tokens = s->total_tokens;
+  a.n_seqs = s->n_seqs;
+  a.max_seqlen = s->max_seqlen;
+  a.cu_seqlens = s->cu_seqlens;
+  a.pos = with_pos ? s->pos_rc : nullptr;
+  a.prefix_kv = s->prefix_kv;
+  a.prefix_len = s->prefix_kv ? s->prefix_len : 0;
+  a.kv_heads = s->kv_heads;
+  return a;
+}
+
+cudaError_t run_linear(vit_ctx *ctx, const void *x, const void *w, const void *b,
+                       const void *res, void *y, int M, int N, int K, int epi, cudaStream_t st) {
+  if (ctx->cfg.dtype == VIT_F32) return launch_gemm_simt(kF32, x, w, b, res, y, M, N, K, epi, st);
+  return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st);
+}
+
+cudaError_t run_attention(vit_ctx *ctx, const void *qkv, void *o, const SeqArgs &s, float scale,
+                          cudaStream_t st) {
+  const vit_config &c = ctx->cfg;
+  if (c.dtype == VIT_F32)
+    return launch_attention_simt(kF32, qkv, o, s, c.heads, c.head_dim, scale, ctx->fr,
+                                 ctx->d_status, st);
+  return launch_attention_tc(qkv, o, s, c.heads, c.head_dim, scale, ctx->fr, ctx->num_sms,
+                             ctx->d_status, st);
+}
+
+struct Workspace {
+  void *h, *qkv, *attn, *x1, *g, *act[2];
+};
+
+size_t workspace_layout(const vit_config &c, int T, Workspace *w, void *base) {
+  const size_t es = esize(c);
+  const size_t C = size_t(c.hidden);
+  const size_t F = (c.flags & VIT_FLAG_NO_MLP) ? 0 : size_t(c.mlp);
+  const size_t sizes[7] = {T * C * es, T * 3 * C * es, T * C * es, T * C * es,
+                           T * F * es, T * C * es, T * C * es};
+  size_t off = 0;
+  void **slots[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  if (w) {
+    slots[0] = &w->h; slots[1] = &w->qkv; slots[2] = &w->attn; slots[3] = &w->x1;
+    slots[4] = &w->g; slots[5] = &w->act[0]; slots[6] = &w->act[1];
+  }
+  for (int i = 0; i < 7; ++i) {
+    if (w) *slots[i] = static_cast<char *>(base) + off;
+    off += align256(sizes[i]);
+  }
+  return off;
+}
+
+vit_status check_layer_weights(const vit_config &c, const vit_layer_weights *w) {
+  if (!w) return VIT_ERR_INVALID_ARG;
+  const void *need[6] = {w->ln1_g, w->ln1_b, w->w_qkv, w->b_qkv, w->w_o, w->b_o};
+  for (const void *p : need)
+    if (!p || (c.dtype == VIT_BF16 && !aligned16(p))) return VIT_ERR_INVALID_ARG;
+  if (!(c.flags & VIT_FLAG_NO_MLP)) {
+    const void *mlp[6] = {w->ln2_g, w->ln2_b, w->w_fc1, w->b_fc1, w->w_fc2, w->b_fc2};
+    for (const void *p : mlp)
+      if (!p || (c.dtype == VIT_BF16 && !aligned16(p))) return VIT_ERR_INVALID_ARG;
+  }
+  return VIT_OK;
+}
+
+// One layer; all arguments already validated.
+vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, void *y,
+                      const vit_seqs *seqs, const Workspace &ws, cudaStream_t st) {
+  const vit_config &c = ctx->cfg;
+  const int T = seqs->total_tokens, C = c.hidden, F = c.mlp;
+  const int dt = c.dtype == VIT_F32 ? kF32 : kBF16;
+  const bool rope = !(c.flags & VIT_FLAG_NO_ROPE) && seqs->pos_rc != nullptr;
+  const float scale = 1.0f / sqrtf(float(c.head_dim));
+  cudaError_t e = cudaSuccess;
+  (void)e;
+  if ((e = launch_layernorm(dt, x, ws.h, w->ln1_g, w->ln1_b, T, C, c.ln_eps, st))) return VIT_ERR_CUDA;
+  if ((e = run_linear(ctx, ws.h, w->w_qkv, w->b_qkv, nullptr, ws.qkv, T, 3 * C, C, kEpiBias, st)))
+    return VIT_ERR_CUDA;
+  if (rope && (e = launch_rope2d(dt, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st)))
+    return VIT_ERR_CUDA;
+  const SeqArgs sa = to_seq_args(seqs, false);
+  if ((e = run_attention(ctx, ws.qkv, ws.attn, sa, scale, st))) return VIT_ERR_CUDA;
+  if (c.flags & VIT_FLAG_NO_MLP) {
+    if ((e = run_linear(ctx, ws.attn, w->w_o, w->b_o, x, y, T, C, C, kEpiResidual, st)))
+      return VIT_ERR_CUDA;
+    return VIT_OK;
+  }
+  if ((e = run_linear(ctx, ws.attn, w->w_o, w->b_o, x, ws.x1, T, C, C, kEpiResidual, st)))
+    return VIT_ERR_CUDA;
+  if ((e = launch_layernorm(dt, ws.x1, ws.h, w->ln2_g, w->ln2_b, T, C, c.ln_eps, st)))
+    return VIT_ERR_CUDA;
+  if ((e = run_linear(ctx, ws.h, w->w_fc1, w->b_fc1, nullptr, ws.g, T, F, C, kEpiGelu, st)))
+    return VIT_ERR_CUDA;
+  if ((e = run_linear(ctx, ws.g, w->w_fc2, w->b_fc2, ws.x1, y, T, C, F, kEpiResidual, st)))
+    return VIT_ERR_CUDA;
+  return VIT_OK;
+}
+
+vit_status check_layer_call(vit_ctx *ctx, const void *x, void *y, const vit_seqs *seqs,
+                            void *workspace, size_t ws_bytes) {
+  if (!ctx || !x || !y) return VIT_ERR_INVALID_ARG;
+  vit_status s = check_seqs(ctx, seqs, true);
+  if (s != VIT_OK) return s;
+  if (x == y) return VIT_ERR_INVALID_ARG;
+  if (ctx->cfg.dtype == VIT_BF16 && (!aligned16(x) || !aligned16(y))) return VIT_ERR_INVALID_ARG;
+  if (seqs->total_tokens > 0 && !(ctx->cfg.flags & VIT_FLAG_NO_ROPE) && !seqs->pos_rc)
+    return VIT_ERR_INVALID_ARG;
+  const size_t need = workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr);
+  if (!workspace || ws_bytes < need) return VIT_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return VIT_ERR_WORKSPACE;
+  return VIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *vit_status_string(vit_status s) {
+  switch (s) {
+    case VIT_OK: return "VIT_OK";
+    case VIT_ERR_INVALID_ARG: return "VIT_ERR_INVALID_ARG";
+    case VIT_ERR_SHAPE: return "VIT_ERR_SHAPE";
+    case VIT_ERR_UNSUPPORTED: return "VIT_ERR_UNSUPPORTED";
+    case VIT_ERR_WORKSPACE: return "VIT_ERR_WORKSPACE";
+    case VIT_ERR_CUDA: return "VIT_ERR_CUDA";
+    case VIT_ERR_TIMEOUT: return "VIT_ERR_TIMEOUT";
+    case VIT_ERR_DEVICE_BOUNDS: return "VIT_ERR_DEVICE_BOUNDS";
+  }
+  return "VIT_ERR_UNKNOWN";
+}
+
+const char *vit_version(void) { return "libvit 0.1 sm_100a"; }
+
+vit_status vit_init(const vit_config *cfg, int device, vit_ctx **out) {
+  if (!out) return VIT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return VIT_ERR_INVALID_ARG;
+  const vit_config &c = *cfg;
+  if (c.dtype != VIT_F32 && c.dtype != VIT_BF16) return VIT_ERR_INVALID_ARG;
+  if (c.hidden <= 0 || c.heads <= 0 || c.head_dim <= 0) return VIT_ERR_INVALID_ARG;
+  if (c.heads * c.head_dim != c.hidden) return VIT_ERR_SHAPE;
+  if (!(c.flags & VIT_FLAG_NO_MLP) && c.mlp <= 0) return VIT_ERR_INVALID_ARG;
+  if (!(c.ln_eps >= 0.f) || !(c.rope_theta > 0.f)) return VIT_ERR_INVALID_ARG;
+  if (c.flags & ~(VIT_FLAG_NO_ROPE | VIT_FLAG_NO_MLP)) return VIT_ERR_INVALID_ARG;
+  const bool hd_ok = c.dtype == VIT_F32 ? (c.head_dim == 64 || c.head_dim == 72 || c.head_dim == 128)
+                                        : (c.head_dim == 72 || c.head_dim == 128);
+  if (!hd_ok) return VIT_ERR_UNSUPPORTED;
+  if (c.hidden % 8 || (!(c.flags & VIT_FLAG_NO_MLP) && c.mlp % 8)) return VIT_ERR_UNSUPPORTED;
+  if (c.hidden > 4096) return VIT_ERR_UNSUPPORTED;  // LayerNorm keeps a row in registers
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+    return VIT_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return VIT_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return VIT_ERR_UNSUPPORTED;
+  DeviceGuard g(device);
+  vit_ctx *ctx = new vit_ctx;
+  ctx->cfg = c;
+  ctx->device = device;
+  ctx->num_sms = prop.multiProcessorCount;
+  ctx->d_status = nullptr;
+  if (cudaMalloc(&ctx->d_status, 4 * sizeof(int)) != cudaSuccess ||
+      cudaMemset(ctx->d_status, 0, 4 * sizeof(int)) != cudaSuccess) {
+    if (ctx->d_status) cudaFree(ctx->d_status);
+    delete ctx;
+    return VIT_ERR_CUDA;
+  }
+  const int h = c.head_dim / 2;
+  memset(&ctx->fr, 0, sizeof(ctx->fr));
+  for (int j = 0; j < c.head_dim / 4 && j < 32; ++j)
+    ctx->fr.wpi[j] = float(pow(double(c.rope_theta), -2.0 * j / h) / M_PI);
+  *out = ctx;
+  return VIT_OK;
+}
+
+void vit_destroy(vit_ctx *ctx) {
+  if (!ctx) return;
+  {
+    DeviceGuard g(ctx->device);
+    if (ctx->d_status) cudaFree(ctx->d_status);
+  }
+  delete ctx;
+}
+
+size_t vit_workspace_bytes(const vit_ctx *ctx, int total_tokens) {
+  if (!ctx || total_tokens < 0) return 0;
+  return workspace_layout(ctx->cfg, total_tokens, nullptr, nullptr);
+}
+
+vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const void *x, void *y,
+                             const vit_seqs *seqs, void *workspace, size_t ws_bytes,
+                             void *stream) {
+  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes);
+  if (s != VIT_OK) return s;
+  if ((s = check_layer_weights(ctx->cfg, w)) != VIT_OK) return s;
+  if (seqs->total_tokens == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  Workspace ws;
+  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, workspace);
+  return layer_impl(ctx, w, x, y, seqs, ws, static_cast<cudaStream_t>(stream));
+}
+
+vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, int n_layers,
+                               const void *x, void *y, const vit_seqs *seqs, void *workspace,
+                               size_t ws_bytes, void *stream) {
+  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes);
+  if (s != VIT_OK) return s;
+  if (!layers || n_layers < 1) return VIT_ERR_INVALID_ARG;
+  for (int i = 0; i < n_layers; ++i)
+    if ((s = check_layer_weights(ctx->cfg, &layers[i])) != VIT_OK) return s;
+  if (seqs->total_tokens == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  Workspace ws;
+  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < n_layers; ++i) {
+    const void *in = i == 0 ? x : ws.act[(i - 1) & 1];
+    void *out = i == n_layers - 1 ? y : ws.act[i & 1];
+    if ((s = layer_impl(ctx, &layers[i], in, out, seqs, ws, st)) != VIT_OK) return s;
+  }
+  return VIT_OK;
+}
+
+vit_status vit_attention(vit_ctx *ctx, const void *qkv, void *o, const vit_seqs *seqs,
+                         float scale, void *stream) {
+  if (!ctx || !qkv || !o) return VIT_ERR_INVALID_ARG;
+  vit_status s = check_seqs(ctx, seqs, true);
+  if (s != VIT_OK) return s;
+  if (ctx->cfg.dtype == VIT_BF16 && (!aligned16(qkv) || !aligned16(o))) return VIT_ERR_INVALID_ARG;
+  if (seqs->total_tokens == 0) return VIT_OK;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf(float(ctx->cfg.head_dim));
+  DeviceGuard g(ctx->device);
+  const SeqArgs sa = to_seq_args(seqs, true);
+  return cuda_status(run_attention(ctx, qkv, o, sa, scale, static_cast<cudaStream_t>(stream)));
+}
+
+vit_status vit_layernorm(vit_ctx *ctx, const void *x, void *y, const void *gamma,
+                         const void *beta, int rows, int cols, float eps, void *stream) {
+  if (!ctx || !x || !y || !gamma || !beta || rows < 0 || cols <= 0 || !(eps >= 0.f))
+    return VIT_ERR_INVALID_ARG;
+  if (cols % 4 || cols > 4096) return VIT_ERR_UNSUPPORTED;
+  const size_t a = esize(ctx->cfg) * 4;
+  const void *ps[4] = {x, y, gamma, beta};
+  for (const void *p : ps)
+    if (reinterpret_cast<uintptr_t>(p) % a) return VIT_ERR_INVALID_ARG;
+  if (rows == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  return cuda_status(launch_layernorm(ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16, x, y, gamma, beta,
+                                      rows, cols, eps, static_cast<cudaStream_t>(stream)));
+}
+
+vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w, const void *bias,
+                      const void *residual, void *y, int M, int N, int K, vit_epilogue epi,
+                      void *stream) {
+  if (!ctx || !x || !w || !y || M < 0 || N <= 0 || K <= 0) return VIT_ERR_INVALID_ARG;
+  if (epi != VIT_EPI_BIAS && epi != VIT_EPI_BIAS_GELU && epi != VIT_EPI_BIAS_RESIDUAL)
+    return VIT_ERR_INVALID_ARG;
+  if (epi == VIT_EPI_BIAS_RESIDUAL && !residual) return VIT_ERR_INVALID_ARG;
+  if (ctx->cfg.dtype == VIT_BF16) {
+    if (K % 8 || N % 8) return VIT_ERR_UNSUPPORTED;
+    const void *ps[5] = {x, w, bias, residual, y};
+    for (const void *p : ps)
+      if (p && !aligned16(p)) return VIT_ERR_INVALID_ARG;
+  }
+  if (M == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  return cuda_status(run_linear(ctx, x, w, bias, epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr,
+                                y, M, N, K, int(epi), static_cast<cudaStream_t>(stream)));
+}
+
+vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc, int total_tokens,
+                      void *stream) {
+  if (!ctx || !qkv || !pos_rc || total_tokens < 0) return VIT_ERR_INVALID_ARG;
+  if (total_tokens == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  const vit_config &c = ctx->cfg;
+  return cuda_status(launch_rope2d(c.dtype == VIT_F32 ? kF32 : kBF16, qkv, pos_rc, total_tokens,
+                                   c.heads, c.head_dim, ctx->fr, static_cast<cudaStream_t>(stream)));
+}
+
+vit_status vit_spatial_merge_2x2(vit_ctx *ctx, const void *x, void *y,
+                                 const int32_t *grids_hw_host, int n_images, int channels,
+                                 void *stream) {
+  if (!ctx || !x || !y || !grids_hw_host || n_images < 0 || channels <= 0)
+    return VIT_ERR_INVALID_ARG;
+  long long total = 0;
+  for (int i = 0; i < n_images; ++i) {
+    const int r = grids_hw_host[2 * i], c = grids_hw_host[2 * i + 1];
+    if (r <= 0 || c <= 0) return VIT_ERR_SHAPE;
+    if (r % 2 || c % 2) return VIT_ERR_SHAPE;
+    total += (long long)r * c;
+  }
+  if (total > INT32_MAX) return VIT_ERR_SHAPE;
+  const size_t row_bytes = size_t(channels) * esize(ctx->cfg);
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  long long base = 0;
+  for (int i0 = 0; i0 < n_images; i0 += kMaxImagesPerLaunch) {
+    const int n = std::min(kMaxImagesPerLaunch, n_images - i0);
+    ImageTable tab;
+    long long max_out = 0;
+    for (int i = 0; i < n; ++i) {
+      const int r = grids_hw_host[2 * (i0 + i)], c = grids_hw_host[2 * (i0 + i) + 1];
+      tab.img[i].rows = r;
+      tab.img[i].cols = c;
+      tab.img[i].base = int(base);
+      base += (long long)r * c;
+      max_out = std::max(max_out, (long long)(r / 2) * (c / 2));
+    }
+    if (launch_merge2x2(tab, n, x, y, row_bytes, max_out, st) != cudaSuccess) return VIT_ERR_CUDA;
+  }
+  return VIT_OK;
+}
+
+vit_status vit_positions_from_grids(vit_ctx *ctx, const int32_t *grids_hw_host, int n_images,
+                                    int32_t *cu_seqlens, int32_t *pos_rc, void *stream) {
+  if (!ctx || !grids_hw_host || !cu_seqlens || !pos_rc || n_images < 1 || n_images > 1024)
+    return VIT_ERR_INVALID_ARG;
+  long long total = 0;
+  for (int i = 0; i < n_images; ++i) {
+    const int r = grids_hw_host[2 * i], c = grids_hw_host[2 * i + 1];
+    if (r <= 0 || c <= 0) return VIT_ERR_SHAPE;
+    total += (long long)r * c;
+  }
+  if (total > INT32_MAX) return VIT_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(pos_rc) & 7u) return VIT_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  long long base = 0;
+  for (int i0 = 0; i0 < n_images; i0 += kMaxImagesPerLaunch) {
+    const int n = std::min(kMaxImagesPerLaunch, n_images - i0);
+    ImageTable tab;
+    int max_tok = 0;
+    for (int i = 0; i < n; ++i) {
+      const int r = grids_hw_host[2 * (i0 + i)], c = grids_hw_host[2 * (i0 + i) + 1];
+      tab.img[i].rows = r;
+      tab.img[i].cols = c;
+      tab.img[i].base = int(base);
+      base += (long long)r * c;
+      max_tok = std::max(max_tok, r * c);
+    }
+    if (launch_positions(tab, n, i0, max_tok, cu_seqlens, pos_rc, st) != cudaSuccess)
+      return VIT_ERR_CUDA;
+  }
+  return VIT_OK;
+}
+
+vit_status vit_get_last_device_status(vit_ctx *ctx) {
+  if (!ctx) return VIT_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return VIT_ERR_CUDA;
+  int h[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(h, ctx->d_status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return VIT_ERR_CUDA;
+  if (cudaMemset(ctx->d_status, 0, sizeof(h)) != cudaSuccess) return VIT_ERR_CUDA;
+  if (h[0] == kDevTimeout) return VIT_ERR_TIMEOUT;
+  if (h[0] == kDevBounds) return VIT_ERR_DEVICE_BOUNDS;
+  return VIT_OK;
+}
+
+}  // extern "C"
