@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Throughput of the ViT encoder hot path on B200.
+
+One step = the whole path over one batch: 27 pre-LN encoder layers over one
+3900-patch image (hidden 1152, 16 x 72 heads, MLP 4304, bf16) followed by the
+2x2 spatial merge to 975 x 4608, all through libvit's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs as one process per GPU (torchrun); every rank runs its own image
+(replicas: the encoder of one image has no exchange to shard), the step time
+is the max over ranks and ``value`` counts the patches of all ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference available:
+the pages publish no runnable code) on the host cores, on a bounded sample
+of the same workload, and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ViT encoder patches/s (27L, 3900 patches, bf16) and % of B200 bf16 tensor peak"
+UNIT = "patches/s"
+WORKLOAD = "c2"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiler captures only: run this many layers (line marked partial)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"vit_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    mx = float(c[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_step_time(max_seconds=15.0):
+    """Times the fp64 oracle on a bounded sample of the workload: layers of
+    the 3900-token stack until ``max_seconds`` (at least one), scaled to all
+    27 layers, plus the merge.  Returns (seconds per step, sample text)."""
+    import numpy as np
+
+    import synth
+    from oracle import run as orun
+    from oracle import vit_ref as R
+
+    wl = synth.get(WORKLOAD)
+    inp = synth.make_inputs(wl, layers=3)
+    cu, pos = R.positions_from_grids(wl.grids)
+    x = synth.to_f64(inp.x, wl.dtype)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        x = R.layer_forward(x, orun.layer_f64(inp, n % 3), cu, pos, wl.heads, wl.head_dim)
+        n += 1
+        if time.perf_counter() - t0 >= max_seconds or n >= wl.layers:
+            break
+    t_layers = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    R.spatial_merge_2x2(x, wl.grids)
+    t_merge = time.perf_counter() - t1
+    step = t_layers / n * wl.layers + t_merge
+    return step, f"{n} of {wl.layers} layers of the 3900-token stack in fp64 (x{wl.layers / n:.1f}) + merge"
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        th = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if th:
+            return int(max(th))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    wl_steps = []
+    for i in range(args.warmup + args.steps):
+        t, sample = oracle_step_time(max_seconds=2.0)
+        if i >= args.warmup:
+            wl_steps.append(t)
+    import statistics
+    t = statistics.mean(wl_steps)
+    value = 3900.0 / t
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, synth.c2)",
+        "config": {"workload": "c2: 27-layer ViT encoder, 3900 patches (50x78 grid), hidden 1152, "
+                               "16x72 heads, MLP 4304, + 2x2 merge", "global_batch": 1,
+                   "seq_len": 3900, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_traffic(kind):
+    """DRAM bytes per launch from a committed ncu summary, when it was taken
+    on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kind)
+    if not e or e.get("source_sha") != source_hash(e.get("sources", [])):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import numpy as np
+    import torch
+
+    import synth
+    import vision_transformer_encoder_layernorm_b200 as vit
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    wl = synth.get(WORKLOAD)
+    T, C = wl.tokens, wl.hidden
+    if args.layers:
+        wl = wl.with_(layers=min(args.layers, wl.layers))
+    flops = wl.flops()
+    inp = synth.make_inputs(wl)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    ctx = vit.Context(C, wl.heads, wl.head_dim, wl.mlp, vit.BF16, device=local_rank)
+    layers = [{k: dev(v) for k, v in lw.items()} for lw in inp.layers]
+    lw_structs = [vit.layer_weights(l) for l in layers]
+    x = dev(inp.x)
+    cu = torch.empty(2, dtype=torch.int32, device="cuda")
+    pos = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+    ctx.positions_from_grids(wl.grids, cu, pos)
+    sq = vit.seqs(T, 1, T, cu, pos)
+    ws = torch.empty(ctx.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(x)
+    out = torch.empty((T // 4, 4 * C), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ctx.encoder_forward(lw_structs, x, y, sq, ws, stream)
+        ctx.spatial_merge_2x2(y, out, wl.grids, C, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ctx.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # ---- timed region: K steps, L2 flushed before each, events around each
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    ctx.profile_read(reset=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    launches = sum(n for n, _ in ctx.profile_read(reset=True).values())
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    t_ms = float(np.mean(step_ms))
+    if dist is not None:
+        tt = torch.tensor([t_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms = float(tt.item())
+    value = world * T / (t_ms / 1e3)
+
+    # ---- per-kernel device time inside the same steps (events around launches)
+    ctx.profile_enable(True)
+    for _ in range(max(2, min(args.steps, 5))):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    prof = ctx.profile_read(reset=True)
+    ctx.profile_enable(False)
+    Fm = wl.mlp
+    work = {  # algorithmic work per launch: (FLOP, bytes)
+        "gemm_qkv": (2.0 * T * 3 * C * C, None), "gemm_out": (2.0 * T * C * C, None),
+        "gemm_fc1": (2.0 * T * Fm * C, None), "gemm_fc2": (2.0 * T * C * Fm, None),
+        "attention": (4.0 * T * T * C, None),
+        "layernorm": (None, 2.0 * T * C * 2 + 2 * C * 2),
+        "rope": (None, 2.0 * T * 2 * C * 2 + T * 8), "merge": (None, 2.0 * T * C * 2),
+    }
+    pk, pk_src = peaks()
+    tensor_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    kernels = {}
+    for name, (n, ms) in prof.items():
+        if n == 0 or name not in work:
+            continue
+        avg_s = ms / n / 1e3
+        fl, by = work[name]
+        if fl is not None:
+            ach = fl / avg_s / 1e12
+            kernels[name] = {"launches": n, "avg_us": avg_s * 1e6, "share": 0.0, "bound": "tensor",
+                             "achieved": ach, "unit": "TFLOP/s", "frac": ach / tensor_peak}
+        else:
+            ach = by / avg_s / 1e9
+            kernels[name] = {"launches": n, "avg_us": avg_s * 1e6, "share": 0.0, "bound": "hbm",
+                             "achieved": ach, "unit": "GB/s", "frac": ach / pk["hbm_gbs"]}
+    tot = sum(prof[k][1] for k in kernels)
+    for k in kernels:
+        kernels[k]["share"] = prof[k][1] / tot if tot else 0.0
+    dom = max(kernels, key=lambda k: prof[k][1])
+    d = kernels[dom]
+    roofline = {"bound": d["bound"], "achieved": d["achieved"],
+                "peak": tensor_peak if d["bound"] == "tensor" else pk["hbm_gbs"],
+                "unit": d["unit"], "frac": d["frac"], "traffic": kernel_traffic(dom),
+                "kernel": dom,
+                "peak_source": f"{pk_src} ({'bf16 sustained' if d['bound'] == 'tensor' else 'HBM copy'})"}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx = torch.empty((T, C), dtype=torch.bfloat16, pin_memory=True)
+        hx.copy_(x.cpu())
+        hout = torch.empty((T // 4, 4 * C), dtype=torch.bfloat16, pin_memory=True)
+        xin = torch.empty_like(x)
+
+        def e2e_step():
+            xin.copy_(hx, non_blocking=True)
+            ctx.encoder_forward(lw_structs, xin, y, sq, ws, stream)
+            ctx.spatial_merge_2x2(y, out, wl.grids, C, stream)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        barrier()
+        for k in range(args.steps):
+            flush.zero_()
+            ee[k][0].record(stream)
+            e2e_step()
+            ee[k][1].record(stream)
+        torch.cuda.synchronize()
+        e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
+        if dist is not None:
+            tt = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * T / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": hx.numel() * hx.element_size(),
+               "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    if ctx.device_status() != 0:
+        raise RuntimeError("device status set during the benchmark")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_cpu, sample = oracle_step_time(max_seconds=15.0)
+        cpu = {"value": T / t_cpu, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        tflops = flops["total"] / (t_ms / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded, synth.c2; random-init weights)",
+            "config": {"workload": "c2: 27-layer ViT encoder, 3900 patches (50x78 grid), "
+                                   "hidden 1152, 16x72 heads, MLP 4304, + 2x2 merge to 975x4608",
+                       "global_batch": world, "seq_len": T,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed before every timed step (256 MiB write)"},
+            "tflops": tflops, "pct_bf16_peak": tflops / tensor_peak,
+            **({"partial": f"{wl.layers} layers (profiler capture, not a bench line)"}
+               if args.layers else {}),
+            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

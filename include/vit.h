@@ -192,6 +192,28 @@ VIT_API vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w,
 VIT_API vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc,
                       int total_tokens, void *stream);
 
+/* ---- launch accounting and per-kernel timing ---- */
+
+/* Kernel kinds counted by the context (one count per kernel launch). */
+typedef enum {
+  VIT_K_LAYERNORM = 0, VIT_K_GEMM_QKV = 1, VIT_K_ROPE = 2, VIT_K_ATTENTION = 3,
+  VIT_K_GEMM_OUT = 4, VIT_K_GEMM_FC1 = 5, VIT_K_GEMM_FC2 = 6, VIT_K_MERGE = 7,
+  VIT_K_POSITIONS = 8, VIT_K_GEMM = 9, /* vit_linear */
+  VIT_K_COUNT = 10
+} vit_kernel_kind;
+
+/* enable != 0: every later kernel launch of this context is bracketed by two
+ * CUDA events recorded on its stream (host-side objects, no device memory);
+ * enable == 0 stops recording.  Not thread-safe while enabled. */
+VIT_API vit_status vit_profile_enable(vit_ctx *ctx, int enable);
+
+/* For kernel kind `kind`: *launches = launches since the last reset (always
+ * counted), *total_ms = summed device time of the launches recorded while
+ * profiling was enabled (synchronises on the recorded events).  reset != 0
+ * clears the counts and recorded events of every kind after reading. */
+VIT_API vit_status vit_profile_read(vit_ctx *ctx, int kind, long long *launches,
+                                    double *total_ms, int reset);
+
 /* ---- status ---- */
 
 /* Synchronises the device, reads the context's device status word, clears

@@ -125,7 +125,8 @@ def test_rope2d(H, d, dt):
     torch.cuda.synchronize()
     q, k, v = R.split_qkv(qr, H, d)
     out = from_dev(qkv).reshape(T, 3, H, d)
-    tol = 1e-2 if dt == "bf16" else 2e-6
+    # fp32: the rotation angle p*w is carried in fp32 (3e-6 rad at p ~ 90)
+    tol = 1e-2 if dt == "bf16" else 2e-5
     assert_close(out[:, 0], R.rope2d(q, pos), tol, 0.99999, "rope q")
     assert_close(out[:, 1], R.rope2d(k, pos), tol, 0.99999, "rope k")
     assert torch.equal(qkv.view(T, 3, H * d)[:, 2], before.view(T, 3, H * d)[:, 2])
@@ -233,7 +234,7 @@ def test_attention_tc_bf16(H, d, lens, P, Hkv, rope):
 def test_attention_simt_f32(d, lens, P, rope):
     H = 2
     y, ref, st = _attention_case("f32", H, d, lens, P, 1 if P else 0, rope, seed=30)
-    assert_close(y, ref, 2e-6, None, f"attention f32 d{d}")
+    assert_close(y, ref, 2e-5, None, f"attention f32 d{d}")
 
 
 def test_attention_full_size_rows():

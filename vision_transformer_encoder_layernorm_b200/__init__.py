@@ -6,7 +6,7 @@ merge.
 
 This module only marshals arguments: every step runs in the CUDA kernels of
 ``libvit.so``.  There is no fallback; importing fails loudly when the library
-has not been built (``python -m vision_transformer_encoder_layernorm_b200.build``).
+has not been built (``python vision_transformer_encoder_layernorm_b200/build.py``).
 Tensors are PyTorch tensors (device memory and streams only).
 """
 from __future__ import annotations
@@ -18,7 +18,7 @@ from typing import Optional, Sequence
 __all__ = [
     "lib", "LIB_PATH", "VitError", "VitConfig", "VitLayerWeights", "VitSeqs", "Context",
     "F32", "BF16", "FLAG_NO_ROPE", "FLAG_NO_MLP", "EPI_BIAS", "EPI_BIAS_GELU",
-    "EPI_BIAS_RESIDUAL", "STATUS", "ABI_FUNCTIONS",
+    "EPI_BIAS_RESIDUAL", "STATUS", "ABI_FUNCTIONS", "KERNEL_KINDS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvit.so")
@@ -26,6 +26,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvit.so")
 F32, BF16 = 0, 1
 FLAG_NO_ROPE, FLAG_NO_MLP = 0x1, 0x2
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_RESIDUAL = 0, 1, 2
+KERNEL_KINDS = ("layernorm", "gemm_qkv", "rope", "attention", "gemm_out", "gemm_fc1",
+                "gemm_fc2", "merge", "positions", "gemm")
 STATUS = {0: "VIT_OK", 1: "VIT_ERR_INVALID_ARG", 2: "VIT_ERR_SHAPE", 3: "VIT_ERR_UNSUPPORTED",
           4: "VIT_ERR_WORKSPACE", 5: "VIT_ERR_CUDA", 6: "VIT_ERR_TIMEOUT",
           7: "VIT_ERR_DEVICE_BOUNDS"}
@@ -75,6 +77,9 @@ ABI_FUNCTIONS = {
     "vit_layernorm": (_I, [_P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P]),
     "vit_linear": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "vit_rope2d": (_I, [_P, _P, _P, _I, _P]),
+    "vit_profile_enable": (_I, [_P, _I]),
+    "vit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_longlong),
+                              ctypes.POINTER(ctypes.c_double), _I]),
     "vit_get_last_device_status": (_I, [_P]),
     "vit_status_string": (ctypes.c_char_p, [_I]),
     "vit_version": (ctypes.c_char_p, []),
@@ -85,7 +90,7 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m vision_transformer_encoder_layernorm_b200.build` (nvcc, sm_100a)")
+            "`python vision_transformer_encoder_layernorm_b200/build.py` (nvcc, sm_100a)")
     h = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in ABI_FUNCTIONS.items():
         fn = getattr(h, name)
@@ -209,3 +214,20 @@ class Context:
 
     def device_status(self) -> int:
         return lib.vit_get_last_device_status(self._h)
+
+    def profile_enable(self, enable: bool = True):
+        _check("vit_profile_enable", lib.vit_profile_enable(self._h, int(bool(enable))))
+
+    def profile_read(self, reset: bool = False):
+        """{kind name: (launches, total device ms)} for every kernel kind."""
+        out = {}
+        for k, name in enumerate(KERNEL_KINDS):
+            n, ms = ctypes.c_longlong(), ctypes.c_double()
+            _check("vit_profile_read", lib.vit_profile_read(self._h, k, ctypes.byref(n),
+                                                            ctypes.byref(ms), 0))
+            out[name] = (n.value, ms.value)
+        if reset:
+            n, ms = ctypes.c_longlong(), ctypes.c_double()
+            _check("vit_profile_read", lib.vit_profile_read(self._h, 0, ctypes.byref(n),
+                                                            ctypes.byref(ms), 1))
+        return out

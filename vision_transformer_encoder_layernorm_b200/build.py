@@ -1,6 +1,6 @@
 """Builds libvit.so in-tree for sm_100a with nvcc (no GPU needed).
 
-    python -m vision_transformer_encoder_layernorm_b200.build [--force]
+    python vision_transformer_encoder_layernorm_b200/build.py [--force]
 
 The shared library is written next to this file; the CUDA runtime is linked
 statically, the driver API (cuTensorMapEncodeTiled) is resolved at run time

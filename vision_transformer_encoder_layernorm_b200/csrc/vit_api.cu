@@ -21,12 +21,49 @@
 #include "../../include/vit.h"
 #include "kernels.h"
 
+// Launch accounting: a count per kernel kind, and (while enabled) a pair of
+// CUDA events around every launch.
+struct VitProfiler {
+  struct Rec {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  bool on = false;
+  long long launches[VIT_K_COUNT] = {};
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void clear() {
+    for (auto &r : recs) {
+      pool.push_back(r.a);
+      pool.push_back(r.b);
+    }
+    recs.clear();
+    for (auto &l : launches) l = 0;
+  }
+  void destroy() {
+    clear();
+    for (auto e : pool) cudaEventDestroy(e);
+    pool.clear();
+  }
+};
+
 struct vit_ctx {
   vit_config cfg;
   int device;
   int num_sms;
   int *d_status;  // 4 ints; [0] = first error code recorded by a kernel
   vit::RopeFreqs fr;
+  VitProfiler prof;
 };
 
 namespace {
@@ -51,6 +88,20 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 vit_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VIT_OK : VIT_ERR_CUDA; }
+
+// Runs one kernel launch `f` of kind `kind` with launch accounting.
+template <class F>
+cudaError_t counted(vit_ctx *ctx, int kind, cudaStream_t st, F &&f) {
+  VitProfiler &p = ctx->prof;
+  p.launches[kind]++;
+  if (!p.on) return f();
+  cudaEvent_t a = p.get(), b = p.get();
+  cudaEventRecord(a, st);
+  const cudaError_t e = f();
+  cudaEventRecord(b, st);
+  p.recs.push_back({kind, a, b});
+  return e;
+}
 
 vit_status check_seqs(const vit_ctx *ctx, const vit_seqs *s, bool allow_prefix) {
   if (!s) return VIT_ERR_INVALID_ARG;
@@ -82,20 +133,24 @@ SeqArgs to_seq_args(const vit_seqs *s, bool with_pos) {
   return a;
 }
 
-cudaError_t run_linear(vit_ctx *ctx, const void *x, const void *w, const void *b,
+cudaError_t run_linear(vit_ctx *ctx, int kind, const void *x, const void *w, const void *b,
                        const void *res, void *y, int M, int N, int K, int epi, cudaStream_t st) {
-  if (ctx->cfg.dtype == VIT_F32) return launch_gemm_simt(kF32, x, w, b, res, y, M, N, K, epi, st);
-  return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st);
+  return counted(ctx, kind, st, [&] {
+    if (ctx->cfg.dtype == VIT_F32) return launch_gemm_simt(kF32, x, w, b, res, y, M, N, K, epi, st);
+    return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st);
+  });
 }
 
 cudaError_t run_attention(vit_ctx *ctx, const void *qkv, void *o, const SeqArgs &s, float scale,
                           cudaStream_t st) {
   const vit_config &c = ctx->cfg;
-  if (c.dtype == VIT_F32)
-    return launch_attention_simt(kF32, qkv, o, s, c.heads, c.head_dim, scale, ctx->fr,
-                                 ctx->d_status, st);
-  return launch_attention_tc(qkv, o, s, c.heads, c.head_dim, scale, ctx->fr, ctx->num_sms,
-                             ctx->d_status, st);
+  return counted(ctx, VIT_K_ATTENTION, st, [&] {
+    if (c.dtype == VIT_F32)
+      return launch_attention_simt(kF32, qkv, o, s, c.heads, c.head_dim, scale, ctx->fr,
+                                   ctx->d_status, st);
+    return launch_attention_tc(qkv, o, s, c.heads, c.head_dim, scale, ctx->fr, ctx->num_sms,
+                               ctx->d_status, st);
+  });
 }
 
 struct Workspace {
@@ -142,37 +197,46 @@ vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, v
   const int dt = c.dtype == VIT_F32 ? kF32 : kBF16;
   const bool rope = !(c.flags & VIT_FLAG_NO_ROPE) && seqs->pos_rc != nullptr;
   const float scale = 1.0f / sqrtf(float(c.head_dim));
-  cudaError_t e = cudaSuccess;
-  (void)e;
-  if ((e = launch_layernorm(dt, x, ws.h, w->ln1_g, w->ln1_b, T, C, c.ln_eps, st))) return VIT_ERR_CUDA;
-  if ((e = run_linear(ctx, ws.h, w->w_qkv, w->b_qkv, nullptr, ws.qkv, T, 3 * C, C, kEpiBias, st)))
+  auto ln = [&](const void *in, const void *g, const void *b) {
+    return counted(ctx, VIT_K_LAYERNORM, st, [&] {
+      return launch_layernorm(dt, in, ws.h, g, b, T, C, c.ln_eps, st);
+    });
+  };
+  if (ln(x, w->ln1_g, w->ln1_b)) return VIT_ERR_CUDA;
+  if (run_linear(ctx, VIT_K_GEMM_QKV, ws.h, w->w_qkv, w->b_qkv, nullptr, ws.qkv, T, 3 * C, C,
+                 kEpiBias, st))
     return VIT_ERR_CUDA;
-  if (rope && (e = launch_rope2d(dt, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st)))
+  if (rope && counted(ctx, VIT_K_ROPE, st, [&] {
+        return launch_rope2d(dt, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st);
+      }))
     return VIT_ERR_CUDA;
   const SeqArgs sa = to_seq_args(seqs, false);
-  if ((e = run_attention(ctx, ws.qkv, ws.attn, sa, scale, st))) return VIT_ERR_CUDA;
+  if (run_attention(ctx, ws.qkv, ws.attn, sa, scale, st)) return VIT_ERR_CUDA;
   if (c.flags & VIT_FLAG_NO_MLP) {
-    if ((e = run_linear(ctx, ws.attn, w->w_o, w->b_o, x, y, T, C, C, kEpiResidual, st)))
+    if (run_linear(ctx, VIT_K_GEMM_OUT, ws.attn, w->w_o, w->b_o, x, y, T, C, C, kEpiResidual, st))
       return VIT_ERR_CUDA;
     return VIT_OK;
   }
-  if ((e = run_linear(ctx, ws.attn, w->w_o, w->b_o, x, ws.x1, T, C, C, kEpiResidual, st)))
+  if (run_linear(ctx, VIT_K_GEMM_OUT, ws.attn, w->w_o, w->b_o, x, ws.x1, T, C, C, kEpiResidual,
+                 st))
     return VIT_ERR_CUDA;
-  if ((e = launch_layernorm(dt, ws.x1, ws.h, w->ln2_g, w->ln2_b, T, C, c.ln_eps, st)))
+  if (ln(ws.x1, w->ln2_g, w->ln2_b)) return VIT_ERR_CUDA;
+  if (run_linear(ctx, VIT_K_GEMM_FC1, ws.h, w->w_fc1, w->b_fc1, nullptr, ws.g, T, F, C, kEpiGelu,
+                 st))
     return VIT_ERR_CUDA;
-  if ((e = run_linear(ctx, ws.h, w->w_fc1, w->b_fc1, nullptr, ws.g, T, F, C, kEpiGelu, st)))
-    return VIT_ERR_CUDA;
-  if ((e = run_linear(ctx, ws.g, w->w_fc2, w->b_fc2, ws.x1, y, T, C, F, kEpiResidual, st)))
+  if (run_linear(ctx, VIT_K_GEMM_FC2, ws.g, w->w_fc2, w->b_fc2, ws.x1, y, T, C, F, kEpiResidual,
+                 st))
     return VIT_ERR_CUDA;
   return VIT_OK;
 }
 
 vit_status check_layer_call(vit_ctx *ctx, const void *x, void *y, const vit_seqs *seqs,
                             void *workspace, size_t ws_bytes) {
-  if (!ctx || !x || !y) return VIT_ERR_INVALID_ARG;
+  if (!ctx) return VIT_ERR_INVALID_ARG;
   vit_status s = check_seqs(ctx, seqs, true);
   if (s != VIT_OK) return s;
-  if (x == y) return VIT_ERR_INVALID_ARG;
+  if (seqs->total_tokens == 0) return VIT_OK;  // nothing is read or written
+  if (!x || !y || x == y) return VIT_ERR_INVALID_ARG;
   if (ctx->cfg.dtype == VIT_BF16 && (!aligned16(x) || !aligned16(y))) return VIT_ERR_INVALID_ARG;
   if (seqs->total_tokens > 0 && !(ctx->cfg.flags & VIT_FLAG_NO_ROPE) && !seqs->pos_rc)
     return VIT_ERR_INVALID_ARG;
@@ -248,6 +312,7 @@ void vit_destroy(vit_ctx *ctx) {
   if (!ctx) return;
   {
     DeviceGuard g(ctx->device);
+    ctx->prof.destroy();
     if (ctx->d_status) cudaFree(ctx->d_status);
   }
   delete ctx;
@@ -294,11 +359,12 @@ vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, in
 
 vit_status vit_attention(vit_ctx *ctx, const void *qkv, void *o, const vit_seqs *seqs,
                          float scale, void *stream) {
-  if (!ctx || !qkv || !o) return VIT_ERR_INVALID_ARG;
+  if (!ctx) return VIT_ERR_INVALID_ARG;
   vit_status s = check_seqs(ctx, seqs, true);
   if (s != VIT_OK) return s;
+  if (seqs->total_tokens == 0) return VIT_OK;  // nothing is read or written
+  if (!qkv || !o) return VIT_ERR_INVALID_ARG;
   if (ctx->cfg.dtype == VIT_BF16 && (!aligned16(qkv) || !aligned16(o))) return VIT_ERR_INVALID_ARG;
-  if (seqs->total_tokens == 0) return VIT_OK;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf(float(ctx->cfg.head_dim));
   DeviceGuard g(ctx->device);
   const SeqArgs sa = to_seq_args(seqs, true);
@@ -316,8 +382,11 @@ vit_status vit_layernorm(vit_ctx *ctx, const void *x, void *y, const void *gamma
     if (reinterpret_cast<uintptr_t>(p) % a) return VIT_ERR_INVALID_ARG;
   if (rows == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
-  return cuda_status(launch_layernorm(ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16, x, y, gamma, beta,
-                                      rows, cols, eps, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(counted(ctx, VIT_K_LAYERNORM, st, [&] {
+    return launch_layernorm(ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16, x, y, gamma, beta, rows,
+                            cols, eps, st);
+  }));
 }
 
 vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w, const void *bias,
@@ -335,8 +404,9 @@ vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w, const void *bi
   }
   if (M == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
-  return cuda_status(run_linear(ctx, x, w, bias, epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr,
-                                y, M, N, K, int(epi), static_cast<cudaStream_t>(stream)));
+  return cuda_status(run_linear(ctx, VIT_K_GEMM, x, w, bias,
+                                epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr, y, M, N, K,
+                                int(epi), static_cast<cudaStream_t>(stream)));
 }
 
 vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc, int total_tokens,
@@ -345,8 +415,11 @@ vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc, int total_
   if (total_tokens == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
   const vit_config &c = ctx->cfg;
-  return cuda_status(launch_rope2d(c.dtype == VIT_F32 ? kF32 : kBF16, qkv, pos_rc, total_tokens,
-                                   c.heads, c.head_dim, ctx->fr, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(counted(ctx, VIT_K_ROPE, st, [&] {
+    return launch_rope2d(c.dtype == VIT_F32 ? kF32 : kBF16, qkv, pos_rc, total_tokens, c.heads,
+                         c.head_dim, ctx->fr, st);
+  }));
 }
 
 vit_status vit_spatial_merge_2x2(vit_ctx *ctx, const void *x, void *y,
@@ -378,7 +451,9 @@ vit_status vit_spatial_merge_2x2(vit_ctx *ctx, const void *x, void *y,
       base += (long long)r * c;
       max_out = std::max(max_out, (long long)(r / 2) * (c / 2));
     }
-    if (launch_merge2x2(tab, n, x, y, row_bytes, max_out, st) != cudaSuccess) return VIT_ERR_CUDA;
+    if (counted(ctx, VIT_K_MERGE, st,
+                [&] { return launch_merge2x2(tab, n, x, y, row_bytes, max_out, st); }))
+      return VIT_ERR_CUDA;
   }
   return VIT_OK;
 }
@@ -410,9 +485,35 @@ vit_status vit_positions_from_grids(vit_ctx *ctx, const int32_t *grids_hw_host, 
       base += (long long)r * c;
       max_tok = std::max(max_tok, r * c);
     }
-    if (launch_positions(tab, n, i0, max_tok, cu_seqlens, pos_rc, st) != cudaSuccess)
+    if (counted(ctx, VIT_K_POSITIONS, st, [&] {
+          return launch_positions(tab, n, i0, max_tok, cu_seqlens, pos_rc, st);
+        }))
       return VIT_ERR_CUDA;
   }
+  return VIT_OK;
+}
+
+vit_status vit_profile_enable(vit_ctx *ctx, int enable) {
+  if (!ctx) return VIT_ERR_INVALID_ARG;
+  ctx->prof.on = enable != 0;
+  return VIT_OK;
+}
+
+vit_status vit_profile_read(vit_ctx *ctx, int kind, long long *launches, double *total_ms,
+                            int reset) {
+  if (!ctx || kind < 0 || kind >= VIT_K_COUNT) return VIT_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  double ms = 0.0;
+  for (auto &r : ctx->prof.recs) {
+    if (r.kind != kind) continue;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return VIT_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return VIT_ERR_CUDA;
+    ms += t;
+  }
+  if (launches) *launches = ctx->prof.launches[kind];
+  if (total_ms) *total_ms = ms;
+  if (reset) ctx->prof.clear();
   return VIT_OK;
 }
 
