@@ -214,6 +214,7 @@ def main():
 
     import synth
     import vision_transformer_encoder_layernorm_b200 as vit
+    from vision_transformer_encoder_layernorm_b200 import replicas
 
     torch.cuda.set_device(local_rank)
     dist = None
@@ -282,10 +283,7 @@ def main():
     launches = sum(n for n, _ in ctx.profile_read(reset=True).values())
     step_ms = [a.elapsed_time(b) for a, b in ev]
     t_ms = float(np.mean(step_ms))
-    if dist is not None:
-        tt = torch.tensor([t_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_ms = float(tt.item())
+    t_ms = replicas.max_over_ranks(t_ms, device="cuda")
     value = world * T / (t_ms / 1e3)
 
     # ---- per-kernel device time inside the same steps (events around launches)
@@ -358,10 +356,7 @@ def main():
             ee[k][1].record(stream)
         torch.cuda.synchronize()
         e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
-        if dist is not None:
-            tt = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = replicas.max_over_ranks(e_ms, device="cuda")
         e2e = {"value": world * T / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": hx.numel() * hx.element_size(),
                "d2h_bytes_per_step": hout.numel() * hout.element_size()}
