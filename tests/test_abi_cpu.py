@@ -77,3 +77,30 @@ def test_init_without_device_reports_cuda_error():
     h = ctypes.c_void_p()
     assert vit.lib.vit_init(ctypes.byref(cfg), 0, ctypes.byref(h)) == 5
     assert not h.value
+
+
+def test_structs_keep_their_tensors_alive():
+    # VitSeqs / VitLayerWeights hold raw device pointers: the binding must keep
+    # the tensors they point to alive, or a temporary passed to seqs() could be
+    # freed and its memory handed to the next allocation
+    import gc
+    import weakref
+
+    import torch
+
+    import vision_transformer_encoder_layernorm_b200 as vit
+    t = torch.zeros(4, dtype=torch.int32)
+    ref = weakref.ref(t)
+    s = vit.seqs(3, 1, 3, t)
+    del t
+    gc.collect()
+    assert ref() is not None and s.cu_seqlens == ref().data_ptr()
+    del s
+    gc.collect()
+    assert ref() is None
+    w = torch.zeros(8)
+    wref = weakref.ref(w)
+    lw = vit.layer_weights({"w_qkv": w})
+    del w
+    gc.collect()
+    assert wref() is not None and lw.w_qkv == wref().data_ptr() and lw.w_o is None

@@ -131,14 +131,22 @@ def _grids_arr(grids: Sequence[Sequence[int]]):
 
 def layer_weights(d) -> VitLayerWeights:
     """A VitLayerWeights from a mapping of the 12 parameter names to tensors
-    (missing or None entries become NULL)."""
-    return VitLayerWeights(*[_ptr(d.get(k)) for k in _WKEYS])
+    (missing or None entries become NULL).  The struct keeps the tensors
+    alive: it holds raw device pointers."""
+    lw = VitLayerWeights(*[_ptr(d.get(k)) for k in _WKEYS])
+    lw._tensors = dict(d)
+    return lw
 
 
 def seqs(total_tokens: int, n_seqs: int, max_seqlen: int, cu_seqlens, pos_rc=None,
          prefix_kv=None, prefix_len: int = 0, kv_heads: int = 0) -> VitSeqs:
-    return VitSeqs(total_tokens, n_seqs, max_seqlen, _ptr(cu_seqlens), _ptr(pos_rc),
-                   _ptr(prefix_kv), prefix_len if prefix_kv is not None else 0, kv_heads)
+    """A VitSeqs for packed sequences.  The struct keeps the cu_seqlens,
+    pos_rc and prefix_kv tensors alive (it holds their raw device pointers),
+    so temporaries passed here cannot be freed and reused while it lives."""
+    s = VitSeqs(total_tokens, n_seqs, max_seqlen, _ptr(cu_seqlens), _ptr(pos_rc),
+                _ptr(prefix_kv), prefix_len if prefix_kv is not None else 0, kv_heads)
+    s._tensors = (cu_seqlens, pos_rc, prefix_kv)
+    return s
 
 
 class Context:
