@@ -130,6 +130,35 @@ VIT_API vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w,
                              const void *x, void *y, const vit_seqs *seqs,
                              void *workspace, size_t ws_bytes, void *stream);
 
+/* vit_layer_forward without a workspace argument, for callers that cannot
+ * allocate device memory when they run a layer: for example a runtime that
+ * has already handed all device memory to its own pool, or a latency-critical
+ * sequence that must not call cudaMalloc/cudaFree (which can block and
+ * synchronise the device).  The pages describe no such call; it exists only
+ * for those callers.
+ *
+ * The layer's intermediates live in one fixed 32 MiB array compiled into the
+ * library (a static __device__ array; every GPU that loads the library holds
+ * it until the process exits).  The call allocates nothing: no cudaMalloc,
+ * cudaFree or allocating library routine.  The caller still passes x, y and
+ * the weights, as for vit_layer_forward.
+ *  - Size limit: vit_workspace_bytes(ctx, total_tokens) must be <= 32 MiB
+ *    (e.g. up to 1,240 tokens at hidden 1152 / MLP 4304); larger calls return
+ *    VIT_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device); make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents.  Nothing in it has to start at zero (every intermediate is
+ *    written before it is read), so nothing is cleared.  Calls whose work
+ *    overlaps on the GPU (different streams, no ordering between them) race
+ *    on the array: order them, e.g. issue them on one stream.
+ *  - Launch counts are kept as for every call; no timing events are created
+ *    during this call even when profiling is enabled. */
+VIT_API vit_status vit_layer_forward_noalloc(vit_ctx *ctx, const vit_layer_weights *w,
+                                             const void *x, void *y, const vit_seqs *seqs,
+                                             void *stream);
+
 /* The stack of n_layers layers; layers is a HOST array of n_layers weight
  * structs (device pointers inside).  Intermediate activations live in the
  * workspace; x is read only; y [T, C] receives the last layer's output. */

@@ -69,6 +69,8 @@ ABI_FUNCTIONS = {
     "vit_workspace_bytes": (ctypes.c_size_t, [_P, _I]),
     "vit_layer_forward": (_I, [_P, ctypes.POINTER(VitLayerWeights), _P, _P,
                                ctypes.POINTER(VitSeqs), _P, ctypes.c_size_t, _P]),
+    "vit_layer_forward_noalloc": (_I, [_P, ctypes.POINTER(VitLayerWeights), _P, _P,
+                                       ctypes.POINTER(VitSeqs), _P]),
     "vit_encoder_forward": (_I, [_P, ctypes.POINTER(VitLayerWeights), _I, _P, _P,
                                  ctypes.POINTER(VitSeqs), _P, ctypes.c_size_t, _P]),
     "vit_attention": (_I, [_P, _P, _P, ctypes.POINTER(VitSeqs), ctypes.c_float, _P]),
@@ -183,6 +185,13 @@ class Context:
         _check("vit_layer_forward", lib.vit_layer_forward(
             self._h, ctypes.byref(lw), _ptr(x), _ptr(y), ctypes.byref(sq), _ptr(workspace),
             workspace.numel() * workspace.element_size(), _stream(stream)))
+
+    def layer_forward_noalloc(self, weights, x, y, sq: VitSeqs, stream=None):
+        """vit_layer_forward_noalloc: the layer with the library's fixed
+        32 MiB scratch instead of a workspace (allocates nothing)."""
+        lw = layer_weights(weights) if not isinstance(weights, VitLayerWeights) else weights
+        _check("vit_layer_forward_noalloc", lib.vit_layer_forward_noalloc(
+            self._h, ctypes.byref(lw), _ptr(x), _ptr(y), ctypes.byref(sq), _stream(stream)))
 
     def encoder_forward(self, layers, x, y, sq: VitSeqs, workspace, stream=None):
         arr = (VitLayerWeights * len(layers))(

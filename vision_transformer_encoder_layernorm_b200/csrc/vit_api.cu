@@ -531,3 +531,66 @@ vit_status vit_get_last_device_status(vit_ctx *ctx) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation layer call
+// vit_layer_forward_noalloc: the same layer as vit_layer_forward, with its
+// scratch (the intermediate activations) in a fixed array compiled into the
+// library instead of a caller-provided workspace.
+#include <map>
+#include <mutex>
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB, per device
+
+// Device-side scratch of the no-allocation call.  Its name in host code is a
+// host stand-in, not a device address: host code only ever passes the
+// address returned by cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_layer_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+std::map<int, void *> g_scratch_addr;  // device ordinal -> device address of g_layer_scratch
+
+// Resolves the scratch's device address on the current device (the caller
+// made ctx->device current), once per device.
+vit_status static_scratch(int device, void **out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  auto it = g_scratch_addr.find(device);
+  if (it != g_scratch_addr.end()) {
+    *out = it->second;
+    return VIT_OK;
+  }
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_layer_scratch) != cudaSuccess || p == nullptr)
+    return VIT_ERR_CUDA;
+  g_scratch_addr[device] = p;
+  *out = p;
+  return VIT_OK;
+}
+
+}  // namespace
+
+extern "C" vit_status vit_layer_forward_noalloc(vit_ctx *ctx, const vit_layer_weights *w,
+                                                const void *x, void *y, const vit_seqs *seqs,
+                                                void *stream) {
+  if (!ctx || !seqs) return VIT_ERR_INVALID_ARG;
+  if (seqs->total_tokens < 0) return VIT_ERR_INVALID_ARG;
+  // size check first, against the fixed scratch, before any device work
+  if (workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr) > kStaticScratchBytes)
+    return VIT_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  void *scratch = nullptr;
+  vit_status s = static_scratch(ctx->device, &scratch);
+  if (s != VIT_OK) return s;
+  if ((s = check_layer_call(ctx, x, y, seqs, scratch, kStaticScratchBytes)) != VIT_OK) return s;
+  if ((s = check_layer_weights(ctx->cfg, w)) != VIT_OK) return s;
+  if (seqs->total_tokens == 0) return VIT_OK;
+  Workspace ws;
+  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, scratch);
+  // launch counts only: no timing events are created during this call
+  const bool prof_on = ctx->prof.on;
+  ctx->prof.on = false;
+  s = layer_impl(ctx, w, x, y, seqs, ws, static_cast<cudaStream_t>(stream));
+  ctx->prof.on = prof_on;
+  return s;
+}
