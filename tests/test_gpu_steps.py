@@ -257,3 +257,36 @@ def test_attention_full_size_rows():
     for h in range(H):
         ref = R.attention_segment(q[rows, h], k[:, h], v[:, h], 1 / np.sqrt(d))
         assert_close(got[:, h], ref, 2e-2, 0.9999, f"row sample head {h}")
+
+
+# ------------------------------------------------------------------ every GEMM variant
+VARIANT_CASES = [(300, 392, 200, 0), (257, 136, 64, 2), (3900, 3456, 1152, 0),
+                 (3900, 1152, 4304, 2), (960, 4304, 1152, 1), (1, 8, 8, 0)]
+
+
+@pytest.mark.parametrize("variant", ["1x128", "1x256", "2x128", "2x192", "2x256"])
+@pytest.mark.parametrize("M,N,K,epi", VARIANT_CASES)
+def test_linear_bf16_each_variant(ctx_bf16, monkeypatch, variant, M, N, K, epi):
+    # VIT_GEMM_TILE pins the GEMM variant (CTAs per MMA x tile width)
+    monkeypatch.setenv("VIT_GEMM_TILE", variant)
+    _, x, xr = _t((M, K), 51, "bf16")
+    _, w, wr = _t((N, K), 52, "bf16", 0.02)
+    _, b, br = _t((N,), 53, "bf16", 0.01)
+    _, res, rr = _t((M, N), 54, "bf16")
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ctx_bf16.linear(x, w, b, y, epi=epi, residual=res if epi == 2 else None)
+    torch.cuda.synchronize()
+    rows = np.arange(M)
+    if M > 1024:
+        g = np.random.Generator(np.random.PCG64(M + N + 7))
+        rows = np.unique(np.concatenate([g.choice(M, 192, replace=False),
+                                         [0, 127, 128, 255, 256, M - 129, M - 1]]))
+    ref = R.linear(xr[rows], wr, br)
+    if epi == 1:
+        ref = R.gelu_tanh(ref)
+    if epi == 2:
+        ref = ref + rr[rows]
+    got = from_dev(y)
+    assert np.all(np.isfinite(got)), "unwritten outputs"
+    assert_close(got[rows], ref, 1e-2, 0.99999, f"linear {variant} {M}x{N}x{K} epi{epi}")
+    assert ctx_bf16.device_status() == 0

@@ -16,7 +16,7 @@
 //   1        TMEM allocator; one lane issues all tcgen05.mma
 //   2-5      softmax warpgroup of query tile 0   (thread = query row)
 //   6-9      softmax warpgroup of query tile 1
-//   10-13    (ROPE only) rotates each own-key K tile in shared memory
+//   10-11    (ROPE only) rotate each own-key K tile in shared memory
 // TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,..), O1 [384,..).
 // head_dim 72 is computed as 80 (4 MMA k-steps from a 64-column 128B-swizzled
 // chunk, 1 from a 16-column 32B-swizzled chunk); Q's columns 72..79 are zeroed
@@ -128,7 +128,7 @@ __device__ __forceinline__ void rope_row_smem(uint8_t *tile, int r, int pr, int 
 }  // namespace attn
 
 template <int HD, bool ROPE>
-__global__ void __launch_bounds__(ROPE ? 448 : 320, 1)
+__global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_x0,
                         const __grid_constant__ CUtensorMap tm_x1,
                         const __grid_constant__ CUtensorMap tm_p0,
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(ROPE ? 448 : 320, 1)
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
-      mbar_init(&bars->k_ready[s], 128);
+      mbar_init(&bars->k_ready[s], 64);
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -351,33 +351,51 @@ __global__ void __launch_bounds__(ROPE ? 448 : 320, 1)
       const uint32_t s_addr = tmem + lane_base + CF::kTmemS + t * 128;
       const uint32_t o_addr = tmem + lane_base + CF::kTmemO + t * 128;
       const float sl2 = prm.scale_log2;
-      float m = -INFINITY, l = 0.f;
+      // head_dim 72: the softmax denominator is accumulated by the tensor core
+      // as O column 72 -- V's first padding column is set to 1.0 before each
+      // P.V -- so the row sum costs no instruction here (and sums exactly the
+      // bf16 P the numerator uses).  head_dim 128 sums in registers.
+      constexpr bool kSumByMma = (HD == 72);
+      float m = -INFINITY;
+      uint64_t l2[4] = {0, 0, 0, 0};  // packed partial row sums (head_dim 128)
       for (int j = 0; j < n_kv && ok; ++j) {
         if (!mbar_wait(&bars->s_full[t], j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int nvalid = j < n_pre ? min(kBlockK, prm.P - j * kBlockK)
                                      : min(kBlockK, len - (j - n_pre) * kBlockK);
-        // pass 1: row max of the raw scores
-        float mx = -INFINITY;
+        uint32_t s[4][32];
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, s[c]);
+        tmem_ld_wait();
+        if (nvalid < kBlockK) {  // keys past the sequence end: -inf, so p = 0
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i >= nvalid) s[c][i] = 0xFF800000u;
+        }
+        // row max: four independent chains of 3-input max
+        float mc[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld32(s_addr + c * 32, v);
-          tmem_ld_wait();
+          float a = __uint_as_float(s[c][0]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i < nvalid) mx = fmaxf(mx, __uint_as_float(v[i]));
+          for (int i = 1; i < 31; i += 2)
+            a = fmax3(a, __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
+          mc[c] = fmaxf(a, __uint_as_float(s[c][31]));
         }
-        const float m_tile = mx * sl2;
+        const float m_tile = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]) * sl2;
         const bool grow = __any_sync(0xffffffffu, m_tile > m + 8.0f);
         if (j == 0) {
           m = m_tile;
         } else if (grow) {
-          // rescale O and l only when the running max grew by more than 2^8
+          // rescale O (and the row sum) only when the running max grew by
+          // more than 8 in log2 units; otherwise keep the stale max
           const bool mine = m_tile > m + 8.0f;
           const float m_new = mine ? m_tile : m;
           const float factor = mine ? ex2_approx(m - m_new) : 1.0f;
+          const uint64_t f2 = f2_pack(factor, factor);
           if (!mbar_wait(&bars->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -387,33 +405,45 @@ __global__ void __launch_bounds__(ROPE ? 448 : 320, 1)
             tmem_ld16(o_addr + c * 16, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * factor);
+            for (int i = 0; i < 8; ++i) {
+              float a, b;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), f2),
+                        a, b);
+              v[2 * i] = __float_as_uint(a);
+              v[2 * i + 1] = __float_as_uint(b);
+            }
             tmem_st16(o_addr + c * 16, v);
           }
           tmem_st_wait();
-          l *= factor;
+          if (!kSumByMma)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) l2[k] = f2_mul(l2[k], f2);
           m = m_new;
         }
-        // pass 2: p = 2^(s*scale*log2e - m), row sum, bf16 P into S's columns
-        const float neg_m = -m;
+        // p = 2^(s*scale*log2e - m) two at a time; bf16 P into S's first 64 columns
+        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld32(s_addr + c * 32, v);
-          tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int c0 = c * 32 + 2 * i;
-            float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * i]), sl2, neg_m));
-            float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * i + 1]), sl2, neg_m));
-            if (c0 >= nvalid) p0 = 0.f;
-            if (c0 + 1 >= nvalid) p1 = 0.f;
-            l += p0 + p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])),
+                             sc2, nm2),
+                      x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if (!kSumByMma) l2[i & 3] = f2_add(l2[i & 3], f2_pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
           }
           tmem_st16(s_addr + c * 16, pk);
+        }
+        if (kSumByMma && t == 0) {
+          // ones in V's column 72 of this key tile (the first padding column)
+          const int st = j % NS;
+          if (!mbar_wait(&bars->v_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
+          *reinterpret_cast<uint16_t *>(smem + CF::kVOff + st * CF::kTile + unit_offset<HD>(r, 9)) =
+              0x3F80u;  // bf16 1.0
+          fence_proxy_async_smem();
         }
         tmem_st_wait();
         tc_fence_before();
@@ -422,43 +452,59 @@ __global__ void __launch_bounds__(ROPE ? 448 : 320, 1)
       // epilogue: O / l -> bf16 rows of o [T, H, HD]
       if (ok && mbar_wait(&bars->o_done[t], (n_kv - 1) & 1, abort_flag)) {
         tc_fence_after();
+        uint32_t ov[CF::HDP / 16][16];
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < CF::HDP / 16; ++c) tmem_ld16(o_addr + c * 16, ov[c]);
+        tmem_ld_wait();
+        float l;
+        if (kSumByMma) {
+          l = __uint_as_float(ov[4][8]);  // O column 72
+        } else {
+          float a, b, c2, d2;
+          f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), a, b);
+          (void)c2;
+          (void)d2;
+          l = a + b;
+        }
         const float inv = 1.0f / l;
-        __nv_bfloat16 *orow = prm.o + size_t(seg0 + qrow) * prm.C + size_t(h) * HD;
+        const uint64_t inv2 = f2_pack(inv, inv);
+        if (qrow < len) {
+          __nv_bfloat16 *orow = prm.o + size_t(seg0 + qrow) * prm.C + size_t(h) * HD;
 #pragma unroll
-        for (int c = 0; c < CF::HDP / 16; ++c) {
-          uint32_t v[16];
-          __syncwarp();
-          tmem_ld16(o_addr + c * 16, v);
-          tmem_ld_wait();
-          if (qrow < len) {
+          for (int u = 0; u < HD / 8; ++u) {  // 16-byte units of the output row
+            uint32_t w[4];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int col = c * 16 + q * 8;
-              if (col < HD) {
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
-                w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
-                w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
-                w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
-                *reinterpret_cast<uint4 *>(orow + col) = w;
-              }
+            for (int e = 0; e < 4; ++e) {
+              const int col = u * 8 + 2 * e;
+              float a, b;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(ov[col / 16][col % 16]),
+                                       __uint_as_float(ov[col / 16][col % 16 + 1])),
+                               inv2),
+                        a, b);
+              w[e] = pack_bf16x2(a, b);
             }
+            *reinterpret_cast<uint4 *>(orow + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
     }
   } else if (ROPE) {
     // ------------------------------------------------------------ K rotation
-    const int r = (warp - 10) * 32 + lane;  // key row inside the tile
+    // two warps; thread rotates key rows r and r + 64 of each own-key tile
+    const int r0 = (warp - 10) * 32 + lane;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j % NS;
       const uint32_t f = (j / NS) & 1;
       if (!mbar_wait(&bars->k_full[st], f, abort_flag)) break;
       if (j >= n_pre) {
-        const int key = (j - n_pre) * kBlockK + r;
-        if (key < len)
-          rope_row_smem<HD>(smem + CF::kKOff + st * CF::kTile, r, prm.pos[2 * (seg0 + key)],
-                            prm.pos[2 * (seg0 + key) + 1], fr);
+#pragma unroll 1
+        for (int r = r0; r < kBlockK; r += 64) {
+          const int key = (j - n_pre) * kBlockK + r;
+          if (key < len)
+            rope_row_smem<HD>(smem + CF::kKOff + st * CF::kTile, r, prm.pos[2 * (seg0 + key)],
+                              prm.pos[2 * (seg0 + key) + 1], fr);
+        }
         fence_proxy_async_smem();
       }
       mbar_arrive(&bars->k_ready[st]);
@@ -483,7 +529,7 @@ static cudaError_t launch_hd(const CUtensorMap *maps, const attn::Params &prm, i
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, ROPE ? 448 : 320, CF::kSmem, st>>>(maps[0], maps[1], maps[2], maps[3], prm, fr);
+  kern<<<grid, ROPE ? 384 : 320, CF::kSmem, st>>>(maps[0], maps[1], maps[2], maps[3], prm, fr);
   return cudaGetLastError();
 }
 

@@ -17,6 +17,8 @@
 // tile i+1.  Every wait is bounded (see mbar_wait); on a timeout the kernel
 // drains its in-flight copies, frees TMEM and reports through `status`.
 #include <cudaTypedefs.h>
+#include <stdio.h>
+#include <stdlib.h>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -70,6 +72,60 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 }
 
 }  // namespace gemm
+
+// One 32-column slice of one output row: fp32 accumulators r -> + bias ->
+// epilogue op -> bf16 stores (columns at or past N are skipped, N % 8 == 0).
+template <int EPI>
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, int col0, int N,
+                                            const __nv_bfloat16 *__restrict__ bias,
+                                            const __nv_bfloat16 *__restrict__ res,
+                                            __nv_bfloat16 *__restrict__ y) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (bias != nullptr) {
+    const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (col0 + 8 * q < N) {
+        const uint4 b4 = __ldg(bp + q);
+        v[8 * q + 0] += bf16_lo(b4.x); v[8 * q + 1] += bf16_hi(b4.x);
+        v[8 * q + 2] += bf16_lo(b4.y); v[8 * q + 3] += bf16_hi(b4.y);
+        v[8 * q + 4] += bf16_lo(b4.z); v[8 * q + 5] += bf16_hi(b4.z);
+        v[8 * q + 6] += bf16_lo(b4.w); v[8 * q + 7] += bf16_hi(b4.w);
+      }
+    }
+  }
+  if (EPI == kEpiGelu) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gemm::gelu_fast(v[i]);
+  }
+  if (EPI == kEpiResidual) {
+    const uint4 *rp = reinterpret_cast<const uint4 *>(res + size_t(row) * N + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (col0 + 8 * q < N) {
+        const uint4 r4 = __ldg(rp + q);
+        v[8 * q + 0] += bf16_lo(r4.x); v[8 * q + 1] += bf16_hi(r4.x);
+        v[8 * q + 2] += bf16_lo(r4.y); v[8 * q + 3] += bf16_hi(r4.y);
+        v[8 * q + 4] += bf16_lo(r4.z); v[8 * q + 5] += bf16_hi(r4.z);
+        v[8 * q + 6] += bf16_lo(r4.w); v[8 * q + 7] += bf16_hi(r4.w);
+      }
+    }
+  }
+  uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + 8 * q < N) {
+      uint4 o;
+      o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+      o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+      o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+      o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+      yp[q] = o;
+    }
+  }
+}
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
@@ -195,55 +251,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
+        __syncwarp();
         tmem_ld32(tmem + (uint32_t(quarter * 32) << 16) + uint32_t(a * BN + c * 32), r);
         tmem_ld_wait();
         const int col0 = nb * BN + c * 32;
-        if (!row_ok || col0 >= N) continue;
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        if (bias != nullptr) {
-          const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (col0 + 8 * q < N) {
-              const uint4 b4 = __ldg(bp + q);
-              v[8 * q + 0] += bf16_lo(b4.x); v[8 * q + 1] += bf16_hi(b4.x);
-              v[8 * q + 2] += bf16_lo(b4.y); v[8 * q + 3] += bf16_hi(b4.y);
-              v[8 * q + 4] += bf16_lo(b4.z); v[8 * q + 5] += bf16_hi(b4.z);
-              v[8 * q + 6] += bf16_lo(b4.w); v[8 * q + 7] += bf16_hi(b4.w);
-            }
-          }
-        }
-        if (EPI == kEpiGelu) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i]);
-        }
-        if (EPI == kEpiResidual) {
-          const uint4 *rp = reinterpret_cast<const uint4 *>(res + size_t(row) * N + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (col0 + 8 * q < N) {
-              const uint4 r4 = __ldg(rp + q);
-              v[8 * q + 0] += bf16_lo(r4.x); v[8 * q + 1] += bf16_hi(r4.x);
-              v[8 * q + 2] += bf16_lo(r4.y); v[8 * q + 3] += bf16_hi(r4.y);
-              v[8 * q + 4] += bf16_lo(r4.z); v[8 * q + 5] += bf16_hi(r4.z);
-              v[8 * q + 6] += bf16_lo(r4.w); v[8 * q + 7] += bf16_hi(r4.w);
-            }
-          }
-        }
-        uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (col0 + 8 * q < N) {
-            uint4 o;
-            o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-            o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-            o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-            o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-            yp[q] = o;
-          }
-        }
+        if (row_ok && col0 < N) store_chunk<EPI>(r, row, col0, N, bias, res, y);
       }
       tc_fence_before();
       __syncwarp();
@@ -256,6 +268,186 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, CF::kTmemCols);
+  }
+  if (threadIdx.x == 0 && bars->abort_flag) report_status(status, kDevTimeout);
+}
+
+// ---------------------------------------------------------------- CTA-pair GEMM
+// The same GEMM with 256-row output tiles computed by a pair of CTAs (a
+// cluster of 2 on two SMs) through tcgen05.mma.cta_group::2: each CTA loads
+// its own 128 rows of x and half of the tile's BN rows of w, the leader CTA
+// (rank 0) issues one M = 256 MMA that reads both CTAs' shared memory, and
+// each CTA's TMEM receives its 128 output rows.  Per SM this halves the w
+// bytes per FLOP compared with a 128 x BN tile on one SM.
+//   - full[s] lives in the leader and counts both CTAs' TMA bytes;
+//   - empty[s] and acc_full[a] are signalled in both CTAs by one multicast
+//     tcgen05.commit of the leader;
+//   - acc_empty[a] lives in the leader and collects the 4 epilogue warps of
+//     both CTAs (remote arrivals from the peer).
+// No load uses cluster multicast.
+namespace gemm {
+template <int BN>
+struct Cfg2 {
+  static constexpr uint32_t kBHalfBytes = (BN / 2) * BK * 2;
+  static constexpr uint32_t kStageBytes = kATileBytes + kBHalfBytes;  // per CTA
+  static constexpr int kStages = int((196u * 1024u) / kStageBytes) > 8 ? 8
+                                                                         : int((196u * 1024u) / kStageBytes);
+  static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 1024;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(256, BN);
+};
+}  // namespace gemm
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(gemm::kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
+                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status) {
+  using namespace gemm;
+  using CF = Cfg2<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  Bars *bars = reinterpret_cast<Bars *>(smem + size_t(CF::kStages) * CF::kStageBytes);
+  volatile int *abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_cta_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int num_m = (M + 2 * BM - 1) / (2 * BM), num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int k_blocks = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CF::kStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], 8);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&bars->tmem_base, CF::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+        const int mb = tile % num_m, nb = tile / num_m;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t *sa = smem + size_t(stage) * CF::kStageBytes;
+          if (leader) mbar_arrive_expect_tx(&bars->full[stage], 2 * CF::kStageBytes);
+          const uint32_t full_leader = map_to_cta(&bars->full[stage], 0);
+          tma_load_2d_pair(sa, &tmA, full_leader, kb * BK, mb * 2 * BM + int(rank) * BM);
+          tma_load_2d_pair(sa + kATileBytes, &tmB, full_leader, kb * BK,
+                           nb * BN + int(rank) * (BN / 2));
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == CF::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        if (leader) {
+          for (int s = 0; s < CF::kStages; ++s)
+            if (issued_mask & (1u << s)) drain_wait(&bars->full[s], (issued_parity >> s) & 1);
+        } else {
+          // the peer's copies complete on the leader's barriers: give them time
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 2000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true, any_mma = false;
+      for (int tile = pair; tile < num_tiles && ok; tile += n_pairs, ++it) {
+        const int a = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&bars->acc_empty[a], aphase ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + uint32_t(a * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&bars->full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + size_t(stage) * CF::kStageBytes);
+          const uint32_t sb = sa + kATileBytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = smem_desc(sa + k * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(sb + k * 32, 16, 1024, 2);
+            mma_bf16_ss_pair(d_tmem, ad, bd, CF::kIdesc, (kb | k) != 0);
+          }
+          any_mma = true;
+          mma_commit_pair_mc(&bars->empty[stage], 0x3);
+          if (++stage == CF::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&bars->acc_full[a], 0x3);
+      }
+      if (!ok && any_mma) {
+        mma_commit_pair_mc(&bars->drain, 0x1);
+        drain_wait(&bars->drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int row_in_tile = int(rank) * BM + quarter * 32 + lane;
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int a = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
+      tc_fence_after();
+      const int row = mb * 2 * BM + row_in_tile;
+      const bool row_ok = row < M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tmem + (uint32_t(quarter * 32) << 16) + uint32_t(a * BN + c * 32), r);
+        tmem_ld_wait();
+        const int col0 = nb * BN + c * 32;
+        if (row_ok && col0 < N) store_chunk<EPI>(r, row, col0, N, bias, res, y);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_cta(&bars->acc_empty[a], 0));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no CTA leaves while the pair's MMAs may still read its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, CF::kTmemCols);
   }
   if (threadIdx.x == 0 && bars->abort_flag) report_status(status, kDevTimeout);
 }
@@ -315,34 +507,113 @@ static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap 
   }
 }
 
-// Tile width: the narrower tile wins when it needs fewer full waves of
-// output tiles (makespan ~ waves x tile width).
-static int choose_bn(int M, int N, int num_sms) {
-  const int mt = (M + gemm::BM - 1) / gemm::BM;
-  long best_cost = -1;
-  int best = 256;
-  for (int bn : {256, 128}) {
-    const long tiles = long(mt) * ((N + bn - 1) / bn);
-    const long waves = (tiles + num_sms - 1) / num_sms;
-    const long cost = waves * bn;
-    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = bn; }
+template <int BN, int EPI>
+static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
+                               const void *res, void *y, int M, int N, int K, int num_sms,
+                               int *status, cudaStream_t st) {
+  using CF = gemm::Cfg2<BN>;
+  auto kern = gemm_tc2_kernel<BN, EPI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.dynamicSmemBytes = CF::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // SM pairs that can hold one CTA pair each (clusters live inside a GPC)
+  static int max_clusters = -1;
+  if (max_clusters < 0) {
+    cfg.gridDim = dim3(2 * (num_sms / 2));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms / 2;
+    }
+    max_clusters = n;
   }
-  return best;
+  const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + BN - 1) / BN);
+  cfg.gridDim = dim3(2 * std::max(1, std::min(tiles, max_clusters)));
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, static_cast<const __nv_bfloat16 *>(b),
+                            static_cast<const __nv_bfloat16 *>(res),
+                            static_cast<__nv_bfloat16 *>(y), M, N, K, status);
+}
+
+template <int BN>
+static cudaError_t launch_pair_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
+                                   const void *b, const void *res, void *y, int M, int N, int K,
+                                   int num_sms, int *status, cudaStream_t st) {
+  switch (epi) {
+    case kEpiGelu:
+      return launch_pair<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+    case kEpiResidual:
+      return launch_pair<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+    default:
+      return launch_pair<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+  }
+}
+
+// GEMM variant = (CTAs per MMA, tile width).  Cost model: output tiles are
+// processed in rounds over the SMs (or SM pairs); per 64-deep k-block an SM
+// spends max(MMA clocks, operand bytes / kIngestBytesPerClk).  The per-SM
+// operand ingest rate is the measured limiter of these GEMMs (their tensor
+// pipe idles while shared memory waits for TMA data), so the pair variant,
+// which loads half of w per SM, usually wins.
+struct GemmVariant {
+  int pair, bn;
+};
+constexpr double kIngestBytesPerClk = 45.0;
+
+static GemmVariant choose_variant(int M, int N, int K, int num_sms) {
+  if (const char *f = getenv("VIT_GEMM_TILE")) {  // e.g. "2x192": tuning and tests
+    int p = 0, bn = 0;
+    if (sscanf(f, "%dx%d", &p, &bn) == 2 && (p == 1 || p == 2) &&
+        (bn == 128 || bn == 256 || (p == 2 && bn == 192)))
+      return {p, bn};
+  }
+  const GemmVariant cands[5] = {{1, 128}, {1, 256}, {2, 128}, {2, 192}, {2, 256}};
+  const int kb = (K + gemm::BK - 1) / gemm::BK;
+  double best = -1;
+  GemmVariant pick = {1, 128};
+  for (const auto &v : cands) {
+    if (v.pair == 2 && M <= gemm::BM) continue;  // a single row tile: no pair to share
+    const long tiles = long((M + v.pair * gemm::BM - 1) / (v.pair * gemm::BM)) *
+                       ((N + v.bn - 1) / v.bn);
+    const long units = num_sms / v.pair;
+    const long rounds = (tiles + units - 1) / units;
+    const double mma = 2.0 * v.bn;
+    const double ingest = (16384.0 + 128.0 * v.bn / v.pair) / kIngestBytesPerClk;
+    const double cost = double(rounds) * kb * std::max(mma, ingest);
+    if (best < 0 || cost < best) { best = cost; pick = v; }
+  }
+  return pick;
 }
 
 cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
                            int M, int N, int K, int epi, int num_sms, int *status,
                            cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  const int bn = choose_bn(M, N, num_sms);
+  const GemmVariant v = choose_variant(M, N, K, num_sms);
+  const int b_rows = v.pair == 2 ? v.bn / 2 : v.bn;
   CUtensorMap ta, tb;
   if (encode_tensor_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, uint64_t(K) * 2,
                            gemm::BK, gemm::BM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (encode_tensor_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, uint64_t(K) * 2,
-                           gemm::BK, bn, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                           gemm::BK, b_rows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  if (bn == 256) return launch_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+  if (v.pair == 2) {
+    if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+    if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+    return launch_pair_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+  }
+  if (v.bn == 256) return launch_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
   return launch_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
 }
 
