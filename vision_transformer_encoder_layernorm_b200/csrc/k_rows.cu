@@ -34,28 +34,41 @@ struct Vec4<__nv_bfloat16> {
 };
 
 // One warp per row; lane l holds vectors l, l+32, l+64, ... (MAXV at most).
+// gamma and beta, the same for every row, are staged once per block in
+// shared memory while the rows are being loaded.
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(256) layernorm_warp_kernel(
     const T *__restrict__ x, T *__restrict__ y, const T *__restrict__ gamma,
     const T *__restrict__ beta, int rows, int cols, float eps) {
   using V = Vec4<T>;
+  using R = typename V::raw;
+  extern __shared__ __align__(16) unsigned char ln_smem[];
+  const int nvec = cols >> 2;  // cols % 4 == 0 checked by the host
+  R *sg = reinterpret_cast<R *>(ln_smem);
+  R *sb = sg + nvec;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (row >= rows) return;
-  const int nvec = cols >> 2;  // cols % 4 == 0 checked by the host
-  const typename V::raw *xr = reinterpret_cast<const typename V::raw *>(x + size_t(row) * cols);
+  const bool active = row < rows;
+  const R *xr = reinterpret_cast<const R *>(x + size_t(active ? row : 0) * cols);
   float v[MAXV][4];
-  float s = 0.f;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int c = lane + 32 * i;
-    if (c < nvec) {
+    if (active && c < nvec) {
       V::unpack(xr[c], v[i]);
-      s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
     } else {
       v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.f;
     }
   }
+  const R *gr = reinterpret_cast<const R *>(gamma);
+  const R *br = reinterpret_cast<const R *>(beta);
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    sg[i] = __ldg(gr + i);
+    sb[i] = __ldg(br + i);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   const float mean = s / float(cols);
@@ -74,16 +87,16 @@ __global__ void __launch_bounds__(256) layernorm_warp_kernel(
 #pragma unroll
   for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
   const float rstd = 1.0f / sqrtf(q / float(cols) + eps);
-  const typename V::raw *gr = reinterpret_cast<const typename V::raw *>(gamma);
-  const typename V::raw *br = reinterpret_cast<const typename V::raw *>(beta);
-  typename V::raw *yr = reinterpret_cast<typename V::raw *>(y + size_t(row) * cols);
+  __syncthreads();
+  if (!active) return;
+  R *yr = reinterpret_cast<R *>(y + size_t(row) * cols);
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int c = lane + 32 * i;
     if (c < nvec) {
       float g[4], b[4], o[4];
-      V::unpack(gr[c], g);
-      V::unpack(br[c], b);
+      V::unpack(sg[c], g);
+      V::unpack(sb[c], b);
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[e] = (v[i][e] - mean) * rstd * g[e] + b[e];
       yr[c] = V::pack(o);
@@ -98,16 +111,21 @@ cudaError_t launch_layernorm_t(const void *x, void *y, const void *g, const void
   const int warps = 8;
   dim3 grid((rows + warps - 1) / warps), block(32 * warps);
   const int nvec = cols / 4;
+  const size_t smem = 2 * size_t(nvec) * sizeof(typename Vec4<T>::raw);
   auto xp = static_cast<const T *>(x);
   auto yp = static_cast<T *>(y);
   auto gp = static_cast<const T *>(g);
   auto bp = static_cast<const T *>(b);
   if (nvec <= 32 * 4)
-    layernorm_warp_kernel<T, 4><<<grid, block, 0, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    layernorm_warp_kernel<T, 4><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+  else if (nvec <= 32 * 9)
+    layernorm_warp_kernel<T, 9><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
   else if (nvec <= 32 * 12)
-    layernorm_warp_kernel<T, 12><<<grid, block, 0, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    layernorm_warp_kernel<T, 12><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+  else if (nvec <= 32 * 24)
+    layernorm_warp_kernel<T, 24><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
   else
-    layernorm_warp_kernel<T, 32><<<grid, block, 0, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    layernorm_warp_kernel<T, 32><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
   return cudaGetLastError();
 }
 
@@ -196,46 +214,101 @@ cudaError_t launch_positions(const ImageTable &tab, int n_images, int cu_offset_
 }
 
 // ---------------------------------------------------------------- 2D RoPE
-// In place on the Q and K parts of qkv [T, 3, H, d].  One thread per
-// (token, Q|K, head, half, pair).
+// In place on the Q and K parts of qkv [T, 3, H, d].  One thread rotates one
+// half-head (d/2 contiguous elements: dims [0, d/2) by the row, [d/2, d) by
+// the column; dim j pairs with j + d/4), read and written with 8-byte vector
+// accesses.  The cos/sin of a block's tokens are computed once into shared
+// memory (2 axes x d/4 frequencies per token) and shared by its 2*H Q/K heads.
 template <typename T>
-__global__ void rope2d_kernel(T *__restrict__ qkv, const int32_t *__restrict__ pos, int T_,
-                              int H, int d, const __grid_constant__ RopeFreqs fr) {
-  const int quarter = d >> 2;                  // pairs per half
-  const long long per_tok = 2LL * H * 2 * quarter;
-  const long long total = (long long)T_ * per_tok;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int t = int(i / per_tok);
-    int r = int(i - (long long)t * per_tok);
-    const int j = r % quarter;
-    r /= quarter;
-    const int axis = r & 1;
-    r >>= 1;
-    const int h = r % H;
-    const int part = r / H;  // 0 Q, 1 K
-    const float p = float(pos[2 * t + axis]);
-    float sn, cs;
-    sincospif(p * fr.wpi[j], &sn, &cs);
-    T *base = qkv + (size_t)t * 3 * H * d + (size_t)part * H * d + (size_t)h * d + axis * 2 * quarter;
-    const float a = to_f32(base[j]), b = to_f32(base[j + quarter]);
-    base[j] = from_f32<T>(a * cs - b * sn);
-    base[j + quarter] = from_f32<T>(b * cs + a * sn);
+struct Vec8B;  // 8 bytes of T
+template <>
+struct Vec8B<__nv_bfloat16> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float *f) {
+    const uint2 r = *reinterpret_cast<const uint2 *>(p);
+    f[0] = bf16_lo(r.x); f[1] = bf16_hi(r.x); f[2] = bf16_lo(r.y); f[3] = bf16_hi(r.y);
   }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float *f) {
+    *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+  }
+};
+template <>
+struct Vec8B<float> {
+  static constexpr int N = 2;
+  static __device__ __forceinline__ void load(const float *p, float *f) {
+    const float2 r = *reinterpret_cast<const float2 *>(p);
+    f[0] = r.x; f[1] = r.y;
+  }
+  static __device__ __forceinline__ void store(float *p, const float *f) {
+    *reinterpret_cast<float2 *>(p) = make_float2(f[0], f[1]);
+  }
+};
+
+template <typename T, int HALF>
+__global__ void __launch_bounds__(256) rope2d_kernel(T *__restrict__ qkv,
+                                                     const int32_t *__restrict__ pos, int T_,
+                                                     int H, int tok_per_block,
+                                                     const __grid_constant__ RopeFreqs fr) {
+  constexpr int Q4 = HALF / 2;  // pairs per half-head
+  using V = Vec8B<T>;
+  extern __shared__ float2 cs[];  // [tok_per_block][2][Q4] = (cos, sin)
+  const int tok0 = blockIdx.x * tok_per_block;
+  const int n_cs = tok_per_block * 2 * Q4;
+  for (int i = threadIdx.x; i < n_cs; i += blockDim.x) {
+    const int t = tok0 + i / (2 * Q4);
+    const int r = i % (2 * Q4);
+    const int axis = r / Q4, j = r % Q4;
+    float sn = 0.f, c = 1.f;
+    if (t < T_) sincospif(float(pos[2 * t + axis]) * fr.wpi[j], &sn, &c);
+    cs[i] = make_float2(c, sn);
+  }
+  __syncthreads();
+  const int units = 4 * H;  // (Q|K) x head x axis per token
+  const int lt = threadIdx.x / units, u = threadIdx.x % units;
+  const int t = tok0 + lt;
+  if (lt >= tok_per_block || t >= T_) return;
+  const int axis = u & 1, h = (u >> 1) % H, part = u / (2 * H);
+  const int d = 2 * HALF;
+  T *p = qkv + (size_t)t * 3 * H * d + (size_t)part * H * d + (size_t)h * d + axis * HALF;
+  float v[HALF];
+#pragma unroll
+  for (int i = 0; i < HALF; i += V::N) V::load(p + i, v + i);
+  const float2 *tc = cs + (lt * 2 + axis) * Q4;
+#pragma unroll
+  for (int j = 0; j < Q4; ++j) {
+    const float2 k = tc[j];
+    const float a = v[j], b = v[j + Q4];
+    v[j] = a * k.x - b * k.y;
+    v[j + Q4] = b * k.x + a * k.y;
+  }
+#pragma unroll
+  for (int i = 0; i < HALF; i += V::N) V::store(p + i, v + i);
+}
+
+template <typename T>
+static cudaError_t launch_rope_t(void *qkv, const int32_t *pos, int T_, int H, int d,
+                                 const RopeFreqs &fr, cudaStream_t st) {
+  const int units = 4 * H;
+  const int tpb = std::max(1, 256 / units);
+  const int threads = tpb * units;
+  if (threads > 1024) return cudaErrorInvalidValue;
+  const int blocks = (T_ + tpb - 1) / tpb;
+  const size_t smem = sizeof(float2) * tpb * 2 * (d / 4);
+  T *q = static_cast<T *>(qkv);
+  switch (d) {
+    case 64: rope2d_kernel<T, 32><<<blocks, threads, smem, st>>>(q, pos, T_, H, tpb, fr); break;
+    case 72: rope2d_kernel<T, 36><<<blocks, threads, smem, st>>>(q, pos, T_, H, tpb, fr); break;
+    case 128: rope2d_kernel<T, 64><<<blocks, threads, smem, st>>>(q, pos, T_, H, tpb, fr); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_rope2d(int dtype, void *qkv, const int32_t *pos, int T_, int H, int d,
                           const RopeFreqs &fr, cudaStream_t st) {
   if (T_ == 0) return cudaSuccess;
-  const long long total = (long long)T_ * 2 * H * (d / 2);
-  const int threads = 256;
-  const int blocks = int(std::min<long long>((total + threads - 1) / threads, 148LL * 16));
-  if (dtype == kF32)
-    rope2d_kernel<float><<<blocks, threads, 0, st>>>(static_cast<float *>(qkv), pos, T_, H, d, fr);
-  else
-    rope2d_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(static_cast<__nv_bfloat16 *>(qkv),
-                                                            pos, T_, H, d, fr);
-  return cudaGetLastError();
+  return dtype == kF32 ? launch_rope_t<float>(qkv, pos, T_, H, d, fr, st)
+                       : launch_rope_t<__nv_bfloat16>(qkv, pos, T_, H, d, fr, st);
 }
 
 }  // namespace vit
