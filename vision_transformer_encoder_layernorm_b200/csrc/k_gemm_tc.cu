@@ -11,8 +11,10 @@
 //               128-byte swizzled, into a STAGES-deep shared-memory ring.
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (128 x BN x 16)
 //               into one of two TMEM accumulators and commits stage releases.
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time (thread = row),
-//               bias / GELU / residual in fp32, bf16 stores.
+//   warps 2-9   epilogue: two warps per TMEM lane quarter (thread = row), each
+//               draining half of the tile's columns 32 at a time; each warp
+//               stages its bias half in shared memory, residual loads are
+//               overlapped with the TMEM load; fp32 math, bf16 stores.
 // The two accumulators let the epilogue of tile i overlap the main loop of
 // tile i+1.  Every wait is bounded (see mbar_wait); on a timeout the kernel
 // drains its in-flight copies, frees TMEM and reports through `status`.
@@ -28,7 +30,8 @@ namespace vit {
 namespace gemm {
 constexpr int BM = 128;
 constexpr int BK = 64;                     // one 128-byte swizzle atom of bf16
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // 2 role warps + 8 epilogue warps
+constexpr int kEpiWarps = 8;
 constexpr uint32_t kATileBytes = BM * BK * 2;  // 16 KB
 
 template <int BN>
@@ -37,12 +40,12 @@ struct Cfg {
   static constexpr uint32_t kStageBytes = kATileBytes + kBTileBytes;
   static constexpr int kStages = (BN >= 256) ? 4 : 6;
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
-  // ring + barriers/bookkeeping + 1 KB alignment slack
-  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 1024;
+  // ring + barriers/bookkeeping + bias slots (8 warps x 128 bf16) + 1 KB alignment slack
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 2048 + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
 };
 
-struct __align__(8) Bars {
+struct __align__(16) Bars {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t acc_full[2];
@@ -73,44 +76,37 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 
 }  // namespace gemm
 
-// One 32-column slice of one output row: fp32 accumulators r -> + bias ->
-// epilogue op -> bf16 stores (columns at or past N are skipped, N % 8 == 0).
+// One 32-column slice of one output row: fp32 accumulators r + bias (from
+// shared memory) -> epilogue op (+ residual rv, already loaded) -> bf16 stores
+// (columns at or past N are skipped; N % 8 == 0).
 template <int EPI>
 __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, int col0, int N,
-                                            const __nv_bfloat16 *__restrict__ bias,
-                                            const __nv_bfloat16 *__restrict__ res,
+                                            const __nv_bfloat16 *bias_s, const uint4 (&rv)[4],
                                             __nv_bfloat16 *__restrict__ y) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  if (bias != nullptr) {
-    const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
+  const uint4 *bp = reinterpret_cast<const uint4 *>(bias_s);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (col0 + 8 * q < N) {
-        const uint4 b4 = __ldg(bp + q);
-        v[8 * q + 0] += bf16_lo(b4.x); v[8 * q + 1] += bf16_hi(b4.x);
-        v[8 * q + 2] += bf16_lo(b4.y); v[8 * q + 3] += bf16_hi(b4.y);
-        v[8 * q + 4] += bf16_lo(b4.z); v[8 * q + 5] += bf16_hi(b4.z);
-        v[8 * q + 6] += bf16_lo(b4.w); v[8 * q + 7] += bf16_hi(b4.w);
-      }
-    }
+  for (int q = 0; q < 4; ++q) {
+    const uint4 b4 = bp[q];
+    v[8 * q + 0] += bf16_lo(b4.x); v[8 * q + 1] += bf16_hi(b4.x);
+    v[8 * q + 2] += bf16_lo(b4.y); v[8 * q + 3] += bf16_hi(b4.y);
+    v[8 * q + 4] += bf16_lo(b4.z); v[8 * q + 5] += bf16_hi(b4.z);
+    v[8 * q + 6] += bf16_lo(b4.w); v[8 * q + 7] += bf16_hi(b4.w);
   }
   if (EPI == kEpiGelu) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gemm::gelu_fast(v[i]);
   }
   if (EPI == kEpiResidual) {
-    const uint4 *rp = reinterpret_cast<const uint4 *>(res + size_t(row) * N + col0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      if (col0 + 8 * q < N) {
-        const uint4 r4 = __ldg(rp + q);
-        v[8 * q + 0] += bf16_lo(r4.x); v[8 * q + 1] += bf16_hi(r4.x);
-        v[8 * q + 2] += bf16_lo(r4.y); v[8 * q + 3] += bf16_hi(r4.y);
-        v[8 * q + 4] += bf16_lo(r4.z); v[8 * q + 5] += bf16_hi(r4.z);
-        v[8 * q + 6] += bf16_lo(r4.w); v[8 * q + 7] += bf16_hi(r4.w);
-      }
+      const uint4 r4 = rv[q];
+      v[8 * q + 0] += bf16_lo(r4.x); v[8 * q + 1] += bf16_hi(r4.x);
+      v[8 * q + 2] += bf16_lo(r4.y); v[8 * q + 3] += bf16_hi(r4.y);
+      v[8 * q + 4] += bf16_lo(r4.z); v[8 * q + 5] += bf16_hi(r4.z);
+      v[8 * q + 6] += bf16_lo(r4.w); v[8 * q + 7] += bf16_hi(r4.w);
     }
   }
   uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
@@ -125,6 +121,56 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, in
       yp[q] = o;
     }
   }
+}
+
+// Epilogue of one accumulator (one output tile) by the 8 epilogue warps:
+// epilogue warp e (= warp - 2) drains TMEM lane quarter (warp & 3), i.e. one
+// row per thread, and column half (e >> 2) of the tile.  The warp's half of
+// the tile bias was staged in its shared-memory slot (bias_w).
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int lane, int row,
+                                              bool row_ok, int n0, int N,
+                                              const __nv_bfloat16 *bias_w,
+                                              const __nv_bfloat16 *__restrict__ res,
+                                              __nv_bfloat16 *__restrict__ y) {
+  constexpr int kChunks = BN / 64;  // 32-column chunks per half
+  const int quarter = warp & 3, half = (warp - 2) >> 2;
+#pragma unroll 1
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = half * kChunks + i;
+    const int col0 = n0 + c * 32;
+    const bool ok = row_ok && col0 < N;
+    uint32_t r[32];
+    __syncwarp();
+    tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c * 32), r);
+    uint4 rv[4];
+    if (EPI == kEpiResidual && ok) {  // in flight together with the TMEM load
+      const uint4 *rp = reinterpret_cast<const uint4 *>(res + size_t(row) * N + col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) rv[q] = (col0 + 8 * q < N) ? __ldg(rp + q) : make_uint4(0, 0, 0, 0);
+    }
+    tmem_ld_wait();
+    if (ok) store_chunk<EPI>(r, row, col0, N, bias_w + i * 32, rv, y);
+  }
+}
+
+// Each epilogue warp stages the bias of its own column half of the tile
+// [n0 + half*BN/2, n0 + (half+1)*BN/2) in its own shared-memory slot (zeros
+// past N or without bias).  Only the warp itself reads the slot, so warp-level
+// synchronisation suffices (no barrier across epilogue warps, which could not
+// be left safely if a bounded wait ran out).
+template <int BN>
+__device__ __forceinline__ void stage_bias_warp(__nv_bfloat16 *bias_w, const __nv_bfloat16 *bias,
+                                                int n0, int N, int warp, int lane) {
+  const int half = (warp - 2) >> 2;
+  __syncwarp();  // previous tile's reads of the slot are done
+  if (lane < BN / 16) {
+    const int col = n0 + half * (BN / 2) + lane * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (bias != nullptr && col < N) v = __ldg(reinterpret_cast<const uint4 *>(bias + col));
+    reinterpret_cast<uint4 *>(bias_w)[lane] = v;
+  }
+  __syncwarp();
 }
 
 template <int BN, int EPI>
@@ -152,7 +198,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 4);
+      mbar_init(&bars->acc_empty[a], kEpiWarps);
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -237,26 +283,19 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
-    const int row_in_tile = quarter * 32 + lane;
+    const int row_in_tile = (warp & 3) * 32 + lane;
+    __nv_bfloat16 *bias_w = reinterpret_cast<__nv_bfloat16 *>(bars + 1) + (warp - 2) * 128;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
+      stage_bias_warp<BN>(bias_w, bias, nb * BN, N, warp, lane);
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * BM + row_in_tile;
-      const bool row_ok = row < M;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tmem + (uint32_t(quarter * 32) << 16) + uint32_t(a * BN + c * 32), r);
-        tmem_ld_wait();
-        const int col0 = nb * BN + c * 32;
-        if (row_ok && col0 < N) store_chunk<EPI>(r, row, col0, N, bias, res, y);
-      }
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N,
+                             bias_w, res, y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
@@ -282,7 +321,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 //   - full[s] lives in the leader and counts both CTAs' TMA bytes;
 //   - empty[s] and acc_full[a] are signalled in both CTAs by one multicast
 //     tcgen05.commit of the leader;
-//   - acc_empty[a] lives in the leader and collects the 4 epilogue warps of
+//   - acc_empty[a] lives in the leader and collects the 8 epilogue warps of
 //     both CTAs (remote arrivals from the peer).
 // No load uses cluster multicast.
 namespace gemm {
@@ -293,7 +332,7 @@ struct Cfg2 {
   static constexpr int kStages = int((196u * 1024u) / kStageBytes) > 8 ? 8
                                                                          : int((196u * 1024u) / kStageBytes);
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
-  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 1024;
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 2048 + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(256, BN);
 };
 }  // namespace gemm
@@ -326,7 +365,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 8);
+      mbar_init(&bars->acc_empty[a], 2 * kEpiWarps);
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -417,26 +456,19 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int quarter = warp & 3;
-    const int row_in_tile = int(rank) * BM + quarter * 32 + lane;
+    const int row_in_tile = int(rank) * BM + (warp & 3) * 32 + lane;
+    __nv_bfloat16 *bias_w = reinterpret_cast<__nv_bfloat16 *>(bars + 1) + (warp - 2) * 128;
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
+      stage_bias_warp<BN>(bias_w, bias, nb * BN, N, warp, lane);
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * 2 * BM + row_in_tile;
-      const bool row_ok = row < M;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tmem + (uint32_t(quarter * 32) << 16) + uint32_t(a * BN + c * 32), r);
-        tmem_ld_wait();
-        const int col0 = nb * BN + c * 32;
-        if (row_ok && col0 < N) store_chunk<EPI>(r, row, col0, N, bias, res, y);
-      }
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N,
+                             bias_w, res, y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_cta(&bars->acc_empty[a], 0));
