@@ -18,6 +18,16 @@ constexpr int kDevOk = 0;
 constexpr int kDevTimeout = 6;
 constexpr int kDevBounds = 7;
 
+// Programmatic dependent launch: a kernel launched with launch_pdl() may
+// start while the previous kernel of its stream is still running.  It calls
+// pdl_trigger() at entry (its own dependents may then be scheduled; a grid is
+// only launched once every CTA of its predecessor has started, so this cannot
+// starve the running grid of SMs) and pdl_wait() before its first access to
+// global memory, which returns once the previous grid has completed and its
+// writes are visible.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void report_status(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }

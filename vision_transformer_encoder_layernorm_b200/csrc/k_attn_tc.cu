@@ -18,6 +18,8 @@
 //   6-9      softmax warpgroup of query tile 1
 //   10-11    (ROPE only) rotate each own-key K tile in shared memory
 // TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,..), O1 [384,..).
+// The two softmax warpgroups alternate (an mbarrier handoff per key tile), so
+// one uses the exp unit while the tensor core serves the other.
 // head_dim 72 is computed as 80 (4 MMA k-steps from a 64-column 128B-swizzled
 // chunk, 1 from a 16-column 32B-swizzled chunk); Q's columns 72..79 are zeroed
 // in shared memory so the neighbouring head's values there contribute 0.
@@ -53,6 +55,7 @@ struct __align__(8) Bars {
   uint64_t q_ready[2];
   uint64_t k_full[4], v_full[4], kv_empty[4], k_ready[4];
   uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t turn[2];  // softmax warpgroups take turns (ping-pong)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -144,6 +147,8 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
   volatile int *abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  pdl_trigger();
+  pdl_wait();
   // ---- work item: pairs of query tiles, longest sequences' last pairs first
   const int S = gridDim.x / (prm.n_pairs * prm.H);
   const int b = blockIdx.x;
@@ -166,6 +171,7 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 128);
       mbar_init(&bars->o_done[t], 1);
+      mbar_init(&bars->turn[t], 128);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -356,10 +362,21 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
       // P.V -- so the row sum costs no instruction here (and sums exactly the
       // bf16 P the numerator uses).  head_dim 128 sums in registers.
       constexpr bool kSumByMma = (HD == 72);
+      // 32-column chunks of each score row whose exponentials run on the FMA
+      // pipe instead of the special-function unit (1 of 4: a 25% share)
+      constexpr int kPolyChunks = 1;
       float m = -INFINITY;
       uint64_t l2[4] = {0, 0, 0, 0};  // packed partial row sums (head_dim 128)
       for (int j = 0; j < n_kv && ok; ++j) {
         if (!mbar_wait(&bars->s_full[t], j & 1, abort_flag)) { ok = false; break; }
+        // ping-pong: with two query tiles the warpgroups run their softmax
+        // phases alternately (the exp unit serves one while the tensor core
+        // works for the other); warpgroup 0 goes first in every round
+        const bool pingpong = n_tiles_q == 2;
+        if (pingpong && !mbar_wait(&bars->turn[t], (j & 1) ^ (t == 0 ? 1u : 0u), abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const int nvalid = j < n_pre ? min(kBlockK, prm.P - j * kBlockK)
                                      : min(kBlockK, len - (j - n_pre) * kBlockK);
@@ -427,16 +444,23 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])),
-                             sc2, nm2),
-                      x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const uint64_t xa = f2_fma(
+                f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sc2, nm2);
+            float p0, p1;
+            if (c < kPolyChunks) {  // this share of the exponentials runs on the FMA pipe
+              exp2_poly_x2(xa, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(xa, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             if (!kSumByMma) l2[i & 3] = f2_add(l2[i & 3], f2_pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
+            pk[i] = pack_bf16x2_alu(p0, p1);
           }
           tmem_st16(s_addr + c * 16, pk);
         }
+        if (pingpong) mbar_arrive(&bars->turn[t ^ 1]);
         if (kSumByMma && t == 0) {
           // ones in V's column 72 of this key tile (the first padding column)
           const int st = j % NS;
@@ -529,8 +553,8 @@ static cudaError_t launch_hd(const CUtensorMap *maps, const attn::Params &prm, i
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, ROPE ? 384 : 320, CF::kSmem, st>>>(maps[0], maps[1], maps[2], maps[3], prm, fr);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(ROPE ? 384 : 320), CF::kSmem, st, 1, maps[0], maps[1],
+                    maps[2], maps[3], prm, fr);
 }
 
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,

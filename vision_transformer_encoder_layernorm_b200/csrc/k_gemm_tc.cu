@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const int num_tiles = num_m * num_n;
   const int k_blocks = (K + BK - 1) / BK;
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < CF::kStages; ++s) {
       mbar_init(&bars->full[s], 1);
@@ -216,6 +217,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  pdl_wait();  // inputs of this GEMM are written by the previous kernel
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -358,6 +360,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const int num_tiles = num_m * num_n;
   const int k_blocks = (K + BK - 1) / BK;
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < CF::kStages; ++s) {
       mbar_init(&bars->full[s], 1);
@@ -383,6 +386,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   cluster_sync_all();  // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  pdl_wait();  // inputs of this GEMM are written by the previous kernel
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -519,10 +523,9 @@ static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const
   if (e != cudaSuccess) return e;
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + BN - 1) / BN);
   const int grid = std::max(1, std::min(tiles, num_sms));
-  kern<<<grid, gemm::kThreads, CF::kSmemBytes, st>>>(
-      ta, tb, static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-      static_cast<__nv_bfloat16 *>(y), M, N, K, status);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb,
+                    static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
+                    static_cast<__nv_bfloat16 *>(y), M, N, K, status);
 }
 
 template <int BN>
@@ -571,10 +574,10 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
     max_clusters = n;
   }
   const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + BN - 1) / BN);
-  cfg.gridDim = dim3(2 * std::max(1, std::min(tiles, max_clusters)));
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, static_cast<const __nv_bfloat16 *>(b),
-                            static_cast<const __nv_bfloat16 *>(res),
-                            static_cast<__nv_bfloat16 *>(y), M, N, K, status);
+  return launch_pdl(kern, dim3(2 * std::max(1, std::min(tiles, max_clusters))),
+                    dim3(gemm::kThreads), CF::kSmemBytes, st, 2, ta, tb,
+                    static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
+                    static_cast<__nv_bfloat16 *>(y), M, N, K, status);
 }
 
 template <int BN>

@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(256) layernorm_warp_kernel(
   using V = Vec4<T>;
   using R = typename V::raw;
   extern __shared__ __align__(16) unsigned char ln_smem[];
+  pdl_trigger();
+  pdl_wait();
   const int nvec = cols >> 2;  // cols % 4 == 0 checked by the host
   R *sg = reinterpret_cast<R *>(ln_smem);
   R *sb = sg + nvec;
@@ -117,15 +119,15 @@ cudaError_t launch_layernorm_t(const void *x, void *y, const void *g, const void
   auto gp = static_cast<const T *>(g);
   auto bp = static_cast<const T *>(b);
   if (nvec <= 32 * 4)
-    layernorm_warp_kernel<T, 4><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    return launch_pdl(layernorm_warp_kernel<T, 4>, grid, block, smem, st, 1, xp, yp, gp, bp, rows, cols, eps);
   else if (nvec <= 32 * 9)
-    layernorm_warp_kernel<T, 9><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    return launch_pdl(layernorm_warp_kernel<T, 9>, grid, block, smem, st, 1, xp, yp, gp, bp, rows, cols, eps);
   else if (nvec <= 32 * 12)
-    layernorm_warp_kernel<T, 12><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    return launch_pdl(layernorm_warp_kernel<T, 12>, grid, block, smem, st, 1, xp, yp, gp, bp, rows, cols, eps);
   else if (nvec <= 32 * 24)
-    layernorm_warp_kernel<T, 24><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    return launch_pdl(layernorm_warp_kernel<T, 24>, grid, block, smem, st, 1, xp, yp, gp, bp, rows, cols, eps);
   else
-    layernorm_warp_kernel<T, 32><<<grid, block, smem, st>>>(xp, yp, gp, bp, rows, cols, eps);
+    return launch_pdl(layernorm_warp_kernel<T, 32>, grid, block, smem, st, 1, xp, yp, gp, bp, rows, cols, eps);
   return cudaGetLastError();
 }
 
@@ -141,6 +143,8 @@ cudaError_t launch_layernorm(int dtype, const void *x, void *y, const void *g, c
 template <typename U>
 __global__ void merge2x2_kernel(const __grid_constant__ ImageTable tab, const U *__restrict__ x,
                                 U *__restrict__ y, int units_per_token) {
+  pdl_trigger();
+  pdl_wait();
   const ImageEntry im = tab.img[blockIdx.y];
   const int half_w = im.cols >> 1;
   const long long out_tokens = (long long)(im.rows >> 1) * half_w;
@@ -168,20 +172,20 @@ cudaError_t launch_merge2x2(const ImageTable &tab, int n_images, const void *x, 
     const int upt = int(row_bytes / 16);
     long long units = max_out_tokens * 4 * upt;
     int bx = int(std::min<long long>((units + threads - 1) / threads, 4096));
-    merge2x2_kernel<uint4><<<dim3(bx, n_images), threads, 0, st>>>(
-        tab, static_cast<const uint4 *>(x), static_cast<uint4 *>(y), upt);
+    return launch_pdl(merge2x2_kernel<uint4>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
+                      static_cast<const uint4 *>(x), static_cast<uint4 *>(y), upt);
   } else if (row_bytes % 4 == 0) {
     const int upt = int(row_bytes / 4);
     long long units = max_out_tokens * 4 * upt;
     int bx = int(std::min<long long>((units + threads - 1) / threads, 4096));
-    merge2x2_kernel<uint32_t><<<dim3(bx, n_images), threads, 0, st>>>(
-        tab, static_cast<const uint32_t *>(x), static_cast<uint32_t *>(y), upt);
+    return launch_pdl(merge2x2_kernel<uint32_t>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
+                      static_cast<const uint32_t *>(x), static_cast<uint32_t *>(y), upt);
   } else {
     const int upt = int(row_bytes / 2);
     long long units = max_out_tokens * 4 * upt;
     int bx = int(std::min<long long>((units + threads - 1) / threads, 4096));
-    merge2x2_kernel<uint16_t><<<dim3(bx, n_images), threads, 0, st>>>(
-        tab, static_cast<const uint16_t *>(x), static_cast<uint16_t *>(y), upt);
+    return launch_pdl(merge2x2_kernel<uint16_t>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
+                      static_cast<const uint16_t *>(x), static_cast<uint16_t *>(y), upt);
   }
   return cudaGetLastError();
 }
@@ -252,6 +256,8 @@ __global__ void __launch_bounds__(256) rope2d_kernel(T *__restrict__ qkv,
   constexpr int Q4 = HALF / 2;  // pairs per half-head
   using V = Vec8B<T>;
   extern __shared__ float2 cs[];  // [tok_per_block][2][Q4] = (cos, sin)
+  pdl_trigger();
+  pdl_wait();
   const int tok0 = blockIdx.x * tok_per_block;
   const int n_cs = tok_per_block * 2 * Q4;
   for (int i = threadIdx.x; i < n_cs; i += blockDim.x) {
@@ -296,12 +302,11 @@ static cudaError_t launch_rope_t(void *qkv, const int32_t *pos, int T_, int H, i
   const size_t smem = sizeof(float2) * tpb * 2 * (d / 4);
   T *q = static_cast<T *>(qkv);
   switch (d) {
-    case 64: rope2d_kernel<T, 32><<<blocks, threads, smem, st>>>(q, pos, T_, H, tpb, fr); break;
-    case 72: rope2d_kernel<T, 36><<<blocks, threads, smem, st>>>(q, pos, T_, H, tpb, fr); break;
-    case 128: rope2d_kernel<T, 64><<<blocks, threads, smem, st>>>(q, pos, T_, H, tpb, fr); break;
+    case 64: return launch_pdl(rope2d_kernel<T, 32>, dim3(blocks), dim3(threads), smem, st, 1, q, pos, T_, H, tpb, fr);
+    case 72: return launch_pdl(rope2d_kernel<T, 36>, dim3(blocks), dim3(threads), smem, st, 1, q, pos, T_, H, tpb, fr);
+    case 128: return launch_pdl(rope2d_kernel<T, 64>, dim3(blocks), dim3(threads), smem, st, 1, q, pos, T_, H, tpb, fr);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_rope2d(int dtype, void *qkv, const int32_t *pos, int T_, int H, int d,

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <stdlib.h>
+
 #include <algorithm>
 
 #include "common.cuh"
@@ -77,6 +79,41 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,
                                 float scale, const RopeFreqs &fr, int num_sms, int *status,
                                 cudaStream_t st);
+
+// Launches `kern` with programmatic dependent launch allowed (and a cluster
+// of cluster_x CTAs when cluster_x > 1).  Kernels launched this way call
+// pdl_wait() before touching global memory.  VIT_NO_PDL=1 in the environment
+// turns the attribute off (plain stream order).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, unsigned cluster_x, Args... args) {
+  static const bool pdl_off = [] {
+    const char *e = getenv("VIT_NO_PDL");
+    return e != nullptr && e[0] == '1';
+  }();
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (!pdl_off) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once).
 CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,

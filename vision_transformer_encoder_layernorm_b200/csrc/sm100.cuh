@@ -276,6 +276,44 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// 2^x for two fp32 lanes on the FMA pipe (offloads the special-function
+// unit).  x = j + f with j = round(x) (the 1.5 * 2^23 shift trick) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted in this project
+// (iteratively reweighted least squares on Chebyshev nodes, max relative
+// error 7.5e-5 on [-1/2, 1/2]); 2^j inserted into the exponent field.
+// x is clamped at -125 so the exponent never leaves the normal range.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float &y0, float &y1) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  a = fmaxf(a, -125.0f);
+  b = fmaxf(b, -125.0f);
+  const uint64_t x = f2_pack(a, b);
+  const uint64_t shift = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, shift);                         // j in the low mantissa bits
+  const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);    // x - j, exact
+  uint64_t p = f2_fma(f2_pack(0.055171653f, 0.055171653f), f, f2_pack(0.24261112f, 0.24261112f));
+  p = f2_fma(p, f, f2_pack(0.69326099f, 0.69326099f));
+  p = f2_fma(p, f, f2_pack(0.99992807f, 0.99992807f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// Two non-negative finite fp32 -> packed bf16x2 (low half = lo) with integer
+// ALU operations only: add half an ulp of bf16 (round half up), keep the high
+// 16 bits of each (byte permute).  Keeps the conversion off the pipe that
+// also executes the exponentials.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // 2^x on the special-function unit (approximate, flush-to-zero).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
