@@ -129,12 +129,65 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, in
 // the tile bias was staged in its shared-memory slot (bias_w).
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int lane, int row,
-                                              bool row_ok, int n0, int N,
+                                              bool row_ok, int n0, int N, const RopeEpi &re,
                                               const __nv_bfloat16 *bias_w,
                                               const __nv_bfloat16 *__restrict__ res,
                                               __nv_bfloat16 *__restrict__ y) {
   constexpr int kChunks = BN / 64;  // 32-column chunks per half
   const int quarter = warp & 3, half = (warp - 2) >> 2;
+  if constexpr (EPI == kEpiRope) {
+    // one whole head (BN/2 columns) per warp: bias, then the 2D rotation of
+    // Q/K pairs (j, j + HD/4) in each half of the head, in fp32
+    constexpr int HD = BN / 2, Q4 = HD / 4, NF = HD / 32;
+    const int col0 = n0 + half * HD;
+    const uint32_t base = tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(half * HD);
+    uint32_t r[NF][32];
+    uint32_t r8[8];
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < NF; ++c) tmem_ld32(base + c * 32, r[c]);
+    if (HD % 32) tmem_ld8(base + NF * 32, r8);
+    tmem_ld_wait();
+    if (!(row_ok && col0 < N)) return;
+    float v[HD];
+#pragma unroll
+    for (int i = 0; i < HD; ++i) {
+      const uint32_t bits = i < NF * 32 ? r[i / 32][i % 32] : r8[i - NF * 32];
+      v[i] = __uint_as_float(bits);
+    }
+    const uint32_t *bw = reinterpret_cast<const uint32_t *>(bias_w);
+#pragma unroll
+    for (int i = 0; i < HD / 2; ++i) {
+      const uint32_t b2 = bw[i];
+      v[2 * i] += bf16_lo(b2);
+      v[2 * i + 1] += bf16_hi(b2);
+    }
+    if (col0 < re.rot_cols) {
+      const int2 pr = reinterpret_cast<const int2 *>(re.pos)[row];
+#pragma unroll
+      for (int axis = 0; axis < 2; ++axis) {
+        const float p = float(axis == 0 ? pr.x : pr.y);
+#pragma unroll
+        for (int j = 0; j < Q4; ++j) {
+          float sn, cs;
+          sincospif(p * re.fr.wpi[j], &sn, &cs);
+          const float a = v[axis * (HD / 2) + j], b = v[axis * (HD / 2) + Q4 + j];
+          v[axis * (HD / 2) + j] = a * cs - b * sn;
+          v[axis * (HD / 2) + Q4 + j] = b * cs + a * sn;
+        }
+      }
+    }
+    uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
+#pragma unroll
+    for (int u = 0; u < HD / 8; ++u) {
+      uint4 o;
+      o.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+      o.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+      o.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+      o.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+      yp[u] = o;
+    }
+  } else {
 #pragma unroll 1
   for (int i = 0; i < kChunks; ++i) {
     const int c = half * kChunks + i;
@@ -151,6 +204,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
     }
     tmem_ld_wait();
     if (ok) store_chunk<EPI>(r, row, col0, N, bias_w + i * 32, rv, y);
+  }
   }
 }
 
@@ -177,7 +231,8 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
-                   __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status) {
+                   __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status,
+                   const __grid_constant__ RopeEpi re) {
   using namespace gemm;
   using CF = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -296,7 +351,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * BM + row_in_tile;
-      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N,
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, re,
                              bias_w, res, y);
       tc_fence_before();
       __syncwarp();
@@ -343,7 +398,8 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
-                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status) {
+                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status,
+                   const __grid_constant__ RopeEpi re) {
   using namespace gemm;
   using CF = Cfg2<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -471,7 +527,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * 2 * BM + row_in_tile;
-      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N,
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, re,
                              bias_w, res, y);
       tc_fence_before();
       __syncwarp();
@@ -515,7 +571,7 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const vo
 template <int BN, int EPI>
 static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
                              const void *res, void *y, int M, int N, int K, int num_sms,
-                             int *status, cudaStream_t st) {
+                             int *status, cudaStream_t st, const RopeEpi &re) {
   using CF = gemm::Cfg<BN>;
   auto kern = gemm_tc_kernel<BN, EPI>;
   cudaError_t e =
@@ -525,7 +581,7 @@ static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const
   const int grid = std::max(1, std::min(tiles, num_sms));
   return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb,
                     static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-                    static_cast<__nv_bfloat16 *>(y), M, N, K, status);
+                    static_cast<__nv_bfloat16 *>(y), M, N, K, status, re);
 }
 
 template <int BN>
@@ -534,18 +590,18 @@ static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap 
                               int num_sms, int *status, cudaStream_t st) {
   switch (epi) {
     case kEpiGelu:
-      return launch_bn<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+      return launch_bn<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{});
     case kEpiResidual:
-      return launch_bn<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+      return launch_bn<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{});
     default:
-      return launch_bn<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+      return launch_bn<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{});
   }
 }
 
 template <int BN, int EPI>
 static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
                                const void *res, void *y, int M, int N, int K, int num_sms,
-                               int *status, cudaStream_t st) {
+                               int *status, cudaStream_t st, const RopeEpi &re) {
   using CF = gemm::Cfg2<BN>;
   auto kern = gemm_tc2_kernel<BN, EPI>;
   cudaError_t e =
@@ -577,20 +633,21 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
   return launch_pdl(kern, dim3(2 * std::max(1, std::min(tiles, max_clusters))),
                     dim3(gemm::kThreads), CF::kSmemBytes, st, 2, ta, tb,
                     static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-                    static_cast<__nv_bfloat16 *>(y), M, N, K, status);
+                    static_cast<__nv_bfloat16 *>(y), M, N, K, status, re);
 }
 
 template <int BN>
 static cudaError_t launch_pair_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
                                    const void *b, const void *res, void *y, int M, int N, int K,
                                    int num_sms, int *status, cudaStream_t st) {
+  const RopeEpi none{};
   switch (epi) {
     case kEpiGelu:
-      return launch_pair<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+      return launch_pair<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st, none);
     case kEpiResidual:
-      return launch_pair<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+      return launch_pair<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st, none);
     default:
-      return launch_pair<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st);
+      return launch_pair<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st, none);
   }
 }
 
@@ -632,9 +689,13 @@ static GemmVariant choose_variant(int M, int N, int K, int num_sms) {
 
 cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
                            int M, int N, int K, int epi, int num_sms, int *status,
-                           cudaStream_t st) {
+                           cudaStream_t st, const RopeEpi *rope) {
   if (M == 0 || N == 0) return cudaSuccess;
-  const GemmVariant v = choose_variant(M, N, K, num_sms);
+  GemmVariant v = choose_variant(M, N, K, num_sms);
+  if (epi == kEpiRope) {  // tiles of two whole heads on a CTA pair
+    if (rope == nullptr || (rope->head_dim != 72 && rope->head_dim != 128)) return cudaErrorInvalidValue;
+    v = {2, 2 * rope->head_dim};
+  }
   const int b_rows = v.pair == 2 ? v.bn / 2 : v.bn;
   CUtensorMap ta, tb;
   if (encode_tensor_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, uint64_t(K) * 2,
@@ -643,6 +704,11 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
   if (encode_tensor_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, uint64_t(K) * 2,
                            gemm::BK, b_rows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (epi == kEpiRope) {
+    if (v.bn == 144)
+      return launch_pair<144, kEpiRope>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
+    return launch_pair<256, kEpiRope>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
+  }
   if (v.pair == 2) {
     if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
     if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);

@@ -58,6 +58,17 @@ cudaError_t launch_rope2d(int dtype, void *qkv, const int32_t *pos, int T, int H
 constexpr int kEpiBias = 0;
 constexpr int kEpiGelu = 1;
 constexpr int kEpiResidual = 2;
+constexpr int kEpiRope = 3;  // bias, then 2D RoPE on columns < rot_cols (QKV projection)
+
+// Arguments of the RoPE epilogue: the GEMM's tile width is 2 * head_dim so
+// each epilogue warp holds whole heads; output columns [0, rot_cols) (Q and
+// K) are rotated by the row's position pos[row] = (r, c).
+struct RopeEpi {
+  const int32_t *pos;
+  int rot_cols;
+  int head_dim;
+  RopeFreqs fr;
+};
 
 // SIMT GEMM (fp32 FFMA; fp32 or bf16 storage): y = epi(x w^T + b).
 cudaError_t launch_gemm_simt(int dtype, const void *x, const void *w, const void *b,
@@ -73,7 +84,7 @@ cudaError_t launch_attention_simt(int dtype, const void *qkv, void *o, const Seq
 struct GemmPlan;
 cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
                            int M, int N, int K, int epi, int num_sms, int *status,
-                           cudaStream_t st);
+                           cudaStream_t st, const RopeEpi *rope = nullptr);
 
 // tcgen05 flash attention, bf16, head_dim 72 or 128.
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,

@@ -4,8 +4,8 @@
 //
 // Layer (pre-LN reading of the KLiteInfer README, "视觉算子" op list):
 //   h  = LN1(x)                      layernorm kernel
-//   qkv = h Wqkv^T + bqkv            GEMM (bias epilogue)
-//   qkv[Q,K] = RoPE2D(qkv[Q,K])      rope kernel, in place (workspace)
+//   qkv = h Wqkv^T + bqkv            GEMM (bias epilogue; bf16: + 2D RoPE on Q, K)
+//   qkv[Q,K] = RoPE2D(qkv[Q,K])      fp32 mode: rope kernel, in place (workspace)
 //   a  = Attn(qkv)                   attention kernel (varlen, prefix)
 //   x1 = x + a Wo^T + bo             GEMM (bias + residual epilogue)
 //   h  = LN2(x1)                     layernorm kernel
@@ -134,10 +134,11 @@ SeqArgs to_seq_args(const vit_seqs *s, bool with_pos) {
 }
 
 cudaError_t run_linear(vit_ctx *ctx, int kind, const void *x, const void *w, const void *b,
-                       const void *res, void *y, int M, int N, int K, int epi, cudaStream_t st) {
+                       const void *res, void *y, int M, int N, int K, int epi, cudaStream_t st,
+                       const RopeEpi *rope = nullptr) {
   return counted(ctx, kind, st, [&] {
     if (ctx->cfg.dtype == VIT_F32) return launch_gemm_simt(kF32, x, w, b, res, y, M, N, K, epi, st);
-    return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st);
+    return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st, rope);
   });
 }
 
@@ -203,10 +204,20 @@ vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, v
     });
   };
   if (ln(x, w->ln1_g, w->ln1_b)) return VIT_ERR_CUDA;
+  // bf16: the QKV GEMM rotates Q and K in its epilogue (tiles of two whole
+  // heads); fp32: a separate RoPE pass over the projection output
+  const bool fused_rope = rope && dt == kBF16 && (c.head_dim == 72 || c.head_dim == 128);
+  RopeEpi re{};
+  if (fused_rope) {
+    re.pos = seqs->pos_rc;
+    re.rot_cols = 2 * C;
+    re.head_dim = c.head_dim;
+    re.fr = ctx->fr;
+  }
   if (run_linear(ctx, VIT_K_GEMM_QKV, ws.h, w->w_qkv, w->b_qkv, nullptr, ws.qkv, T, 3 * C, C,
-                 kEpiBias, st))
+                 fused_rope ? kEpiRope : kEpiBias, st, fused_rope ? &re : nullptr))
     return VIT_ERR_CUDA;
-  if (rope && counted(ctx, VIT_K_ROPE, st, [&] {
+  if (rope && !fused_rope && counted(ctx, VIT_K_ROPE, st, [&] {
         return launch_rope2d(dt, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st);
       }))
     return VIT_ERR_CUDA;
