@@ -11,15 +11,16 @@
 // Prefix K/V (LightX2V NeoPP README, "KV file layout": [2, seq, kv_heads, d]
 // per layer) is read through its own TMA descriptors as the first key tiles.
 //
-// CTA = (sequence, head, two 128-row query tiles).  Warps:
+// CTA = (sequence, head, two 128-row query tiles), 20 warps:
 //   0        TMA producer (Q tiles once, then K and V tiles through a ring)
 //   1        TMEM allocator; one lane issues all tcgen05.mma
-//   2-5      softmax warpgroup of query tile 0   (thread = query row)
-//   6-9      softmax warpgroup of query tile 1
-//   10-11    (ROPE only) rotate each own-key K tile in shared memory
+//   2-3      (ROPE only) rotate each own-key K tile in shared memory
+//   4-11     softmax of query tile 0, 12-19 of query tile 1: two threads per
+//            query row, one per 64-column half of the score row; the pair
+//            swaps partial row maxima through shared memory each key tile
+// Four softmax warps per SM sub-partition keep the exp unit, the FMA and the
+// integer pipes fed while a warp waits on a TMEM load or a barrier.
 // TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,..), O1 [384,..).
-// The two softmax warpgroups alternate (an mbarrier handoff per key tile), so
-// one uses the exp unit while the tensor core serves the other.
 // head_dim 72 is computed as 80 (4 MMA k-steps from a 64-column 128B-swizzled
 // chunk, 1 from a 16-column 32B-swizzled chunk); Q's columns 72..79 are zeroed
 // in shared memory so the neighbouring head's values there contribute 0.
@@ -43,7 +44,8 @@ struct Cfg {
   static constexpr uint32_t kKOff = 2 * kTile;
   static constexpr uint32_t kVOff = kKOff + kStages * kTile;
   static constexpr uint32_t kBarOff = kVOff + kStages * kTile;
-  static constexpr size_t kSmem = size_t(kBarOff) + 1024 + 1024;
+  static constexpr uint32_t kXOff = kBarOff + 512;             // row-max exchange [2][2][128] f32
+  static constexpr size_t kSmem = size_t(kXOff) + 2048 + 1024;
   static constexpr uint32_t kTmemS = 0, kTmemO = 256;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, kBlockK, 0, 0);
   static constexpr uint32_t kIdescPV0 = idesc_bf16_f32(128, HD == 72 ? 64 : 128, 0, 1);
@@ -55,11 +57,14 @@ struct __align__(8) Bars {
   uint64_t q_ready[2];
   uint64_t k_full[4], v_full[4], kv_empty[4], k_ready[4];
   uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t turn[2];  // softmax warpgroups take turns (ping-pong)
+  uint64_t xchg[2][4];  // per (query tile, lane quarter): the 64 threads of a row pair
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
+constexpr int kThreads = 640;
 
 struct Params {
   int H, C, Hkv, P, n_pairs;
@@ -95,20 +100,25 @@ __device__ __forceinline__ uint32_t unit_offset(int r, int u) {
 template <int HD>
 __device__ __forceinline__ void rope_row_smem(uint8_t *tile, int r, int pr, int pc,
                                               const RopeFreqs &fr) {
-  constexpr int NU = HD / 8;  // 16-byte units holding real data (9 or 16)
-  uint32_t w[NU * 4];
-#pragma unroll
-  for (int u = 0; u < NU; ++u) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(tile + unit_offset<HD>(r, u));
-    w[4 * u + 0] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
-  }
   constexpr int Q4 = HD / 4;
+  // one axis at a time: the 16-byte units holding dims [axis HD/2, axis HD/2 + HD/2)
+  // (head_dim 72: unit 4 holds the end of the row half and the start of the
+  // column half, and is read back after the first axis wrote it)
 #pragma unroll
   for (int axis = 0; axis < 2; ++axis) {
+    constexpr int kUnits = (HD / 2 + 7) / 8 + (HD % 16 ? 1 : 0);
+    const int u0 = (axis * (HD / 2)) / 8;
+    uint32_t w[kUnits * 4];
+#pragma unroll
+    for (int k = 0; k < kUnits; ++k) {
+      if (u0 + k >= HD / 8) continue;
+      const uint4 v = *reinterpret_cast<const uint4 *>(tile + unit_offset<HD>(r, u0 + k));
+      w[4 * k + 0] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+    }
     const float p = float(axis == 0 ? pr : pc);
 #pragma unroll
     for (int j = 0; j < Q4; ++j) {
-      const int d1 = axis * (HD / 2) + j, d2 = d1 + Q4;
+      const int d1 = axis * (HD / 2) + j - u0 * 8, d2 = d1 + Q4;  // dims relative to unit u0
       float sn, cs;
       sincospif(p * fr.wpi[j], &sn, &cs);
       const uint32_t w1 = w[d1 >> 1], w2 = w[d2 >> 1];
@@ -121,17 +131,64 @@ __device__ __forceinline__ void rope_row_smem(uint8_t *tile, int r, int pr, int 
       const uint32_t w2n = w[d2 >> 1];
       w[d2 >> 1] = (d2 & 1) ? ((w2n & 0xFFFFu) | (hb << 16)) : ((w2n & 0xFFFF0000u) | hb);
     }
-  }
 #pragma unroll
-  for (int u = 0; u < NU; ++u)
-    *reinterpret_cast<uint4 *>(tile + unit_offset<HD>(r, u)) =
-        make_uint4(w[4 * u + 0], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    for (int k = 0; k < kUnits; ++k) {
+      if (u0 + k >= HD / 8) continue;
+      *reinterpret_cast<uint4 *>(tile + unit_offset<HD>(r, u0 + k)) =
+          make_uint4(w[4 * k + 0], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    }
+  }
+}
+
+// A bounded mbarrier wait whose outcome is the same for all 32 lanes (the
+// warp-collective TMEM accesses and votes that follow need a converged warp).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Normalises one half of a finished output row (O / l) and stores it as bf16:
+// half 0 writes the first ceil(HD/16) 16-byte units of the row, half 1 the
+// rest.  head_dim 72 reads l from O column 72 (accumulated by the tensor core);
+// head_dim 128 gets it from the caller.  orow == nullptr: load only (row past
+// the sequence end; the TMEM loads are warp-collective).
+template <int HD, int HALF>
+__device__ __forceinline__ void store_o_half(uint32_t o_addr, float l_sum, __nv_bfloat16 *orow) {
+  constexpr int NU = HD / 8;
+  constexpr int U0 = HALF ? (NU + 1) / 2 : 0, U1 = HALF ? NU : (NU + 1) / 2;
+  constexpr int C0 = (U0 * 8) / 16, C1 = (U1 * 8 - 1) / 16;  // 16-column TMEM chunks used
+  uint32_t ov[Cfg<HD>::HDP / 16][16];
+  __syncwarp();
+#pragma unroll
+  for (int c = C0; c <= C1; ++c) tmem_ld16(o_addr + c * 16, ov[c]);
+  if constexpr (HD == 72 && C1 < 4) tmem_ld16(o_addr + 64, ov[4]);
+  tmem_ld_wait();
+  float l = l_sum;
+  if constexpr (HD == 72) l = __uint_as_float(ov[4][8]);
+  const float inv = 1.0f / l;
+  const uint64_t inv2 = f2_pack(inv, inv);
+  if (orow == nullptr) return;
+#pragma unroll
+  for (int u = U0; u < U1; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = u * 8 + 2 * e;
+      float a, b;
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(ov[col / 16][col % 16]),
+                               __uint_as_float(ov[col / 16][col % 16 + 1])),
+                       inv2),
+                a, b);
+      w[e] = pack_bf16x2(a, b);
+    }
+    *reinterpret_cast<uint4 *>(orow + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 }  // namespace attn
 
 template <int HD, bool ROPE>
-__global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
+__global__ void __launch_bounds__(attn::kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_x0,
                         const __grid_constant__ CUtensorMap tm_x1,
                         const __grid_constant__ CUtensorMap tm_p0,
@@ -169,9 +226,9 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_ready[t], 128);
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], 128);
+      mbar_init(&bars->p_full[t], 256);
       mbar_init(&bars->o_done[t], 1);
-      mbar_init(&bars->turn[t], 128);
+      for (int q = 0; q < 4; ++q) mbar_init(&bars->xchg[t][q], 64);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -336,73 +393,87 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
         drain_wait(&bars->drain, 0);
       }
     }
-  } else if (warp < 10) {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;       // query tile of this warpgroup
+    const int sw = warp - 4;
+    const int t = sw >> 3;               // query tile of this warp
+    const int half = (sw >> 2) & 1;      // which 64 of the 128 score columns
     const int quarter = warp & 3;        // TMEM lane quarter
     const int r = quarter * 32 + lane;   // query row inside the tile
     if (t < n_tiles_q) {
       const int qrow = q0 + t * kBlockQ + r;  // row inside the sequence
-      bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
-      if (ok) {
-        uint8_t *qt = smem + CF::kQOff + t * CF::kTile;
-        if (ROPE && qrow < len)
-          rope_row_smem<HD>(qt, r, prm.pos[2 * (seg0 + qrow)], prm.pos[2 * (seg0 + qrow) + 1], fr);
-        if (HD == 72)  // zero the 8 padding columns 72..79 (logical unit 9)
-          *reinterpret_cast<uint4 *>(qt + unit_offset<HD>(r, 9)) = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
+      bool ok = true;
+      if (half == 0) {
+        ok = mbar_wait(&bars->q_full, 0, abort_flag);
+        if (ok) {
+          uint8_t *qt = smem + CF::kQOff + t * CF::kTile;
+          if (ROPE && qrow < len)
+            rope_row_smem<HD>(qt, r, prm.pos[2 * (seg0 + qrow)], prm.pos[2 * (seg0 + qrow) + 1], fr);
+          if (HD == 72)  // zero the 8 padding columns 72..79 (logical unit 9)
+            *reinterpret_cast<uint4 *>(qt + unit_offset<HD>(r, 9)) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(&bars->q_ready[t]);
       }
-      mbar_arrive(&bars->q_ready[t]);
+      ok = __all_sync(0xffffffffu, ok);
       const uint32_t lane_base = uint32_t(quarter * 32) << 16;
       const uint32_t s_addr = tmem + lane_base + CF::kTmemS + t * 128;
       const uint32_t o_addr = tmem + lane_base + CF::kTmemO + t * 128;
+      float *xv = reinterpret_cast<float *>(smem + CF::kXOff) + t * 256;  // [half][row]
+      uint64_t *xb = &bars->xchg[t][quarter];
       const float sl2 = prm.scale_log2;
       // head_dim 72: the softmax denominator is accumulated by the tensor core
       // as O column 72 -- V's first padding column is set to 1.0 before each
-      // P.V -- so the row sum costs no instruction here (and sums exactly the
-      // bf16 P the numerator uses).  head_dim 128 sums in registers.
+      // P.V -- so the row sum costs no instruction here and sums exactly the
+      // bf16 P the numerator uses.  That also lets P be rounded toward zero
+      // (one byte permute per pair): the rounding's mean cancels between
+      // numerator and denominator and its spread equals round-to-nearest's.
+      // head_dim 128 sums in registers and rounds P to nearest.
       constexpr bool kSumByMma = (HD == 72);
-      // 32-column chunks of each score row whose exponentials run on the FMA
-      // pipe instead of the special-function unit (1 of 4: a 25% share)
-      constexpr int kPolyChunks = 1;
+      // pairs of this thread's 64 exponentials that run on the FMA pipe
+      // instead of the special-function unit (8 of 32: a 25% share)
+      constexpr int kPolyPairs = 8;
+      constexpr int kOC = CF::HDP / 16;         // 16-column chunks of O
+      constexpr int kOCHalf = (kOC + 1) / 2;   // rescaled by half 0; the rest by half 1
+      const int oc_lo = half ? kOCHalf : 0, oc_hi = half ? kOC : kOCHalf;
       float m = -INFINITY;
-      uint64_t l2[4] = {0, 0, 0, 0};  // packed partial row sums (head_dim 128)
+      uint64_t l2[2] = {0, 0};  // packed partial row sums (head_dim 128)
       for (int j = 0; j < n_kv && ok; ++j) {
-        if (!mbar_wait(&bars->s_full[t], j & 1, abort_flag)) { ok = false; break; }
-        // ping-pong: with two query tiles the warpgroups run their softmax
-        // phases alternately (the exp unit serves one while the tensor core
-        // works for the other); warpgroup 0 goes first in every round
-        const bool pingpong = n_tiles_q == 2;
-        if (pingpong && !mbar_wait(&bars->turn[t], (j & 1) ^ (t == 0 ? 1u : 0u), abort_flag)) {
-          ok = false;
-          break;
-        }
+        if (!warp_wait(&bars->s_full[t], j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const int nvalid = j < n_pre ? min(kBlockK, prm.P - j * kBlockK)
-                                     : min(kBlockK, len - (j - n_pre) * kBlockK);
-        uint32_t s[4][32];
+        const int nvalid = (j < n_pre ? min(kBlockK, prm.P - j * kBlockK)
+                                      : min(kBlockK, len - (j - n_pre) * kBlockK)) -
+                           half * 64;  // valid keys among this thread's 64 columns
+        uint32_t s[2][32];
         __syncwarp();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, s[c]);
+        tmem_ld32(s_addr + half * 64, s[0]);
+        tmem_ld32(s_addr + half * 64 + 32, s[1]);
         tmem_ld_wait();
-        if (nvalid < kBlockK) {  // keys past the sequence end: -inf, so p = 0
+        if (nvalid < 64) {  // keys past the sequence end: -inf, so p = 0
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               if (c * 32 + i >= nvalid) s[c][i] = 0xFF800000u;
         }
-        // row max: four independent chains of 3-input max
-        float mc[4];
+        float mc[2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float a = __uint_as_float(s[c][0]);
 #pragma unroll
           for (int i = 1; i < 31; i += 2)
             a = fmax3(a, __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
           mc[c] = fmaxf(a, __uint_as_float(s[c][31]));
         }
-        const float m_tile = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]) * sl2;
+        // swap partial maxima with the thread that holds the row's other half
+        // (its P columns overlap this half's S columns, so the swap also
+        // orders this thread's TMEM loads before the partner's P stores)
+        xv[half * 128 + r] = fmaxf(mc[0], mc[1]) * sl2;
+        tc_fence_before();
+        mbar_arrive(xb);
+        if (!warp_wait(xb, j & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const float m_tile = fmaxf(xv[r], xv[128 + r]);
         const bool grow = __any_sync(0xffffffffu, m_tile > m + 8.0f);
         if (j == 0) {
           m = m_tile;
@@ -413,10 +484,11 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
           const float m_new = mine ? m_tile : m;
           const float factor = mine ? ex2_approx(m - m_new) : 1.0f;
           const uint64_t f2 = f2_pack(factor, factor);
-          if (!mbar_wait(&bars->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&bars->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < CF::HDP / 16; ++c) {
+          for (int c = 0; c < kOC; ++c) {
+            if (c < oc_lo || c >= oc_hi) continue;
             uint32_t v[16];
             __syncwarp();
             tmem_ld16(o_addr + c * 16, v);
@@ -434,20 +506,21 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
           tmem_st_wait();
           if (!kSumByMma)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) l2[k] = f2_mul(l2[k], f2);
+            for (int k = 0; k < 2; ++k) l2[k] = f2_mul(l2[k], f2);
           m = m_new;
         }
-        // p = 2^(s*scale*log2e - m) two at a time; bf16 P into S's first 64 columns
+        // p = 2^(s*scale*log2e - m) two at a time; bf16 P of keys
+        // [64 half, 64 half + 64) into S columns [32 half, 32 half + 32)
         const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const uint64_t xa = f2_fma(
                 f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sc2, nm2);
             float p0, p1;
-            if (c < kPolyChunks) {  // this share of the exponentials runs on the FMA pipe
+            if (c * 16 + i < kPolyPairs) {  // this share of the exponentials runs on the FMA pipe
               exp2_poly_x2(xa, p0, p1);
             } else {
               float x0, x1;
@@ -455,16 +528,19 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
             }
-            if (!kSumByMma) l2[i & 3] = f2_add(l2[i & 3], f2_pack(p0, p1));
-            pk[i] = pack_bf16x2_alu(p0, p1);
+            if (kSumByMma) {
+              pk[i] = pack_bf16x2_trunc(p0, p1);
+            } else {
+              l2[i & 1] = f2_add(l2[i & 1], f2_pack(p0, p1));
+              pk[i] = pack_bf16x2_alu(p0, p1);
+            }
           }
-          tmem_st16(s_addr + c * 16, pk);
+          tmem_st16(s_addr + half * 32 + c * 16, pk);
         }
-        if (pingpong) mbar_arrive(&bars->turn[t ^ 1]);
-        if (kSumByMma && t == 0) {
+        if (kSumByMma && t == 0 && half == 0) {
           // ones in V's column 72 of this key tile (the first padding column)
           const int st = j % NS;
-          if (!mbar_wait(&bars->v_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&bars->v_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
           *reinterpret_cast<uint16_t *>(smem + CF::kVOff + st * CF::kTile + unit_offset<HD>(r, 9)) =
               0x3F80u;  // bf16 1.0
           fence_proxy_async_smem();
@@ -473,50 +549,34 @@ __global__ void __launch_bounds__(ROPE ? 384 : 320, 1)
         tc_fence_before();
         mbar_arrive(&bars->p_full[t]);
       }
-      // epilogue: O / l -> bf16 rows of o [T, H, HD]
-      if (ok && mbar_wait(&bars->o_done[t], (n_kv - 1) & 1, abort_flag)) {
+      // epilogue: O / l -> bf16 rows of o [T, H, HD], each thread its half of the row
+      if (ok && warp_wait(&bars->o_done[t], (n_kv - 1) & 1, abort_flag)) {
         tc_fence_after();
-        uint32_t ov[CF::HDP / 16][16];
-        __syncwarp();
-#pragma unroll
-        for (int c = 0; c < CF::HDP / 16; ++c) tmem_ld16(o_addr + c * 16, ov[c]);
-        tmem_ld_wait();
-        float l;
-        if (kSumByMma) {
-          l = __uint_as_float(ov[4][8]);  // O column 72
-        } else {
+        float l = 0.0f;
+        bool have_l = true;
+        if (!kSumByMma) {  // add the two halves' partial sums
           float a, b, c2, d2;
-          f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), a, b);
-          (void)c2;
-          (void)d2;
-          l = a + b;
+          f2_unpack(l2[0], a, b);
+          f2_unpack(l2[1], c2, d2);
+          xv[half * 128 + r] = (a + b) + (c2 + d2);
+          mbar_arrive(xb);
+          have_l = warp_wait(xb, n_kv & 1, abort_flag);
+          l = xv[r] + xv[128 + r];
         }
-        const float inv = 1.0f / l;
-        const uint64_t inv2 = f2_pack(inv, inv);
-        if (qrow < len) {
-          __nv_bfloat16 *orow = prm.o + size_t(seg0 + qrow) * prm.C + size_t(h) * HD;
-#pragma unroll
-          for (int u = 0; u < HD / 8; ++u) {  // 16-byte units of the output row
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int col = u * 8 + 2 * e;
-              float a, b;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(ov[col / 16][col % 16]),
-                                       __uint_as_float(ov[col / 16][col % 16 + 1])),
-                               inv2),
-                        a, b);
-              w[e] = pack_bf16x2(a, b);
-            }
-            *reinterpret_cast<uint4 *>(orow + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+        if (have_l) {
+          __nv_bfloat16 *orow =
+              qrow < len ? prm.o + size_t(seg0 + qrow) * prm.C + size_t(h) * HD : nullptr;
+          if (half == 0)
+            store_o_half<HD, 0>(o_addr, l, orow);
+          else
+            store_o_half<HD, 1>(o_addr, l, orow);
         }
       }
     }
-  } else if (ROPE) {
+  } else if (ROPE && warp < 4) {
     // ------------------------------------------------------------ K rotation
-    // two warps; thread rotates key rows r and r + 64 of each own-key tile
-    const int r0 = (warp - 10) * 32 + lane;
+    // warps 2-3; thread rotates key rows r and r + 64 of each own-key tile
+    const int r0 = (warp - 2) * 32 + lane;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j % NS;
       const uint32_t f = (j / NS) & 1;
@@ -553,7 +613,7 @@ static cudaError_t launch_hd(const CUtensorMap *maps, const attn::Params &prm, i
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(grid), dim3(ROPE ? 384 : 320), CF::kSmem, st, 1, maps[0], maps[1],
+  return launch_pdl(kern, dim3(grid), dim3(attn::kThreads), CF::kSmem, st, 1, maps[0], maps[1],
                     maps[2], maps[3], prm, fr);
 }
 

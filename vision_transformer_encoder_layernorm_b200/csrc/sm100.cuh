@@ -322,6 +322,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
   return r;
 }
 
+// Two non-negative finite fp32 -> packed bf16x2 (low half = lo) rounded
+// toward zero: the high 16 bits of each, one byte permute.
+__device__ __forceinline__ uint32_t pack_bf16x2_trunc(float lo, float hi) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
+  return r;
+}
+
 // 2^x on the special-function unit (approximate, flush-to-zero).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
