@@ -13,17 +13,25 @@
 //
 // CTA = (sequence, head, two 128-row query tiles), 20 warps:
 //   0        TMA producer (Q tiles once, then K and V tiles through a ring)
-//   1        TMEM allocator; one lane issues all tcgen05.mma
-//   2-3      (ROPE only) rotate each own-key K tile in shared memory
+//   1, 2     MMA issuers of query tiles 0 and 1 (one lane each; warp 1 also
+//            owns the TMEM allocation): each follows its own tile's
+//            softmax, so neither tile's MMAs wait behind the other's
+//   3        (ROPE only) rotate each own-key K tile in shared memory
 //   4-11     softmax of query tile 0, 12-19 of query tile 1: two threads per
-//            query row, one per 64-column half of the score row; the pair
-//            swaps partial row maxima through shared memory each key tile
-// Four softmax warps per SM sub-partition keep the exp unit, the FMA and the
-// integer pipes fed while a warp waits on a TMEM load or a barrier.
-// TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,..), O1 [384,..).
+//            query row, one per half of the key tile's score columns; the
+//            pair swaps partial row maxima through shared memory
+// Per query tile t, TMEM holds S_t (fp32 scores of one key tile), P_t (bf16
+// probabilities, its own columns) and O_t.  Because P does not overwrite S,
+// the MMA warp issues S_t(j+1) = Q_t K_{j+1}^T as soon as the softmax threads
+// have loaded S_t(j) into registers: the tensor core computes the next key
+// tile's scores while the exponentials of this one run, and O_t += P_t V_j
+// follows when P_t(j) is stored.  To fit 2 x (S + P + O) in the 512 TMEM
+// columns a key tile has 112 keys at head_dim 72 and 80 at head_dim 128.
 // head_dim 72 is computed as 80 (4 MMA k-steps from a 64-column 128B-swizzled
 // chunk, 1 from a 16-column 32B-swizzled chunk); Q's columns 72..79 are zeroed
 // in shared memory so the neighbouring head's values there contribute 0.
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -31,40 +39,64 @@ namespace vit {
 namespace attn {
 
 constexpr int kBlockQ = 128;
-constexpr int kBlockK = 128;
+constexpr int kThreads = 640;
+
+__host__ __device__ constexpr uint32_t round_up_1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
 template <int HD>
 struct Cfg {
   static constexpr int HDP = HD == 72 ? 80 : 128;            // padded head_dim
-  static constexpr uint32_t kChunk0 = 128 * 128;              // 128 rows x 64 bf16
-  static constexpr uint32_t kChunk1 = HD == 72 ? 128 * 32 : 128 * 128;
-  static constexpr uint32_t kTile = kChunk0 + kChunk1;        // one operand tile
-  static constexpr int kStages = HD == 72 ? 4 : 2;
+  static constexpr int BK = HD == 72 ? 112 : 80;             // keys per key tile
+  static constexpr int HC = BK / 2;                          // score columns per softmax thread
+  static constexpr uint32_t kQChunk0 = kBlockQ * 128;        // 128 rows x 64 bf16
+  static constexpr uint32_t kQChunk1 = HD == 72 ? kBlockQ * 32 : kBlockQ * 128;
+  static constexpr uint32_t kQTile = kQChunk0 + kQChunk1;
+  static constexpr uint32_t kKChunk0 = BK * 128;             // multiple of 1024
+  static constexpr uint32_t kKChunk1 = HD == 72 ? BK * 32 : BK * 128;
+  static constexpr uint32_t kKTile = round_up_1k(kKChunk0 + kKChunk1);
+  // head_dim 72: V is stored as five 16-column 32B-swizzled chunks so that
+  // one N = 80 MMA per k-step covers it (head_dim 128: as K, two 64-column
+  // 128B-swizzled chunks, one N = 128 MMA)
+  static constexpr uint32_t kVChunk = HD == 72 ? BK * 32 : BK * 128;
+  static constexpr int kVChunks = HD == 72 ? 5 : 2;
+  static constexpr int kStages = HD == 72 ? 5 : 3;
   static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kKOff = 2 * kTile;
-  static constexpr uint32_t kVOff = kKOff + kStages * kTile;
-  static constexpr uint32_t kBarOff = kVOff + kStages * kTile;
-  static constexpr uint32_t kXOff = kBarOff + 512;             // row-max exchange [2][2][128] f32
-  static constexpr size_t kSmem = size_t(kXOff) + 2048 + 1024;
-  static constexpr uint32_t kTmemS = 0, kTmemO = 256;
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, kBlockK, 0, 0);
-  static constexpr uint32_t kIdescPV0 = idesc_bf16_f32(128, HD == 72 ? 64 : 128, 0, 1);
-  static constexpr uint32_t kIdescPV1 = idesc_bf16_f32(128, 16, 0, 1);
+  static constexpr uint32_t kKOff = 2 * kQTile;
+  static constexpr uint32_t kVOff = kKOff + kStages * kKTile;
+  static constexpr uint32_t kBarOff = kVOff + kStages * kKTile;
+  static constexpr uint32_t kXOff = kBarOff + 512;             // row-max exchange [2][2][2][128] f32
+  static constexpr size_t kSmem = size_t(kXOff) + 4096 + 1024;
+  // TMEM columns (16-aligned): S0, S1, P0, P1, O0, O1
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = BK;
+  static constexpr uint32_t kTmemP0 = 2 * BK, kTmemP1 = (2 * BK + BK / 2 + 15) / 16 * 16;
+  static constexpr uint32_t kTmemO0 = HD == 72 ? 352 : 256, kTmemO1 = kTmemO0 + (HD == 72 ? 80 : 128);
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BK, 0, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, HDP, 0, 1);
+  __host__ __device__ static constexpr uint32_t tmem_s(int t) { return t ? kTmemS1 : kTmemS0; }
+  __host__ __device__ static constexpr uint32_t tmem_p(int t) { return t ? kTmemP1 : kTmemP0; }
+  __host__ __device__ static constexpr uint32_t tmem_o(int t) { return t ? kTmemO1 : kTmemO0; }
 };
+static_assert(Cfg<72>::kVChunks * Cfg<72>::kVChunk <= Cfg<72>::kKTile &&
+                  Cfg<128>::kVChunks * Cfg<128>::kVChunk <= Cfg<128>::kKTile,
+              "V tile");
+static_assert(Cfg<72>::kSmem <= 232448 && Cfg<128>::kSmem <= 232448, "shared memory");
+static_assert(Cfg<72>::kTmemP1 + Cfg<72>::BK / 2 <= Cfg<72>::kTmemO0 && Cfg<72>::kTmemO1 + 80 <= 512,
+              "TMEM layout, head_dim 72");
+static_assert(Cfg<128>::kTmemP1 + Cfg<128>::BK / 2 <= Cfg<128>::kTmemO0 &&
+                  Cfg<128>::kTmemO1 + 128 <= 512,
+              "TMEM layout, head_dim 128");
 
 struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t q_ready[2];
-  uint64_t k_full[4], v_full[4], kv_empty[4], k_ready[4];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t k_full[5], v_full[5], kv_empty[5], k_ready[5];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t xchg[2][4];  // per (query tile, lane quarter): the 64 threads of a row pair
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort_flag;
 };
-
 static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
-constexpr int kThreads = 640;
 
 struct Params {
   int H, C, Hkv, P, n_pairs;
@@ -83,23 +115,23 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Byte offset of logical 16-byte unit u (0..HDP/8-1) of row r inside an
-// operand tile: chunk 0 (units 0..7) is 128B-swizzled, chunk 1 is 32B-swizzled
-// (head_dim 72, units 8..9) or 128B-swizzled (head_dim 128, units 8..15).
+// operand tile whose chunk 0 takes chunk0 bytes: chunk 0 (units 0..7) is
+// 128B-swizzled, chunk 1 is 32B-swizzled (head_dim 72, units 8..9) or
+// 128B-swizzled (head_dim 128, units 8..15).
 template <int HD>
-__device__ __forceinline__ uint32_t unit_offset(int r, int u) {
-  using CF = Cfg<HD>;
+__device__ __forceinline__ uint32_t unit_offset(int r, int u, uint32_t chunk0) {
   if (u < 8) return uint32_t(r * 128 + ((u ^ (r & 7)) << 4));
   const int v = u - 8;
-  if (HD == 72) return CF::kChunk0 + uint32_t(r * 32 + ((v ^ ((r >> 2) & 1)) << 4));
-  return CF::kChunk0 + uint32_t(r * 128 + ((v ^ (r & 7)) << 4));
+  if (HD == 72) return chunk0 + uint32_t(r * 32 + ((v ^ ((r >> 2) & 1)) << 4));
+  return chunk0 + uint32_t(r * 128 + ((v ^ (r & 7)) << 4));
 }
 
 // Rotates row r of an operand tile in place by 2D RoPE at position (pr, pc):
 // dims [0, HD/2) by pr, [HD/2, HD) by pc; in a half, dim j pairs with j+HD/4.
 // fr.wpi[j] = theta^(-2j/(HD/2)) / pi.
 template <int HD>
-__device__ __forceinline__ void rope_row_smem(uint8_t *tile, int r, int pr, int pc,
-                                              const RopeFreqs &fr) {
+__device__ __forceinline__ void rope_row_smem(uint8_t *tile, uint32_t chunk0, int r, int pr,
+                                              int pc, const RopeFreqs &fr) {
   constexpr int Q4 = HD / 4;
   // one axis at a time: the 16-byte units holding dims [axis HD/2, axis HD/2 + HD/2)
   // (head_dim 72: unit 4 holds the end of the row half and the start of the
@@ -112,7 +144,7 @@ __device__ __forceinline__ void rope_row_smem(uint8_t *tile, int r, int pr, int 
 #pragma unroll
     for (int k = 0; k < kUnits; ++k) {
       if (u0 + k >= HD / 8) continue;
-      const uint4 v = *reinterpret_cast<const uint4 *>(tile + unit_offset<HD>(r, u0 + k));
+      const uint4 v = *reinterpret_cast<const uint4 *>(tile + unit_offset<HD>(r, u0 + k, chunk0));
       w[4 * k + 0] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
     }
     const float p = float(axis == 0 ? pr : pc);
@@ -134,7 +166,7 @@ __device__ __forceinline__ void rope_row_smem(uint8_t *tile, int r, int pr, int 
 #pragma unroll
     for (int k = 0; k < kUnits; ++k) {
       if (u0 + k >= HD / 8) continue;
-      *reinterpret_cast<uint4 *>(tile + unit_offset<HD>(r, u0 + k)) =
+      *reinterpret_cast<uint4 *>(tile + unit_offset<HD>(r, u0 + k, chunk0)) =
           make_uint4(w[4 * k + 0], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
     }
   }
@@ -189,14 +221,18 @@ __device__ __forceinline__ void store_o_half(uint32_t o_addr, float l_sum, __nv_
 
 template <int HD, bool ROPE>
 __global__ void __launch_bounds__(attn::kThreads, 1)
-    attention_tc_kernel(const __grid_constant__ CUtensorMap tm_x0,
-                        const __grid_constant__ CUtensorMap tm_x1,
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q0,
+                        const __grid_constant__ CUtensorMap tm_q1,
+                        const __grid_constant__ CUtensorMap tm_k0,
+                        const __grid_constant__ CUtensorMap tm_k1,
                         const __grid_constant__ CUtensorMap tm_p0,
                         const __grid_constant__ CUtensorMap tm_p1, const attn::Params prm,
                         const __grid_constant__ RopeFreqs fr) {
   using namespace attn;
   using CF = Cfg<HD>;
   constexpr int NS = CF::kStages;
+  constexpr int BK = CF::BK;
+  constexpr int HC = CF::HC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -217,8 +253,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const int q0 = pair * 2 * kBlockQ;
   if (q0 >= len) return;  // uniform across the CTA, before any barrier or TMEM use
   const int n_tiles_q = (len - q0 > kBlockQ) ? 2 : 1;
-  const int n_pre = prm.P > 0 ? (prm.P + kBlockK - 1) / kBlockK : 0;
-  const int n_kv = n_pre + (len + kBlockK - 1) / kBlockK;
+  const int n_pre = prm.P > 0 ? (prm.P + BK - 1) / BK : 0;
+  const int n_kv = n_pre + (len + BK - 1) / BK;
   const int hk = h / (prm.H / prm.Hkv);
 
   if (threadIdx.x == 0) {
@@ -226,6 +262,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_ready[t], 128);
       mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->s_free[t], 256);
       mbar_init(&bars->p_full[t], 256);
       mbar_init(&bars->o_done[t], 1);
       for (int q = 0; q < 4; ++q) mbar_init(&bars->xchg[t][q], 64);
@@ -233,10 +270,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
-      mbar_init(&bars->k_ready[s], 64);
+      mbar_init(&bars->kv_empty[s], n_tiles_q);  // one commit per query tile
+      mbar_init(&bars->k_ready[s], 32);
     }
-    mbar_init(&bars->drain, 1);
+    for (int t = 0; t < 2; ++t) mbar_init(&bars->drain[t], 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -253,27 +290,27 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   auto kv_coords = [&](int j, bool is_v, int &row, int &col, bool &prefix, int &nvalid) {
     if (j < n_pre) {
       prefix = true;
-      row = (seq * 2 + (is_v ? 1 : 0)) * prm.P + j * kBlockK;
+      row = (seq * 2 + (is_v ? 1 : 0)) * prm.P + j * BK;
       col = hk * HD;
-      nvalid = min(kBlockK, prm.P - j * kBlockK);
+      nvalid = min(BK, prm.P - j * BK);
     } else {
       prefix = false;
       const int jj = j - n_pre;
-      row = seg0 + jj * kBlockK;
+      row = seg0 + jj * BK;
       col = (is_v ? 2 : 1) * prm.C + h * HD;
-      nvalid = min(kBlockK, len - jj * kBlockK);
+      nvalid = min(BK, len - jj * BK);
     }
   };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
-      mbar_arrive_expect_tx(&bars->q_full, n_tiles_q * CF::kTile);
+      mbar_arrive_expect_tx(&bars->q_full, n_tiles_q * CF::kQTile);
       for (int t = 0; t < n_tiles_q; ++t) {
-        uint8_t *qt = smem + CF::kQOff + t * CF::kTile;
+        uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
         const int row = seg0 + q0 + t * kBlockQ;
-        tma_load_2d(qt, &tm_x0, &bars->q_full, h * HD, row);
-        tma_load_2d(qt + CF::kChunk0, &tm_x1, &bars->q_full, h * HD + 64, row);
+        tma_load_2d(qt, &tm_q0, &bars->q_full, h * HD, row);
+        tma_load_2d(qt + CF::kQChunk0, &tm_q1, &bars->q_full, h * HD + 64, row);
       }
       bool ok = true;
       uint32_t issued = 0, issued_par = 0;
@@ -283,16 +320,23 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (!mbar_wait(&bars->kv_empty[st], f ^ 1, abort_flag)) { ok = false; break; }
         int row, col, nvalid;
         bool pre;
-        uint8_t *kt = smem + CF::kKOff + st * CF::kTile;
-        uint8_t *vt = smem + CF::kVOff + st * CF::kTile;
+        uint8_t *kt = smem + CF::kKOff + st * CF::kKTile;
+        uint8_t *vt = smem + CF::kVOff + st * CF::kKTile;
         kv_coords(j, false, row, col, pre, nvalid);
-        mbar_arrive_expect_tx(&bars->k_full[st], CF::kTile);
-        tma_load_2d(kt, pre ? &tm_p0 : &tm_x0, &bars->k_full[st], col, row);
-        tma_load_2d(kt + CF::kChunk0, pre ? &tm_p1 : &tm_x1, &bars->k_full[st], col + 64, row);
+        mbar_arrive_expect_tx(&bars->k_full[st], CF::kKChunk0 + CF::kKChunk1);
+        tma_load_2d(kt, pre ? &tm_p0 : &tm_k0, &bars->k_full[st], col, row);
+        tma_load_2d(kt + CF::kKChunk0, pre ? &tm_p1 : &tm_k1, &bars->k_full[st], col + 64, row);
         kv_coords(j, true, row, col, pre, nvalid);
-        mbar_arrive_expect_tx(&bars->v_full[st], CF::kTile);
-        tma_load_2d(vt, pre ? &tm_p0 : &tm_x0, &bars->v_full[st], col, row);
-        tma_load_2d(vt + CF::kChunk0, pre ? &tm_p1 : &tm_x1, &bars->v_full[st], col + 64, row);
+        mbar_arrive_expect_tx(&bars->v_full[st], CF::kVChunks * CF::kVChunk);
+        if (HD == 72) {
+#pragma unroll
+          for (int c = 0; c < CF::kVChunks; ++c)
+            tma_load_2d(vt + c * CF::kVChunk, pre ? &tm_p1 : &tm_k1, &bars->v_full[st], col + 16 * c,
+                        row);
+        } else {
+          tma_load_2d(vt, pre ? &tm_p0 : &tm_k0, &bars->v_full[st], col, row);
+          tma_load_2d(vt + CF::kVChunk, pre ? &tm_p1 : &tm_k1, &bars->v_full[st], col + 64, row);
+        }
         issued |= 1u << st;
         issued_par = (issued_par & ~(1u << st)) | (f << st);
       }
@@ -305,17 +349,19 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    const int t = warp - 1;  // query tile served by this warp
+    if (t < n_tiles_q && elect_one()) {
       bool ok = true, any = false;
-      const uint32_t sq = smem_u32(smem + CF::kQOff);
+      const uint32_t qa = smem_u32(smem + CF::kQOff + t * CF::kQTile);
       const uint32_t sk = smem_u32(smem + CF::kKOff);
       const uint32_t sv = smem_u32(smem + CF::kVOff);
+      const uint32_t s_tm = tmem + CF::tmem_s(t), p_tm = tmem + CF::tmem_p(t),
+                     o_tm = tmem + CF::tmem_o(t);
       // S_t = Q_t K_j^T over HDP/16 k-steps
-      auto issue_s = [&](int t, int st) {
-        const uint32_t qa = sq + t * CF::kTile, ka = sk + st * CF::kTile;
-        const uint32_t d = tmem + CF::kTmemS + t * 128;
+      auto issue_s = [&](int st) {
+        const uint32_t ka = sk + st * CF::kKTile;
 #pragma unroll
         for (int k = 0; k < CF::HDP / 16; ++k) {
           uint64_t ad, bd;
@@ -323,32 +369,26 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             ad = smem_desc(qa + k * 32, 16, 1024, 2);
             bd = smem_desc(ka + k * 32, 16, 1024, 2);
           } else if (HD == 72) {
-            ad = smem_desc(qa + CF::kChunk0, 16, 256, 6);
-            bd = smem_desc(ka + CF::kChunk0, 16, 256, 6);
+            ad = smem_desc(qa + CF::kQChunk0, 16, 256, 6);
+            bd = smem_desc(ka + CF::kKChunk0, 16, 256, 6);
           } else {
-            ad = smem_desc(qa + CF::kChunk0 + (k - 4) * 32, 16, 1024, 2);
-            bd = smem_desc(ka + CF::kChunk0 + (k - 4) * 32, 16, 1024, 2);
+            ad = smem_desc(qa + CF::kQChunk0 + (k - 4) * 32, 16, 1024, 2);
+            bd = smem_desc(ka + CF::kKChunk0 + (k - 4) * 32, 16, 1024, 2);
           }
-          mma_bf16_ss(d, ad, bd, CF::kIdescS, k > 0);
+          mma_bf16_ss(s_tm, ad, bd, CF::kIdescS, k > 0);
         }
       };
-      // O_t += P_t V_j; P_t is bf16 in TMEM (S_t's first 64 columns)
-      auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t va = sv + st * CF::kTile;
-        const uint32_t p = tmem + CF::kTmemS + t * 128;
-        const uint32_t d = tmem + CF::kTmemO + t * 128;
+      // O_t += P_t V_j; P_t is bf16 in its own TMEM columns (2 keys per column)
+      auto issue_pv = [&](int st, bool acc) {
+        const uint32_t va = sv + st * CF::kKTile;
 #pragma unroll
-        for (int k = 0; k < kBlockK / 16; ++k) {
+        for (int k = 0; k < BK / 16; ++k) {
           const uint32_t accf = (acc || k > 0) ? 1u : 0u;
-          if (HD == 72) {
-            mma_bf16_ts(d, p + k * 8, smem_desc(va + k * 2048, 16384, 1024, 2), CF::kIdescPV0,
-                        accf);
-            mma_bf16_ts(d + 64, p + k * 8, smem_desc(va + CF::kChunk0 + k * 512, 4096, 256, 6),
-                        CF::kIdescPV1, accf);
-          } else {
-            mma_bf16_ts(d, p + k * 8, smem_desc(va + k * 2048, 16384, 1024, 2), CF::kIdescPV0,
-                        accf);
-          }
+          // V is the MN-major B operand: 16 keys (rows) per k-step, the
+          // column chunks kVChunk bytes apart along N
+          const uint64_t bd = HD == 72 ? smem_desc(va + k * 512, CF::kVChunk, 256, 6)
+                                       : smem_desc(va + k * 2048, CF::kVChunk, 1024, 2);
+          mma_bf16_ts(o_tm, p_tm + k * 8, bd, CF::kIdescPV, accf);
         }
       };
       auto wait_k = [&](int j) -> bool {
@@ -358,46 +398,38 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     : mbar_wait(&bars->k_full[st], f, abort_flag);
       };
       do {
-        for (int t = 0; t < n_tiles_q; ++t)
-          if (!mbar_wait(&bars->q_ready[t], 0, abort_flag)) { ok = false; break; }
-        if (!ok || !wait_k(0)) { ok = false; break; }
+        if (!mbar_wait(&bars->q_ready[t], 0, abort_flag) || !wait_k(0)) { ok = false; break; }
         tc_fence_after();
-        for (int t = 0; t < n_tiles_q; ++t) {
-          issue_s(t, 0);
-          mma_commit(&bars->s_full[t]);
-        }
+        issue_s(0);
+        mma_commit(&bars->s_full[t]);
         any = true;
-        for (int j = 0; j < n_kv && ok; ++j) {
+        for (int j = 0; j < n_kv; ++j) {
           const int st = j % NS;
-          const uint32_t f = (j / NS) & 1;
-          if (!mbar_wait(&bars->v_full[st], f, abort_flag)) { ok = false; break; }
-          for (int t = 0; t < n_tiles_q; ++t) {
-            if (!mbar_wait(&bars->p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          // S_t(j+1) as soon as the softmax threads hold S_t(j) in registers
+          if (j + 1 < n_kv) {
+            if (!wait_k(j + 1) || !mbar_wait(&bars->s_free[t], j & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, st, j > 0);
-            mma_commit(&bars->o_done[t]);
-            if (j + 1 < n_kv) {
-              if (!wait_k(j + 1)) { ok = false; break; }
-              // S_t(j+1) overwrites P_t(j): wait until O_t += P_t V_j has finished
-              if (!mbar_wait(&bars->o_done[t], j & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              issue_s(t, (j + 1) % NS);
-              mma_commit(&bars->s_full[t]);
-            }
+            issue_s((j + 1) % NS);
+            mma_commit(&bars->s_full[t]);
           }
-          mma_commit(&bars->kv_empty[st]);
+          if (!mbar_wait(&bars->v_full[st], (j / NS) & 1, abort_flag) ||
+              !mbar_wait(&bars->p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(st, j > 0);
+          mma_commit(&bars->o_done[t]);
+          mma_commit(&bars->kv_empty[st]);  // this tile is done with K_j and V_j
         }
       } while (false);
       if (!ok && any) {
-        mma_commit(&bars->drain);
-        drain_wait(&bars->drain, 0);
+        mma_commit(&bars->drain[t]);
+        drain_wait(&bars->drain[t], 0);
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int sw = warp - 4;
     const int t = sw >> 3;               // query tile of this warp
-    const int half = (sw >> 2) & 1;      // which 64 of the 128 score columns
+    const int half = (sw >> 2) & 1;      // which half of the key tile's score columns
     const int quarter = warp & 3;        // TMEM lane quarter
     const int r = quarter * 32 + lane;   // query row inside the tile
     if (t < n_tiles_q) {
@@ -406,20 +438,23 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       if (half == 0) {
         ok = mbar_wait(&bars->q_full, 0, abort_flag);
         if (ok) {
-          uint8_t *qt = smem + CF::kQOff + t * CF::kTile;
+          uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
           if (ROPE && qrow < len)
-            rope_row_smem<HD>(qt, r, prm.pos[2 * (seg0 + qrow)], prm.pos[2 * (seg0 + qrow) + 1], fr);
+            rope_row_smem<HD>(qt, CF::kQChunk0, r, prm.pos[2 * (seg0 + qrow)],
+                              prm.pos[2 * (seg0 + qrow) + 1], fr);
           if (HD == 72)  // zero the 8 padding columns 72..79 (logical unit 9)
-            *reinterpret_cast<uint4 *>(qt + unit_offset<HD>(r, 9)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(qt + unit_offset<HD>(r, 9, CF::kQChunk0)) =
+                make_uint4(0, 0, 0, 0);
           fence_proxy_async_smem();
         }
         mbar_arrive(&bars->q_ready[t]);
       }
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-      const uint32_t s_addr = tmem + lane_base + CF::kTmemS + t * 128;
-      const uint32_t o_addr = tmem + lane_base + CF::kTmemO + t * 128;
-      float *xv = reinterpret_cast<float *>(smem + CF::kXOff) + t * 256;  // [half][row]
+      const uint32_t s_addr = tmem + lane_base + CF::tmem_s(t) + half * HC;
+      const uint32_t p_addr = tmem + lane_base + CF::tmem_p(t) + half * (HC / 2);
+      const uint32_t o_addr = tmem + lane_base + CF::tmem_o(t);
+      float *xv = reinterpret_cast<float *>(smem + CF::kXOff) + t * 256;  // [j&1][t][half][row]
       uint64_t *xb = &bars->xchg[t][quarter];
       const float sl2 = prm.scale_log2;
       // head_dim 72: the softmax denominator is accumulated by the tensor core
@@ -430,9 +465,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       // numerator and denominator and its spread equals round-to-nearest's.
       // head_dim 128 sums in registers and rounds P to nearest.
       constexpr bool kSumByMma = (HD == 72);
-      // pairs of this thread's 64 exponentials that run on the FMA pipe
-      // instead of the special-function unit (8 of 32: a 25% share)
-      constexpr int kPolyPairs = 8;
+      // pairs of this thread's HC exponentials that run on the FMA pipe
+      // instead of the special-function unit (a quarter)
+      constexpr int kPolyPairs = HC / 8;
       constexpr int kOC = CF::HDP / 16;         // 16-column chunks of O
       constexpr int kOCHalf = (kOC + 1) / 2;   // rescaled by half 0; the rest by half 1
       const int oc_lo = half ? kOCHalf : 0, oc_hi = half ? kOC : kOCHalf;
@@ -441,39 +476,33 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       for (int j = 0; j < n_kv && ok; ++j) {
         if (!warp_wait(&bars->s_full[t], j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const int nvalid = (j < n_pre ? min(kBlockK, prm.P - j * kBlockK)
-                                      : min(kBlockK, len - (j - n_pre) * kBlockK)) -
-                           half * 64;  // valid keys among this thread's 64 columns
-        uint32_t s[2][32];
+        const int nvalid = (j < n_pre ? min(BK, prm.P - j * BK) : min(BK, len - (j - n_pre) * BK)) -
+                           half * HC;  // valid keys among this thread's columns
+        uint32_t s[HC];
         __syncwarp();
-        tmem_ld32(s_addr + half * 64, s[0]);
-        tmem_ld32(s_addr + half * 64 + 32, s[1]);
+        tmem_ld_cols<HC>(s_addr, s);
         tmem_ld_wait();
-        if (nvalid < 64) {  // keys past the sequence end: -inf, so p = 0
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c * 32 + i >= nvalid) s[c][i] = 0xFF800000u;
-        }
-        float mc[2];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float a = __uint_as_float(s[c][0]);
-#pragma unroll
-          for (int i = 1; i < 31; i += 2)
-            a = fmax3(a, __uint_as_float(s[c][i]), __uint_as_float(s[c][i + 1]));
-          mc[c] = fmaxf(a, __uint_as_float(s[c][31]));
-        }
-        // swap partial maxima with the thread that holds the row's other half
-        // (its P columns overlap this half's S columns, so the swap also
-        // orders this thread's TMEM loads before the partner's P stores)
-        xv[half * 128 + r] = fmaxf(mc[0], mc[1]) * sl2;
         tc_fence_before();
+        mbar_arrive(&bars->s_free[t]);  // S_t may now be overwritten by the next key tile
+        if (nvalid < HC) {  // keys past the sequence end: -inf, so p = 0
+#pragma unroll
+          for (int i = 0; i < HC; ++i)
+            if (i >= nvalid) s[i] = 0xFF800000u;
+        }
+        float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
+#pragma unroll
+        for (int i = 2; i + 3 < HC; i += 4) {
+          a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+          a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+        }
+        if constexpr ((HC - 2) % 4 != 0)
+          a0 = fmax3(a0, __uint_as_float(s[HC - 2]), __uint_as_float(s[HC - 1]));
+        // swap partial maxima with the thread that holds the row's other half
+        float *xj = xv + (j & 1) * 512;
+        xj[half * 128 + r] = fmaxf(a0, a1) * sl2;
         mbar_arrive(xb);
         if (!warp_wait(xb, j & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const float m_tile = fmaxf(xv[r], xv[128 + r]);
+        const float m_tile = fmaxf(xj[r], xj[128 + r]);
         const bool grow = __any_sync(0xffffffffu, m_tile > m + 8.0f);
         if (j == 0) {
           m = m_tile;
@@ -509,18 +538,20 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             for (int k = 0; k < 2; ++k) l2[k] = f2_mul(l2[k], f2);
           m = m_new;
         }
-        // p = 2^(s*scale*log2e - m) two at a time; bf16 P of keys
-        // [64 half, 64 half + 64) into S columns [32 half, 32 half + 32)
+        // p = 2^(s*scale*log2e - m) two at a time, packed bf16 pairs; stored
+        // to P_t in two pieces (the first once O_t += P_t V_{j-1} has read
+        // the previous P_t, which by then has normally finished)
         const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
+        constexpr int NP = HC / 2, NP0 = NP >= 16 ? 16 : NP;
+        uint32_t pk[NP];
+        auto exp_pairs = [&](auto i0c, auto i1c) {
+          constexpr int i0 = decltype(i0c)::value, i1 = decltype(i1c)::value;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint64_t xa = f2_fma(
-                f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])), sc2, nm2);
+          for (int i = i0; i < i1; ++i) {
+            const uint64_t xa =
+                f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
             float p0, p1;
-            if (c * 16 + i < kPolyPairs) {  // this share of the exponentials runs on the FMA pipe
+            if (i < kPolyPairs) {  // this share of the exponentials runs on the FMA pipe
               exp2_poly_x2(xa, p0, p1);
             } else {
               float x0, x1;
@@ -535,16 +566,29 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
               pk[i] = pack_bf16x2_alu(p0, p1);
             }
           }
-          tmem_st16(s_addr + half * 32 + c * 16, pk);
+        };
+        exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
+        if (j > 0 && !warp_wait(&bars->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st_cols<NP0>(p_addr, pk);
+        if constexpr (NP > NP0) {
+          exp_pairs(std::integral_constant<int, NP0>{}, std::integral_constant<int, NP>{});
+          tmem_st_cols<NP - NP0>(p_addr + NP0, pk + NP0);
         }
-        if (kSumByMma && t == 0 && half == 0) {
-          // ones in V's column 72 of this key tile (the first padding column)
+        if (kSumByMma && half == 0 && r < BK) {
+          // ones in V's column 72 of this key tile (the first padding column);
+          // both query tiles write it (the same value) so that each tile's
+          // P.V depends only on its own softmax
           const int st = j % NS;
-          if (!warp_wait(&bars->v_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
-          *reinterpret_cast<uint16_t *>(smem + CF::kVOff + st * CF::kTile + unit_offset<HD>(r, 9)) =
-              0x3F80u;  // bf16 1.0
-          fence_proxy_async_smem();
+          if (!mbar_wait(&bars->v_full[st], (j / NS) & 1, abort_flag)) ok = false;
+          if (ok) {
+            // dim 72: 16-byte unit 1 of the fifth 32B-swizzled chunk
+            *reinterpret_cast<uint16_t *>(smem + CF::kVOff + st * CF::kKTile + 4 * CF::kVChunk +
+                                          r * 32 + ((1 ^ ((r >> 2) & 1)) << 4)) = 0x3F80u;  // 1.0
+            fence_proxy_async_smem();
+          }
         }
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_full[t]);
@@ -558,10 +602,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           float a, b, c2, d2;
           f2_unpack(l2[0], a, b);
           f2_unpack(l2[1], c2, d2);
-          xv[half * 128 + r] = (a + b) + (c2 + d2);
+          float *xj = xv + (n_kv & 1) * 512;
+          xj[half * 128 + r] = (a + b) + (c2 + d2);
           mbar_arrive(xb);
           have_l = warp_wait(xb, n_kv & 1, abort_flag);
-          l = xv[r] + xv[128 + r];
+          l = xj[r] + xj[128 + r];
         }
         if (have_l) {
           __nv_bfloat16 *orow =
@@ -573,21 +618,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
       }
     }
-  } else if (ROPE && warp < 4) {
+  } else if (ROPE && warp == 3) {
     // ------------------------------------------------------------ K rotation
-    // warps 2-3; thread rotates key rows r and r + 64 of each own-key tile
-    const int r0 = (warp - 2) * 32 + lane;
+    // thread rotates key rows lane, lane + 32, ... of each own-key tile
+    const int r0 = lane;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j % NS;
       const uint32_t f = (j / NS) & 1;
       if (!mbar_wait(&bars->k_full[st], f, abort_flag)) break;
       if (j >= n_pre) {
 #pragma unroll 1
-        for (int r = r0; r < kBlockK; r += 64) {
-          const int key = (j - n_pre) * kBlockK + r;
+        for (int r = r0; r < BK; r += 32) {
+          const int key = (j - n_pre) * BK + r;
           if (key < len)
-            rope_row_smem<HD>(smem + CF::kKOff + st * CF::kTile, r, prm.pos[2 * (seg0 + key)],
-                              prm.pos[2 * (seg0 + key) + 1], fr);
+            rope_row_smem<HD>(smem + CF::kKOff + st * CF::kKTile, CF::kKChunk0, r,
+                              prm.pos[2 * (seg0 + key)], prm.pos[2 * (seg0 + key) + 1], fr);
         }
         fence_proxy_async_smem();
       }
@@ -614,7 +659,7 @@ static cudaError_t launch_hd(const CUtensorMap *maps, const attn::Params &prm, i
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmem));
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(attn::kThreads), CF::kSmem, st, 1, maps[0], maps[1],
-                    maps[2], maps[3], prm, fr);
+                    maps[2], maps[3], maps[4], maps[5], prm, fr);
 }
 
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,
@@ -625,33 +670,36 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
   const int C = H * d;
   const int Hkv = s.kv_heads > 0 ? s.kv_heads : H;
   const int P = s.prefix_kv ? s.prefix_len : 0;
-  CUtensorMap maps[4];
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const bool small = (d == 72);
+  const uint32_t bk = small ? attn::Cfg<72>::BK : attn::Cfg<128>::BK;
+  const uint32_t w1 = small ? 16 : 64;  // inner box of a tile's second chunk
+  const auto sw1 = small ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  // maps: Q chunk 0/1 (128-row boxes), K/V chunk 0/1 (key-tile boxes), prefix chunk 0/1
+  CUtensorMap maps[6];
+  bool good = true;
   // qkv viewed as [T, 3C]
-  if (encode_tensor_map_2d(&maps[0], BF, qkv, 3ull * C, s.total_tokens, 6ull * C, 64, 128,
-                           CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  if (encode_tensor_map_2d(&maps[1], BF, qkv, 3ull * C, s.total_tokens, 6ull * C, small ? 16 : 64,
-                           128, small ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) !=
-      CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  good &= encode_tensor_map_2d(&maps[0], BF, qkv, 3ull * C, s.total_tokens, 6ull * C, 64,
+                               attn::kBlockQ, CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS;
+  good &= encode_tensor_map_2d(&maps[1], BF, qkv, 3ull * C, s.total_tokens, 6ull * C, w1,
+                               attn::kBlockQ, sw1) == CUDA_SUCCESS;
+  good &= encode_tensor_map_2d(&maps[2], BF, qkv, 3ull * C, s.total_tokens, 6ull * C, 64, bk,
+                               CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS;
+  good &= encode_tensor_map_2d(&maps[3], BF, qkv, 3ull * C, s.total_tokens, 6ull * C, w1, bk,
+                               sw1) == CUDA_SUCCESS;
   if (P > 0) {
     // prefix viewed as [S * 2 * P, Hkv * d]
     const uint64_t rows = uint64_t(s.n_seqs) * 2 * P;
-    if (encode_tensor_map_2d(&maps[2], BF, s.prefix_kv, uint64_t(Hkv) * d, rows,
-                             uint64_t(Hkv) * d * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) !=
-        CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-    if (encode_tensor_map_2d(&maps[3], BF, s.prefix_kv, uint64_t(Hkv) * d, rows,
-                             uint64_t(Hkv) * d * 2, small ? 16 : 64, 128,
-                             small ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) !=
-        CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+    good &= encode_tensor_map_2d(&maps[4], BF, s.prefix_kv, uint64_t(Hkv) * d, rows,
+                                 uint64_t(Hkv) * d * 2, 64, bk, CU_TENSOR_MAP_SWIZZLE_128B) ==
+            CUDA_SUCCESS;
+    good &= encode_tensor_map_2d(&maps[5], BF, s.prefix_kv, uint64_t(Hkv) * d, rows,
+                                 uint64_t(Hkv) * d * 2, w1, bk, sw1) == CUDA_SUCCESS;
   } else {
-    maps[2] = maps[0];
-    maps[3] = maps[1];
+    maps[4] = maps[2];
+    maps[5] = maps[3];
   }
+  if (!good) return cudaErrorInvalidValue;
   attn::Params prm;
   prm.H = H;
   prm.C = C;

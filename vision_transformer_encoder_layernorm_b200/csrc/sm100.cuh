@@ -75,30 +75,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on phase `parity` of an mbarrier.  Returns false (and sets the
-// CTA's shared abort flag) when the wait exceeds kWaitTimeoutNs, or as soon as
-// another thread of the CTA has aborted.  Callers stop their role loop on
-// false; the kernel then drains its in-flight copies (bounded) and returns.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity,
-                                            volatile int *abort_flag) {
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t n = 0;
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++n & 31u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// sleeps in hardware (issuing nothing) until the phase completes or about
+// hint_ns pass, instead of spinning on the barrier.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
 }
 
+// Bounded wait on phase `parity` of an mbarrier.  Returns false (and sets the
+// CTA's shared abort flag) when the wait exceeds kWaitTimeoutNs, or as soon as
+// another thread of the CTA has aborted (checked at least every millisecond).
+// Callers stop their role loop on false; the kernel then drains its in-flight
+// copies (bounded) and returns.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort_flag);
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- TMA
@@ -251,6 +260,48 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+
+// N consecutive TMEM columns of this thread's lane <-> r[0..N), issued as
+// pieces of 32/16/8 (loads, N % 8 == 0) or 16/8/4 (stores, N % 4 == 0).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t *r) {
+  static_assert(N % 8 == 0, "load width");
+  if constexpr (N >= 32) {
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+    tmem_ld_cols<N - 32>(taddr + 32, r + 32);
+  } else if constexpr (N >= 16) {
+    tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+    tmem_ld_cols<N - 16>(taddr + 16, r + 16);
+  } else if constexpr (N >= 8) {
+    tmem_ld8(taddr, *reinterpret_cast<uint32_t(*)[8]>(r));
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t *r) {
+  static_assert(N % 4 == 0, "store width");
+  if constexpr (N >= 16) {
+    tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(r));
+    tmem_st_cols<N - 16>(taddr + 16, r + 16);
+  } else if constexpr (N >= 8) {
+    tmem_st8(taddr, *reinterpret_cast<const uint32_t(*)[8]>(r));
+    tmem_st_cols<N - 8>(taddr + 8, r + 8);
+  } else if constexpr (N >= 4) {
+    tmem_st4(taddr, *reinterpret_cast<const uint32_t(*)[4]>(r));
+  }
 }
 
 // Packed fp32x2 arithmetic (one instruction for two lanes of fp32 data).
