@@ -11,12 +11,17 @@
 // Prefix K/V (LightX2V NeoPP README, "KV file layout": [2, seq, kv_heads, d]
 // per layer) is read through its own TMA descriptors as the first key tiles.
 //
-// CTA = (sequence, head, two 128-row query tiles), 20 warps:
+// Persistent: one CTA per SM walks a static list of work items = (sequence,
+// head, two 128-row query tiles), full pairs first, round-robin over CTAs;
+// every barrier phase is counted across items.  20 warps:
 //   0        TMA producer (Q tiles once, then K and V tiles through a ring)
 //   1, 2     MMA issuers of query tiles 0 and 1 (one lane each; warp 1 also
 //            owns the TMEM allocation): each follows its own tile's
 //            softmax, so neither tile's MMAs wait behind the other's
-//   3        (ROPE only) rotate each own-key K tile in shared memory
+//   3        prepares each item's Q tiles (head_dim 72: zero the padding
+//            columns; ROPE: rotate) and each key tile (ROPE: rotate own-key
+//            K rows; head_dim 72: ones in V's column 72, the row sums), so
+//            the next item's first S overlaps the softmax epilogue
 //   4-11     softmax of query tile 0, 12-19 of query tile 1: two threads per
 //            query row, one per half of the key tile's score columns; the
 //            pair swaps partial row maxima through shared memory
@@ -30,6 +35,7 @@
 // head_dim 72 is computed as 80 (4 MMA k-steps from a 64-column 128B-swizzled
 // chunk, 1 from a 16-column 32B-swizzled chunk); Q's columns 72..79 are zeroed
 // in shared memory so the neighbouring head's values there contribute 0.
+#include <cstdlib>
 #include <type_traits>
 
 #include "kernels.h"
@@ -40,6 +46,7 @@ namespace attn {
 
 constexpr int kBlockQ = 128;
 constexpr int kThreads = 640;
+constexpr int kRegsLow = 64, kRegsHigh = 104;  // warpgroup 0 / softmax warpgroups
 
 __host__ __device__ constexpr uint32_t round_up_1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
@@ -87,9 +94,9 @@ static_assert(Cfg<128>::kTmemP1 + Cfg<128>::BK / 2 <= Cfg<128>::kTmemO0 &&
               "TMEM layout, head_dim 128");
 
 struct __align__(8) Bars {
-  uint64_t q_full;
+  uint64_t q_full[2], q_empty[2];
   uint64_t q_ready[2];
-  uint64_t k_full[5], v_full[5], kv_empty[5], k_ready[5];
+  uint64_t k_full[5], v_full[5], kv_empty[5], k_ready[5], v_ready[5];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t xchg[2][4];  // per (query tile, lane quarter): the 64 threads of a row pair
   uint64_t drain[2];
@@ -99,13 +106,36 @@ struct __align__(8) Bars {
 static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
 struct Params {
-  int H, C, Hkv, P, n_pairs;
+  int H, C, Hkv, P, n_pairs, n_seqs;
   float scale_log2;      // softmax scale * log2(e)
   const int32_t *cu;
   const int32_t *pos;
   __nv_bfloat16 *o;
   int *status;
 };
+
+// One work item: query tiles [q0, q0 + 256) of head h of sequence seq.
+struct Item {
+  int seq, h, hk, seg0, len, q0, n_tiles_q, n_kv;
+};
+
+// Work item w (pairs in ascending order, so a sequence's last, partial pair
+// comes after all full ones); false if the pair lies past the sequence end.
+__device__ __forceinline__ bool decode_item(int w, const Params &prm, int bk, Item &it) {
+  const int per_pair = prm.H * prm.n_seqs;
+  const int pair = w / per_pair, rem = w - pair * per_pair;
+  it.seq = rem % prm.n_seqs;
+  it.h = rem / prm.n_seqs;
+  it.hk = it.h / (prm.H / prm.Hkv);
+  it.seg0 = prm.cu[it.seq];
+  it.len = prm.cu[it.seq + 1] - it.seg0;
+  it.q0 = pair * 2 * kBlockQ;
+  if (it.q0 >= it.len) return false;
+  it.n_tiles_q = (it.len - it.q0 > kBlockQ) ? 2 : 1;
+  const int n_pre = prm.P > 0 ? (prm.P + bk - 1) / bk : 0;
+  it.n_kv = n_pre + (it.len + bk - 1) / bk;
+  return true;
+}
 
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -233,6 +263,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   constexpr int NS = CF::kStages;
   constexpr int BK = CF::BK;
   constexpr int HC = CF::HC;
+  constexpr bool kPrep = ROPE || HD == 72;  // warp 3 has Q / K / V tiles to touch up
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -242,38 +273,28 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
   pdl_trigger();
   pdl_wait();
-  // ---- work item: pairs of query tiles, longest sequences' last pairs first
-  const int S = gridDim.x / (prm.n_pairs * prm.H);
-  const int b = blockIdx.x;
-  const int pair = prm.n_pairs - 1 - b / (prm.H * S);
-  const int rem = b % (prm.H * S);
-  const int seq = rem % S, h = rem / S;
-  const int seg0 = prm.cu[seq];
-  const int len = prm.cu[seq + 1] - seg0;
-  const int q0 = pair * 2 * kBlockQ;
-  if (q0 >= len) return;  // uniform across the CTA, before any barrier or TMEM use
-  const int n_tiles_q = (len - q0 > kBlockQ) ? 2 : 1;
+  const int n_items = prm.n_pairs * prm.H * prm.n_seqs;
   const int n_pre = prm.P > 0 ? (prm.P + BK - 1) / BK : 0;
-  const int n_kv = n_pre + (len + BK - 1) / BK;
-  const int hk = h / (prm.H / prm.Hkv);
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&bars->q_ready[t], 128);
+      mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->q_empty[t], 1);
+      mbar_init(&bars->q_ready[t], 32);
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->s_free[t], 256);
       mbar_init(&bars->p_full[t], 256);
       mbar_init(&bars->o_done[t], 1);
       for (int q = 0; q < 4; ++q) mbar_init(&bars->xchg[t][q], 64);
+      mbar_init(&bars->drain[t], 1);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], n_tiles_q);  // one commit per query tile
+      mbar_init(&bars->kv_empty[s], 2);  // one commit per query tile (tile 0 twice if alone)
       mbar_init(&bars->k_ready[s], 32);
+      mbar_init(&bars->v_ready[s], 32);
     }
-    for (int t = 0; t < 2; ++t) mbar_init(&bars->drain[t], 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -285,63 +306,80 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // registers: 640 threads x 96 at launch; warps 0-3 (one warpgroup) give
+  // back 32 each, the four softmax warpgroups take 8 more:
+  // 128 x 64 + 512 x 104 = 640 x 96
+  static_assert(128 * kRegsLow + 512 * kRegsHigh <= kThreads * 96, "register split");
 
-  // key tile j -> (map, column of head's chunk 0, first row, valid keys)
-  auto kv_coords = [&](int j, bool is_v, int &row, int &col, bool &prefix, int &nvalid) {
+  // key tile j of an item -> (prefix?, column of the head's chunk 0, first row)
+  auto kv_coords = [&](const Item &it, int j, bool is_v, int &row, int &col, bool &prefix) {
     if (j < n_pre) {
       prefix = true;
-      row = (seq * 2 + (is_v ? 1 : 0)) * prm.P + j * BK;
-      col = hk * HD;
-      nvalid = min(BK, prm.P - j * BK);
+      row = (it.seq * 2 + (is_v ? 1 : 0)) * prm.P + j * BK;
+      col = it.hk * HD;
     } else {
       prefix = false;
-      const int jj = j - n_pre;
-      row = seg0 + jj * BK;
-      col = (is_v ? 2 : 1) * prm.C + h * HD;
-      nvalid = min(BK, len - jj * BK);
+      row = it.seg0 + (j - n_pre) * BK;
+      col = (is_v ? 2 : 1) * prm.C + it.h * HD;
     }
   };
 
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
-      mbar_arrive_expect_tx(&bars->q_full, n_tiles_q * CF::kQTile);
-      for (int t = 0; t < n_tiles_q; ++t) {
-        uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
-        const int row = seg0 + q0 + t * kBlockQ;
-        tma_load_2d(qt, &tm_q0, &bars->q_full, h * HD, row);
-        tma_load_2d(qt + CF::kQChunk0, &tm_q1, &bars->q_full, h * HD + 64, row);
-      }
       bool ok = true;
-      uint32_t issued = 0, issued_par = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % NS;
-        const uint32_t f = (j / NS) & 1;
-        if (!mbar_wait(&bars->kv_empty[st], f ^ 1, abort_flag)) { ok = false; break; }
-        int row, col, nvalid;
-        bool pre;
-        uint8_t *kt = smem + CF::kKOff + st * CF::kKTile;
-        uint8_t *vt = smem + CF::kVOff + st * CF::kKTile;
-        kv_coords(j, false, row, col, pre, nvalid);
-        mbar_arrive_expect_tx(&bars->k_full[st], CF::kKChunk0 + CF::kKChunk1);
-        tma_load_2d(kt, pre ? &tm_p0 : &tm_k0, &bars->k_full[st], col, row);
-        tma_load_2d(kt + CF::kKChunk0, pre ? &tm_p1 : &tm_k1, &bars->k_full[st], col + 64, row);
-        kv_coords(j, true, row, col, pre, nvalid);
-        mbar_arrive_expect_tx(&bars->v_full[st], CF::kVChunks * CF::kVChunk);
-        if (HD == 72) {
-#pragma unroll
-          for (int c = 0; c < CF::kVChunks; ++c)
-            tma_load_2d(vt + c * CF::kVChunk, pre ? &tm_p1 : &tm_k1, &bars->v_full[st], col + 16 * c,
-                        row);
-        } else {
-          tma_load_2d(vt, pre ? &tm_p0 : &tm_k0, &bars->v_full[st], col, row);
-          tma_load_2d(vt + CF::kVChunk, pre ? &tm_p1 : &tm_k1, &bars->v_full[st], col + 64, row);
+      uint32_t J = 0;                 // key tiles loaded so far (ring position)
+      uint32_t act[2] = {0, 0};       // items in which each query tile was active
+      uint32_t issued = 0, issued_par = 0, q_issued = 0;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        Item it;
+        if (!decode_item(w, prm, BK, it)) continue;
+        for (int t = 0; t < it.n_tiles_q; ++t) {
+          // the previous item's S MMAs of this tile have finished reading Q_t
+          if (act[t] > 0 && !mbar_wait(&bars->q_empty[t], (act[t] - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
+          const int row = it.seg0 + it.q0 + t * kBlockQ;
+          mbar_arrive_expect_tx(&bars->q_full[t], CF::kQTile);
+          tma_load_2d(qt, &tm_q0, &bars->q_full[t], it.h * HD, row);
+          tma_load_2d(qt + CF::kQChunk0, &tm_q1, &bars->q_full[t], it.h * HD + 64, row);
+          q_issued = (q_issued & ~(3u << (2 * t))) | ((1u | ((act[t] & 1) << 1)) << (2 * t));
+          ++act[t];
         }
-        issued |= 1u << st;
-        issued_par = (issued_par & ~(1u << st)) | (f << st);
+        for (int j = 0; j < it.n_kv && ok; ++j, ++J) {
+          const int st = J % NS;
+          const uint32_t f = (J / NS) & 1;
+          if (!mbar_wait(&bars->kv_empty[st], f ^ 1, abort_flag)) { ok = false; break; }
+          int row, col;
+          bool pre;
+          uint8_t *kt = smem + CF::kKOff + st * CF::kKTile;
+          uint8_t *vt = smem + CF::kVOff + st * CF::kKTile;
+          kv_coords(it, j, false, row, col, pre);
+          mbar_arrive_expect_tx(&bars->k_full[st], CF::kKChunk0 + CF::kKChunk1);
+          tma_load_2d(kt, pre ? &tm_p0 : &tm_k0, &bars->k_full[st], col, row);
+          tma_load_2d(kt + CF::kKChunk0, pre ? &tm_p1 : &tm_k1, &bars->k_full[st], col + 64, row);
+          kv_coords(it, j, true, row, col, pre);
+          mbar_arrive_expect_tx(&bars->v_full[st], CF::kVChunks * CF::kVChunk);
+          if (HD == 72) {
+#pragma unroll
+            for (int c = 0; c < CF::kVChunks; ++c)
+              tma_load_2d(vt + c * CF::kVChunk, pre ? &tm_p1 : &tm_k1, &bars->v_full[st],
+                          col + 16 * c, row);
+          } else {
+            tma_load_2d(vt, pre ? &tm_p0 : &tm_k0, &bars->v_full[st], col, row);
+            tma_load_2d(vt + CF::kVChunk, pre ? &tm_p1 : &tm_k1, &bars->v_full[st], col + 64, row);
+          }
+          issued |= 1u << st;
+          issued_par = (issued_par & ~(1u << st)) | (f << st);
+        }
       }
-      if (!ok) {
-        drain_wait(&bars->q_full, 0);
+      if (!ok) {  // wait (bounded) for the copies still in flight before the CTA exits
+        for (int t = 0; t < 2; ++t)
+          if (q_issued & (1u << (2 * t))) drain_wait(&bars->q_full[t], (q_issued >> (2 * t + 1)) & 1);
         for (int s = 0; s < NS; ++s)
           if (issued & (1u << s)) {
             drain_wait(&bars->k_full[s], (issued_par >> s) & 1);
@@ -352,7 +390,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
     const int t = warp - 1;  // query tile served by this warp
-    if (t < n_tiles_q && elect_one()) {
+    if (elect_one()) {
       bool ok = true, any = false;
       const uint32_t qa = smem_u32(smem + CF::kQOff + t * CF::kQTile);
       const uint32_t sk = smem_u32(smem + CF::kKOff);
@@ -391,90 +429,164 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           mma_bf16_ts(o_tm, p_tm + k * 8, bd, CF::kIdescPV, accf);
         }
       };
-      auto wait_k = [&](int j) -> bool {
-        const int st = j % NS;
-        const uint32_t f = (j / NS) & 1;
+      auto wait_k = [&](uint32_t J) -> bool {
+        const int st = J % NS;
+        const uint32_t f = (J / NS) & 1;
         return ROPE ? mbar_wait(&bars->k_ready[st], f, abort_flag)
                     : mbar_wait(&bars->k_full[st], f, abort_flag);
       };
-      do {
-        if (!mbar_wait(&bars->q_ready[t], 0, abort_flag) || !wait_k(0)) { ok = false; break; }
+      uint32_t J = 0;     // ring position (key tiles of all items so far)
+      uint32_t tc = 0;    // key tiles processed by this query tile so far
+      uint32_t act = 0;   // items in which this query tile was active
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        Item it;
+        if (!decode_item(w, prm, BK, it)) continue;
+        if (t >= it.n_tiles_q) {  // tile 0's issuer commits this tile's share of kv_empty
+          J += it.n_kv;
+          continue;
+        }
+        const bool alone = it.n_tiles_q == 1;
+        const int n_kv = it.n_kv;
+        // Q_t loaded and prepared; S_t of the previous item loaded by the softmax
+        if (!mbar_wait(kPrep ? &bars->q_ready[t] : &bars->q_full[t], act & 1, abort_flag) ||
+            (tc > 0 && !mbar_wait(&bars->s_free[t], (tc - 1) & 1, abort_flag)) || !wait_k(J)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        issue_s(0);
+        issue_s(J % NS);
         mma_commit(&bars->s_full[t]);
+        if (n_kv == 1) mma_commit(&bars->q_empty[t]);
         any = true;
         for (int j = 0; j < n_kv; ++j) {
-          const int st = j % NS;
+          const uint32_t Jj = J + j, tj = tc + j;
+          const int st = Jj % NS;
           // S_t(j+1) as soon as the softmax threads hold S_t(j) in registers
           if (j + 1 < n_kv) {
-            if (!wait_k(j + 1) || !mbar_wait(&bars->s_free[t], j & 1, abort_flag)) { ok = false; break; }
+            if (!wait_k(Jj + 1) || !mbar_wait(&bars->s_free[t], tj & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            issue_s((j + 1) % NS);
+            issue_s((Jj + 1) % NS);
             mma_commit(&bars->s_full[t]);
+            if (j + 2 == n_kv) mma_commit(&bars->q_empty[t]);  // last S of the item: Q_t free after it
           }
-          if (!mbar_wait(&bars->v_full[st], (j / NS) & 1, abort_flag) ||
-              !mbar_wait(&bars->p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(HD == 72 ? &bars->v_ready[st] : &bars->v_full[st], (Jj / NS) & 1, abort_flag) ||
+              !mbar_wait(&bars->p_full[t], tj & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_pv(st, j > 0);
           mma_commit(&bars->o_done[t]);
           mma_commit(&bars->kv_empty[st]);  // this tile is done with K_j and V_j
+          if (alone) mma_commit(&bars->kv_empty[st]);
         }
-      } while (false);
+        J += n_kv;
+        tc += n_kv;
+        ++act;
+      }
       if (!ok && any) {
         mma_commit(&bars->drain[t]);
         drain_wait(&bars->drain[t], 0);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp == 3 && kPrep) {
+    // ------------------------------------------------------------ Q, K, V touch-ups
+    // thread handles rows lane, lane + 32, ... of each tile
+    uint32_t J = 0;
+    uint32_t act[2] = {0, 0};
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      Item it;
+      if (!decode_item(w, prm, BK, it)) continue;
+      for (int t = 0; t < it.n_tiles_q; ++t) {
+        if (!mbar_wait(&bars->q_full[t], act[t] & 1, abort_flag)) { ok = false; break; }
+        uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
+#pragma unroll 1
+        for (int r = lane; r < kBlockQ; r += 32) {
+          const int qrow = it.q0 + t * kBlockQ + r;
+          if (ROPE && qrow < it.len)
+            rope_row_smem<HD>(qt, CF::kQChunk0, r, prm.pos[2 * (it.seg0 + qrow)],
+                              prm.pos[2 * (it.seg0 + qrow) + 1], fr);
+          if (HD == 72)  // zero the 8 padding columns 72..79 (logical unit 9)
+            *reinterpret_cast<uint4 *>(qt + unit_offset<HD>(r, 9, CF::kQChunk0)) =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_ready[t]);
+        ++act[t];
+      }
+      for (int j = 0; j < it.n_kv && ok; ++j, ++J) {
+        const int st = J % NS;
+        const uint32_t f = (J / NS) & 1;
+        if (ROPE) {
+          if (!mbar_wait(&bars->k_full[st], f, abort_flag)) { ok = false; break; }
+          if (j >= n_pre) {
+#pragma unroll 1
+            for (int r = lane; r < BK; r += 32) {
+              const int key = (j - n_pre) * BK + r;
+              if (key < it.len)
+                rope_row_smem<HD>(smem + CF::kKOff + st * CF::kKTile, CF::kKChunk0, r,
+                                  prm.pos[2 * (it.seg0 + key)], prm.pos[2 * (it.seg0 + key) + 1], fr);
+            }
+            fence_proxy_async_smem();
+          }
+          mbar_arrive(&bars->k_ready[st]);
+        }
+        if (HD == 72) {
+          // V's column 72 (16-byte unit 1 of the fifth 32B-swizzled chunk) = 1.0:
+          // O column 72 then accumulates the softmax row sum on the tensor core
+          if (!mbar_wait(&bars->v_full[st], f, abort_flag)) { ok = false; break; }
+          uint8_t *vt = smem + CF::kVOff + st * CF::kKTile + 4 * CF::kVChunk;
+#pragma unroll
+          for (int r = lane; r < BK; r += 32)
+            *reinterpret_cast<uint16_t *>(vt + r * 32 + ((1 ^ ((r >> 2) & 1)) << 4)) = 0x3F80u;
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->v_ready[st]);
+        }
+      }
+    }
+  }
+  } else {  // warps 4-19
+  regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax
     const int sw = warp - 4;
     const int t = sw >> 3;               // query tile of this warp
     const int half = (sw >> 2) & 1;      // which half of the key tile's score columns
     const int quarter = warp & 3;        // TMEM lane quarter
     const int r = quarter * 32 + lane;   // query row inside the tile
-    if (t < n_tiles_q) {
-      const int qrow = q0 + t * kBlockQ + r;  // row inside the sequence
-      bool ok = true;
-      if (half == 0) {
-        ok = mbar_wait(&bars->q_full, 0, abort_flag);
-        if (ok) {
-          uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
-          if (ROPE && qrow < len)
-            rope_row_smem<HD>(qt, CF::kQChunk0, r, prm.pos[2 * (seg0 + qrow)],
-                              prm.pos[2 * (seg0 + qrow) + 1], fr);
-          if (HD == 72)  // zero the 8 padding columns 72..79 (logical unit 9)
-            *reinterpret_cast<uint4 *>(qt + unit_offset<HD>(r, 9, CF::kQChunk0)) =
-                make_uint4(0, 0, 0, 0);
-          fence_proxy_async_smem();
-        }
-        mbar_arrive(&bars->q_ready[t]);
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-      const uint32_t s_addr = tmem + lane_base + CF::tmem_s(t) + half * HC;
-      const uint32_t p_addr = tmem + lane_base + CF::tmem_p(t) + half * (HC / 2);
-      const uint32_t o_addr = tmem + lane_base + CF::tmem_o(t);
-      float *xv = reinterpret_cast<float *>(smem + CF::kXOff) + t * 256;  // [j&1][t][half][row]
-      uint64_t *xb = &bars->xchg[t][quarter];
-      const float sl2 = prm.scale_log2;
-      // head_dim 72: the softmax denominator is accumulated by the tensor core
-      // as O column 72 -- V's first padding column is set to 1.0 before each
-      // P.V -- so the row sum costs no instruction here and sums exactly the
-      // bf16 P the numerator uses.  That also lets P be rounded toward zero
-      // (one byte permute per pair): the rounding's mean cancels between
-      // numerator and denominator and its spread equals round-to-nearest's.
-      // head_dim 128 sums in registers and rounds P to nearest.
-      constexpr bool kSumByMma = (HD == 72);
-      // pairs of this thread's HC exponentials that run on the FMA pipe
-      // instead of the special-function unit (a quarter)
-      constexpr int kPolyPairs = HC / 8;
-      constexpr int kOC = CF::HDP / 16;         // 16-column chunks of O
-      constexpr int kOCHalf = (kOC + 1) / 2;   // rescaled by half 0; the rest by half 1
-      const int oc_lo = half ? kOCHalf : 0, oc_hi = half ? kOC : kOCHalf;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + CF::tmem_s(t) + half * HC;
+    const uint32_t p_addr = tmem + lane_base + CF::tmem_p(t) + half * (HC / 2);
+    const uint32_t o_addr = tmem + lane_base + CF::tmem_o(t);
+    float *xv = reinterpret_cast<float *>(smem + CF::kXOff) + t * 256;  // [phase&1][t][half][row]
+    uint64_t *xb = &bars->xchg[t][quarter];
+    const float sl2 = prm.scale_log2;
+    // head_dim 72: the softmax denominator is accumulated by the tensor core
+    // as O column 72 -- warp 3 sets V's first padding column to 1.0 before
+    // each P.V -- so the row sum costs no instruction here and sums exactly the
+    // bf16 P the numerator uses.  That also lets P be rounded toward zero
+    // (one byte permute per pair): the rounding's mean cancels between
+    // numerator and denominator and its spread equals round-to-nearest's.
+    // head_dim 128 sums in registers and rounds P to nearest.
+    constexpr bool kSumByMma = (HD == 72);
+    // pairs of this thread's HC exponentials that run on the FMA pipe
+    // instead of the special-function unit (a quarter)
+    constexpr int kPolyPairs = HC / 8;
+    constexpr int kOC = CF::HDP / 16;         // 16-column chunks of O
+    constexpr int kOCHalf = (kOC + 1) / 2;   // rescaled by half 0; the rest by half 1
+    const int oc_lo = half ? kOCHalf : 0, oc_hi = half ? kOC : kOCHalf;
+    bool ok = true;
+    uint32_t tc = 0;    // key tiles processed by this query tile so far
+    uint32_t xc = 0;    // row-pair exchanges so far
+    uint32_t act = 0;   // items in which this query tile was active
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      Item it;
+      if (!decode_item(w, prm, BK, it)) continue;
+      if (t >= it.n_tiles_q) continue;
+      const int n_kv = it.n_kv, len = it.len;
+      const int qrow = it.q0 + t * kBlockQ + r;  // row inside the sequence
       float m = -INFINITY;
       uint64_t l2[2] = {0, 0};  // packed partial row sums (head_dim 128)
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (!warp_wait(&bars->s_full[t], j & 1, abort_flag)) { ok = false; break; }
+      for (int j = 0; j < n_kv; ++j) {
+        const uint32_t tj = tc + j, xj_ph = xc + j;
+        if (!warp_wait(&bars->s_full[t], tj & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int nvalid = (j < n_pre ? min(BK, prm.P - j * BK) : min(BK, len - (j - n_pre) * BK)) -
                            half * HC;  // valid keys among this thread's columns
@@ -498,22 +610,31 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if constexpr ((HC - 2) % 4 != 0)
           a0 = fmax3(a0, __uint_as_float(s[HC - 2]), __uint_as_float(s[HC - 1]));
         // swap partial maxima with the thread that holds the row's other half
-        float *xj = xv + (j & 1) * 512;
-        xj[half * 128 + r] = fmaxf(a0, a1) * sl2;
+        float *xj = xv + (xj_ph & 1) * 512;
+        const float m_loc = fmaxf(a0, a1) * sl2;
+        xj[half * 128 + r] = m_loc;
         mbar_arrive(xb);
-        if (!warp_wait(xb, j & 1, abort_flag)) { ok = false; break; }
-        const float m_tile = fmaxf(xj[r], xj[128 + r]);
-        const bool grow = __any_sync(0xffffffffu, m_tile > m + 8.0f);
-        if (j == 0) {
-          m = m_tile;
-        } else if (grow) {
-          // rescale O (and the row sum) only when the running max grew by
-          // more than 8 in log2 units; otherwise keep the stale max
+        // The row max only matters when it grows by more than 8 (log2 units)
+        // over the running max m; otherwise m stays (stale) and the final
+        // O / l division absorbs it exactly.  So unless this thread already
+        // sees such growth (or it is the first key tile), the exponentials
+        // start with m while the partner's max is on its way, and are redone
+        // in the rare case that the partner's half grows.
+        bool exchanged = false;
+        float m_tile = m;
+        auto take_max = [&]() -> bool {
+          if (!warp_wait(xb, xj_ph & 1, abort_flag)) return false;
+          m_tile = fmaxf(xj[r], xj[128 + r]);
+          exchanged = true;
+          return true;
+        };
+        // rescale O (and the row sum) to a running max that grew by more than 8
+        auto grow_to = [&]() -> bool {
           const bool mine = m_tile > m + 8.0f;
           const float m_new = mine ? m_tile : m;
           const float factor = mine ? ex2_approx(m - m_new) : 1.0f;
           const uint64_t f2 = f2_pack(factor, factor);
-          if (!warp_wait(&bars->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&bars->o_done[t], (tj - 1) & 1, abort_flag)) return false;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < kOC; ++c) {
@@ -537,15 +658,26 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 2; ++k) l2[k] = f2_mul(l2[k], f2);
           m = m_new;
+          return true;
+        };
+        if (j == 0 || __any_sync(0xffffffffu, m_loc > m + 8.0f)) {
+          if (!take_max()) { ok = false; break; }
+          if (j == 0) {
+            m = m_tile;
+          } else if (__any_sync(0xffffffffu, m_tile > m + 8.0f)) {
+            if (!grow_to()) { ok = false; break; }
+          }
         }
         // p = 2^(s*scale*log2e - m) two at a time, packed bf16 pairs; stored
         // to P_t in two pieces (the first once O_t += P_t V_{j-1} has read
         // the previous P_t, which by then has normally finished)
-        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
         constexpr int NP = HC / 2, NP0 = NP >= 16 ? 16 : NP;
         uint32_t pk[NP];
+        const uint64_t sc2 = f2_pack(sl2, sl2);
         auto exp_pairs = [&](auto i0c, auto i1c) {
           constexpr int i0 = decltype(i0c)::value, i1 = decltype(i1c)::value;
+          const uint64_t nm2 = f2_pack(-m, -m);
+          uint64_t lsum[2] = {0, 0};
 #pragma unroll
           for (int i = i0; i < i1; ++i) {
             const uint64_t xa =
@@ -562,81 +694,58 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             if (kSumByMma) {
               pk[i] = pack_bf16x2_trunc(p0, p1);
             } else {
-              l2[i & 1] = f2_add(l2[i & 1], f2_pack(p0, p1));
+              lsum[i & 1] = f2_add(lsum[i & 1], f2_pack(p0, p1));
               pk[i] = pack_bf16x2_alu(p0, p1);
             }
           }
+          return f2_add(lsum[0], lsum[1]);
         };
-        exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
-        if (j > 0 && !warp_wait(&bars->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
+        uint64_t part0 = exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
+        if (!exchanged) {
+          if (!take_max()) { ok = false; break; }
+          if (__any_sync(0xffffffffu, m_tile > m + 8.0f)) {  // the partner's half grew: redo
+            if (!grow_to()) { ok = false; break; }
+            part0 = exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
+          }
+        }
+        if (!kSumByMma) l2[0] = f2_add(l2[0], part0);
+        if (j > 0 && !warp_wait(&bars->o_done[t], (tj - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         tmem_st_cols<NP0>(p_addr, pk);
         if constexpr (NP > NP0) {
-          exp_pairs(std::integral_constant<int, NP0>{}, std::integral_constant<int, NP>{});
+          const uint64_t part1 =
+              exp_pairs(std::integral_constant<int, NP0>{}, std::integral_constant<int, NP>{});
+          if (!kSumByMma) l2[1] = f2_add(l2[1], part1);
           tmem_st_cols<NP - NP0>(p_addr + NP0, pk + NP0);
         }
-        if (kSumByMma && half == 0 && r < BK) {
-          // ones in V's column 72 of this key tile (the first padding column);
-          // both query tiles write it (the same value) so that each tile's
-          // P.V depends only on its own softmax
-          const int st = j % NS;
-          if (!mbar_wait(&bars->v_full[st], (j / NS) & 1, abort_flag)) ok = false;
-          if (ok) {
-            // dim 72: 16-byte unit 1 of the fifth 32B-swizzled chunk
-            *reinterpret_cast<uint16_t *>(smem + CF::kVOff + st * CF::kKTile + 4 * CF::kVChunk +
-                                          r * 32 + ((1 ^ ((r >> 2) & 1)) << 4)) = 0x3F80u;  // 1.0
-            fence_proxy_async_smem();
-          }
-        }
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_full[t]);
       }
+      if (!ok) break;
       // epilogue: O / l -> bf16 rows of o [T, H, HD], each thread its half of the row
-      if (ok && warp_wait(&bars->o_done[t], (n_kv - 1) & 1, abort_flag)) {
-        tc_fence_after();
-        float l = 0.0f;
-        bool have_l = true;
-        if (!kSumByMma) {  // add the two halves' partial sums
-          float a, b, c2, d2;
-          f2_unpack(l2[0], a, b);
-          f2_unpack(l2[1], c2, d2);
-          float *xj = xv + (n_kv & 1) * 512;
-          xj[half * 128 + r] = (a + b) + (c2 + d2);
-          mbar_arrive(xb);
-          have_l = warp_wait(xb, n_kv & 1, abort_flag);
-          l = xj[r] + xj[128 + r];
-        }
-        if (have_l) {
-          __nv_bfloat16 *orow =
-              qrow < len ? prm.o + size_t(seg0 + qrow) * prm.C + size_t(h) * HD : nullptr;
-          if (half == 0)
-            store_o_half<HD, 0>(o_addr, l, orow);
-          else
-            store_o_half<HD, 1>(o_addr, l, orow);
-        }
+      if (!warp_wait(&bars->o_done[t], (tc + n_kv - 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float l = 0.0f;
+      if (!kSumByMma) {  // add the two halves' partial sums
+        float a, b, c2, d2;
+        f2_unpack(l2[0], a, b);
+        f2_unpack(l2[1], c2, d2);
+        float *xj = xv + ((xc + n_kv) & 1) * 512;
+        xj[half * 128 + r] = (a + b) + (c2 + d2);
+        mbar_arrive(xb);
+        if (!warp_wait(xb, (xc + n_kv) & 1, abort_flag)) { ok = false; break; }
+        l = xj[r] + xj[128 + r];
       }
-    }
-  } else if (ROPE && warp == 3) {
-    // ------------------------------------------------------------ K rotation
-    // thread rotates key rows lane, lane + 32, ... of each own-key tile
-    const int r0 = lane;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j % NS;
-      const uint32_t f = (j / NS) & 1;
-      if (!mbar_wait(&bars->k_full[st], f, abort_flag)) break;
-      if (j >= n_pre) {
-#pragma unroll 1
-        for (int r = r0; r < BK; r += 32) {
-          const int key = (j - n_pre) * BK + r;
-          if (key < len)
-            rope_row_smem<HD>(smem + CF::kKOff + st * CF::kKTile, CF::kKChunk0, r,
-                              prm.pos[2 * (seg0 + key)], prm.pos[2 * (seg0 + key) + 1], fr);
-        }
-        fence_proxy_async_smem();
-      }
-      mbar_arrive(&bars->k_ready[st]);
+      __nv_bfloat16 *orow =
+          qrow < len ? prm.o + size_t(it.seg0 + qrow) * prm.C + size_t(it.h) * HD : nullptr;
+      if (half == 0)
+        store_o_half<HD, 0>(o_addr, l, orow);
+      else
+        store_o_half<HD, 1>(o_addr, l, orow);
+      tc += n_kv;
+      xc += n_kv + (kSumByMma ? 0 : 1);
+      ++act;
     }
   }
 
@@ -665,7 +774,6 @@ static cudaError_t launch_hd(const CUtensorMap *maps, const attn::Params &prm, i
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,
                                 float scale, const RopeFreqs &fr, int num_sms, int *status,
                                 cudaStream_t st) {
-  (void)num_sms;
   if (s.total_tokens == 0 || s.max_seqlen == 0) return cudaSuccess;
   const int C = H * d;
   const int Hkv = s.kv_heads > 0 ? s.kv_heads : H;
@@ -706,12 +814,20 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
   prm.Hkv = Hkv;
   prm.P = P;
   prm.n_pairs = (s.max_seqlen + 2 * attn::kBlockQ - 1) / (2 * attn::kBlockQ);
+  prm.n_seqs = s.n_seqs;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.cu = s.cu_seqlens;
   prm.pos = s.pos;
   prm.o = static_cast<__nv_bfloat16 *>(o);
   prm.status = status;
-  const int grid = prm.n_pairs * H * s.n_seqs;
+  const int n_items = prm.n_pairs * H * s.n_seqs;
+  // persistent (one CTA per SM walking the items) or one CTA per item
+  static const int grid_mode = [] {
+    const char *e = getenv("VIT_ATTN_GRID");
+    return e ? atoi(e) : 0;
+  }();
+  const bool persistent = grid_mode == 1 || (grid_mode == 0 && d == 72);
+  const int grid = (persistent && n_items > num_sms) ? num_sms : n_items;
   const bool rope = s.pos != nullptr;
   if (d == 72)
     return rope ? launch_hd<72, true>(maps, prm, grid, fr, st)

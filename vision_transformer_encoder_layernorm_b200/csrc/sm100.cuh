@@ -304,6 +304,18 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t *r) 
   }
 }
 
+// Warpgroup register reallocation: every warp of a warpgroup executes the
+// same one.  The increases of all warpgroups must fit in what the decreases
+// free from the registers the CTA was launched with.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Packed fp32x2 arithmetic (one instruction for two lanes of fp32 data).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
