@@ -567,8 +567,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     // head_dim 128 sums in registers and rounds P to nearest.
     constexpr bool kSumByMma = (HD == 72);
     // pairs of this thread's HC exponentials that run on the FMA pipe
-    // instead of the special-function unit (a quarter)
-    constexpr int kPolyPairs = HC / 8;
+    // instead of the special-function unit (about a tenth)
+    constexpr int kPolyPairs = HC / 16;
     constexpr int kOC = CF::HDP / 16;         // 16-column chunks of O
     constexpr int kOCHalf = (kOC + 1) / 2;   // rescaled by half 0; the rest by half 1
     const int oc_lo = half ? kOCHalf : 0, oc_hi = half ? kOC : kOCHalf;
