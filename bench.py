@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="enqueue the library calls every step instead of replaying a CUDA graph")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiler captures only: run this many layers (line marked partial)")
     return ap.parse_args()
@@ -253,9 +255,23 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # > 126 MB L2
     stream = torch.cuda.current_stream()
 
+    def direct_step(st=stream):
+        ctx.encoder_forward(lw_structs, x, y, sq, ws, st)
+        ctx.spatial_merge_2x2(y, out, wl.grids, C, st)
+
+    # one step = the 27-layer stack + merge, replayed as a CUDA graph of the
+    # library's launches (vit_graph_*), or enqueued call by call
+    graph = None
+    if not args.no_graph:
+        cs = ctx.graph_begin()
+        direct_step(cs)
+        graph = ctx.graph_end()
+
     def step():
-        ctx.encoder_forward(lw_structs, x, y, sq, ws, stream)
-        ctx.spatial_merge_2x2(y, out, wl.grids, C, stream)
+        if graph is not None:
+            graph.launch(stream)
+        else:
+            direct_step()
 
     for _ in range(args.warmup):
         step()
@@ -281,6 +297,8 @@ def main():
     barrier()
     clk = clocks.stop()
     launches = sum(n for n, _ in ctx.profile_read(reset=True).values())
+    if graph is not None:  # replays do not pass through the host-side counters
+        launches = graph.kernels * args.steps
     step_ms = [a.elapsed_time(b) for a, b in ev]
     t_ms = float(np.mean(step_ms))
     t_ms = replicas.max_over_ranks(t_ms, device="cuda")
@@ -290,7 +308,7 @@ def main():
     ctx.profile_enable(True)
     for _ in range(max(2, min(args.steps, 5))):
         flush.zero_()
-        step()
+        direct_step()
     torch.cuda.synchronize()
     prof = ctx.profile_read(reset=True)
     ctx.profile_enable(False)
@@ -335,12 +353,10 @@ def main():
         hx = torch.empty((T, C), dtype=torch.bfloat16, pin_memory=True)
         hx.copy_(x.cpu())
         hout = torch.empty((T // 4, 4 * C), dtype=torch.bfloat16, pin_memory=True)
-        xin = torch.empty_like(x)
 
         def e2e_step():
-            xin.copy_(hx, non_blocking=True)
-            ctx.encoder_forward(lw_structs, xin, y, sq, ws, stream)
-            ctx.spatial_merge_2x2(y, out, wl.grids, C, stream)
+            x.copy_(hx, non_blocking=True)
+            step()
             hout.copy_(out, non_blocking=True)
 
         for _ in range(2):
@@ -380,7 +396,9 @@ def main():
                                    "hidden 1152, 16x72 heads, MLP 4304, + 2x2 merge to 975x4608",
                        "global_batch": world, "seq_len": T,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed before every timed step (256 MiB write)"},
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "launch": ("one CUDA-graph replay of the library's launches per step"
+                                  if graph is not None else "library calls enqueued every step")},
             "tflops": tflops, "pct_bf16_peak": tflops / tensor_peak,
             **({"partial": f"{wl.layers} layers (profiler capture, not a bench line)"}
                if args.layers else {}),
@@ -388,6 +406,8 @@ def main():
             "e2e": e2e, "gpu_launches": launches, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+    if graph is not None:
+        graph.close()
     ctx.close()
     if dist is not None:
         dist.barrier()

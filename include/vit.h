@@ -167,6 +167,26 @@ VIT_API vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *la
                                const vit_seqs *seqs, void *workspace,
                                size_t ws_bytes, void *stream);
 
+/* ---- CUDA graphs of library calls --------------------------------------
+ * Stream capture, so a whole stack (and the merge) replays with one launch.
+ * vit_graph_begin returns a stream owned by the context; enqueue any calls of
+ * this context on it (their arguments are checked as usual), then
+ * vit_graph_end instantiates the captured work into *out.  Every pointer
+ * and size passed while capturing is baked into the graph: each launch
+ * re-runs the same kernels on the same buffers, which the caller keeps
+ * alive and may refill between launches.  One capture per context at a
+ * time (else VIT_ERR_INVALID_ARG); a failed capture returns VIT_ERR_CUDA
+ * and leaves *out NULL.  The pages have no counterpart: their runtime
+ * launches op by op without CUDA graphs (KLiteInfer README, section
+ * 已知限制与后续).
+ * vit_graph_kernels: this library's kernel launches in one replay. */
+typedef struct vit_graph vit_graph;
+VIT_API vit_status vit_graph_begin(vit_ctx *ctx, void **capture_stream);
+VIT_API vit_status vit_graph_end(vit_ctx *ctx, vit_graph **out);
+VIT_API vit_status vit_graph_launch(vit_graph *g, void *stream);
+VIT_API long long vit_graph_kernels(const vit_graph *g);
+VIT_API void vit_graph_destroy(vit_graph *g);
+
 /* Bidirectional multi-head attention over packed sequences ("视觉算子":
  * softmax(Q K^T * scale) V per head and sequence).  qkv [T, 3, H, d]
  * (the QKV projection's output layout), o [T, H, d].  With seqs->pos_rc the

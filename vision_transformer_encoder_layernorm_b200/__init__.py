@@ -18,7 +18,7 @@ from typing import Optional, Sequence
 __all__ = [
     "lib", "LIB_PATH", "VitError", "VitConfig", "VitLayerWeights", "VitSeqs", "Context",
     "F32", "BF16", "FLAG_NO_ROPE", "FLAG_NO_MLP", "EPI_BIAS", "EPI_BIAS_GELU",
-    "EPI_BIAS_RESIDUAL", "STATUS", "ABI_FUNCTIONS", "KERNEL_KINDS",
+    "EPI_BIAS_RESIDUAL", "STATUS", "ABI_FUNCTIONS", "KERNEL_KINDS", "Graph",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvit.so")
@@ -82,6 +82,11 @@ ABI_FUNCTIONS = {
     "vit_profile_enable": (_I, [_P, _I]),
     "vit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_longlong),
                               ctypes.POINTER(ctypes.c_double), _I]),
+    "vit_graph_begin": (_I, [_P, ctypes.POINTER(_P)]),
+    "vit_graph_end": (_I, [_P, ctypes.POINTER(_P)]),
+    "vit_graph_launch": (_I, [_P, _P]),
+    "vit_graph_kernels": (ctypes.c_longlong, [_P]),
+    "vit_graph_destroy": (None, [_P]),
     "vit_get_last_device_status": (_I, [_P]),
     "vit_status_string": (ctypes.c_char_p, [_I]),
     "vit_version": (ctypes.c_char_p, []),
@@ -149,6 +154,29 @@ def seqs(total_tokens: int, n_seqs: int, max_seqlen: int, cu_seqlens, pos_rc=Non
                 _ptr(prefix_kv), prefix_len if prefix_kv is not None else 0, kv_heads)
     s._tensors = (cu_seqlens, pos_rc, prefix_kv)
     return s
+
+
+class Graph:
+    """A captured sequence of library calls (see vit_graph_begin in vit.h).
+    Every pointer used while capturing is baked in: keep those tensors alive."""
+
+    def __init__(self, handle: int):
+        self._h = handle
+        self.kernels = int(lib.vit_graph_kernels(handle))
+
+    def launch(self, stream=None):
+        _check("vit_graph_launch", lib.vit_graph_launch(self._h, _stream(stream)))
+
+    def close(self):
+        if self._h:
+            lib.vit_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class Context:
@@ -234,6 +262,19 @@ class Context:
 
     def profile_enable(self, enable: bool = True):
         _check("vit_profile_enable", lib.vit_profile_enable(self._h, int(bool(enable))))
+
+    def graph_begin(self) -> int:
+        """Starts capturing this context's calls; returns the capture stream
+        (pass it as `stream=` to the calls to record)."""
+        h = _P()
+        _check("vit_graph_begin", lib.vit_graph_begin(self._h, ctypes.byref(h)))
+        return h.value
+
+    def graph_end(self) -> "Graph":
+        """Ends the capture started by graph_begin and returns the graph."""
+        h = _P()
+        _check("vit_graph_end", lib.vit_graph_end(self._h, ctypes.byref(h)))
+        return Graph(h.value)
 
     def profile_read(self, reset: bool = False):
         """{kind name: (launches, total device ms)} for every kernel kind."""

@@ -18,6 +18,8 @@
 
 #include <vector>
 
+#include <new>
+
 #include "../../include/vit.h"
 #include "kernels.h"
 
@@ -64,6 +66,16 @@ struct vit_ctx {
   int *d_status;  // 4 ints; [0] = first error code recorded by a kernel
   vit::RopeFreqs fr;
   VitProfiler prof;
+  // stream capture in progress (vit_graph_begin .. vit_graph_end)
+  cudaStream_t cap_stream = nullptr;
+  bool cap_prof_on = false;
+  long long cap_launches0 = 0;
+};
+
+struct vit_graph {
+  cudaGraphExec_t exec = nullptr;
+  int device = 0;
+  long long kernels = 0;  // library kernel launches captured
 };
 
 namespace {
@@ -273,6 +285,84 @@ const char *vit_status_string(vit_status s) {
     case VIT_ERR_DEVICE_BOUNDS: return "VIT_ERR_DEVICE_BOUNDS";
   }
   return "VIT_ERR_UNKNOWN";
+}
+
+// ---------------------------------------------------------------- CUDA graphs
+// Stream capture of any sequence of this library's calls: the caller enqueues
+// them on the stream vit_graph_begin returns; vit_graph_end instantiates the
+// captured work (launches keep their programmatic-dependent-launch edges).
+// Per-launch profiling events are off during the capture.
+
+static long long total_launches(const vit_ctx *ctx) {
+  long long n = 0;
+  for (long long l : ctx->prof.launches) n += l;
+  return n;
+}
+
+vit_status vit_graph_begin(vit_ctx *ctx, void **capture_stream) {
+  if (!ctx || !capture_stream) return VIT_ERR_INVALID_ARG;
+  *capture_stream = nullptr;
+  if (ctx->cap_stream) return VIT_ERR_INVALID_ARG;  // one capture at a time per context
+  DeviceGuard g(ctx->device);
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return VIT_ERR_CUDA;
+  // relaxed: the launch paths may query or set function attributes while capturing
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return VIT_ERR_CUDA;
+  }
+  ctx->cap_stream = cs;
+  ctx->cap_prof_on = ctx->prof.on;
+  ctx->prof.on = false;
+  ctx->cap_launches0 = total_launches(ctx);
+  *capture_stream = cs;
+  return VIT_OK;
+}
+
+vit_status vit_graph_end(vit_ctx *ctx, vit_graph **out) {
+  if (!ctx || !out) return VIT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!ctx->cap_stream) return VIT_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(ctx->cap_stream, &graph);
+  cudaStreamDestroy(ctx->cap_stream);
+  ctx->cap_stream = nullptr;
+  ctx->prof.on = ctx->cap_prof_on;
+  const long long kernels = total_launches(ctx) - ctx->cap_launches0;
+  if (e != cudaSuccess || graph == nullptr) {
+    if (graph) cudaGraphDestroy(graph);
+    return VIT_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ei != cudaSuccess) return VIT_ERR_CUDA;
+  vit_graph *gr = new (std::nothrow) vit_graph;
+  if (!gr) {
+    cudaGraphExecDestroy(exec);
+    return VIT_ERR_CUDA;
+  }
+  gr->exec = exec;
+  gr->device = ctx->device;
+  gr->kernels = kernels;
+  *out = gr;
+  return VIT_OK;
+}
+
+vit_status vit_graph_launch(vit_graph *g, void *stream) {
+  if (!g) return VIT_ERR_INVALID_ARG;
+  DeviceGuard dg(g->device);
+  return cuda_status(cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)));
+}
+
+long long vit_graph_kernels(const vit_graph *g) { return g ? g->kernels : 0; }
+
+void vit_graph_destroy(vit_graph *g) {
+  if (!g) return;
+  DeviceGuard dg(g->device);
+  cudaGraphExecDestroy(g->exec);
+  delete g;
 }
 
 const char *vit_version(void) { return "libvit 0.1 sm_100a"; }
