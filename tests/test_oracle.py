@@ -385,3 +385,59 @@ def test_workload_flop_counts():
     assert f["gemm"] == 27 * 2.0 * T * C * (4 * C + 2 * Fm)
     assert f["attn"] == 27 * 4.0 * T * T * C
     assert abs(f["total"] - 5.0987e12) / 5.0987e12 < 1e-4
+
+
+# ------------------------------------------------------------------ embedding
+from oracle import embed_ref as E  # noqa: E402
+
+
+@pytest.mark.parametrize("p,rows,cols,C", [(14, 3, 5, 24), (4, 2, 2, 8), (2, 1, 3, 5)])
+def test_patch_embed_matches_conv2d(p, rows, cols, C):
+    r = rng(70 + p)
+    img = r.standard_normal((3, rows * p, cols * p))
+    w = r.standard_normal((C, 3, p, p))
+    b = r.standard_normal(C)
+    got = E.patch_embed(img, w.reshape(C, -1), b, p)
+    ref = F.conv2d(torch.tensor(img)[None], torch.tensor(w), torch.tensor(b), stride=p)
+    ref = ref[0].permute(1, 2, 0).reshape(rows * cols, C).numpy()  # tokens row-major
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("gh,gw,oh,ow", [(27, 27, 50, 78), (27, 27, 6, 4), (5, 7, 5, 7),
+                                         (4, 3, 9, 2), (1, 1, 3, 3), (6, 6, 1, 1)])
+def test_bilinear_matches_torch_interpolate(gh, gw, oh, ow):
+    t = rng(80 + oh).standard_normal((gh, gw, 3))
+    got = E.bilinear_resize(t, oh, ow)
+    ref = F.interpolate(torch.tensor(t).permute(2, 0, 1)[None], size=(oh, ow), mode="bilinear",
+                        align_corners=False)[0].permute(1, 2, 0).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_bilinear_affine_closed_form():
+    # table value 2y + x on a 2x2 grid; 4 outputs per axis sit at the clamped
+    # half-pixel source coordinates 0, 1/4, 3/4, 1, where bilinear
+    # interpolation reproduces the affine function exactly
+    t = np.array([[0.0, 1.0], [2.0, 3.0]])[:, :, None]
+    got = E.bilinear_resize(t, 4, 4)[:, :, 0]
+    c = np.array([0.0, 0.25, 0.75, 1.0])
+    np.testing.assert_array_equal(got, 2 * c[:, None] + c[None, :])
+
+
+def test_bilinear_identity_and_constant():
+    t = rng(90).standard_normal((5, 6, 4))
+    np.testing.assert_array_equal(E.bilinear_resize(t, 5, 6), t)  # s = i exactly
+    k = np.full((3, 4, 2), 1.75)
+    np.testing.assert_allclose(E.bilinear_resize(k, 7, 11), 1.75, rtol=0, atol=1e-15)
+
+
+def test_embed_images_packs_images_in_order():
+    r = rng(91)
+    p, C = 2, 6
+    grids = [(2, 3), (1, 2)]
+    imgs = [r.standard_normal((3, a * p, b * p)) for a, b in grids]
+    w, b, t = r.standard_normal((C, 12)), r.standard_normal(C), r.standard_normal((4, 4, C))
+    got = E.embed_images(imgs, grids, p, w, b, t)
+    assert got.shape == (8, C)
+    first = E.patch_embed(imgs[0], w, b, p) + E.bilinear_resize(t, 2, 3).reshape(6, C)
+    second = E.patch_embed(imgs[1], w, b, p) + E.bilinear_resize(t, 1, 2).reshape(2, C)
+    np.testing.assert_array_equal(got, np.concatenate([first, second]))
