@@ -376,6 +376,35 @@ def main():
         e2e = {"value": world * T / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": hx.numel() * hx.element_size(),
                "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    # ---- beyond the encoder: patch embedding of the same image (50 x 78
+    # patches of 14 x 14 pixels, 27 x 27 position table), timed on its own
+    nxt = None
+    if world == 1 and not args.layers:
+        ei = synth.make_embed_inputs(wl, patch=14, table_hw=(27, 27))
+        px = dev(np.concatenate([im.reshape(-1) for im in ei.images]))
+        w_pe, b_pe, table = dev(ei.w_pe), dev(ei.b_pe), dev(ei.table)
+        emb = torch.empty((T, C), dtype=torch.bfloat16, device="cuda")
+        ews = torch.empty(ctx.embed_workspace_bytes(T, 14), dtype=torch.uint8, device="cuda")
+        cs = ctx.graph_begin()  # device time of the 4 launches, no host gaps
+        ctx.patch_embed(px, wl.grids, 14, w_pe, b_pe, table, emb, ews, cs)
+        eg = ctx.graph_end()
+        for _ in range(3):
+            eg.launch(stream)
+        n_rep = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        e0.record(stream)
+        for _ in range(n_rep):
+            eg.launch(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        eg.close()
+        us = e0.elapsed_time(e1) * 1e3 / n_rep
+        fl = 2.0 * T * C * 3 * 14 * 14
+        nxt = {"patch_embed": {"workload": "3900 tokens (50x78 patches of 14x14x3), C 1152, "
+                                           "27x27 position table", "us": us,
+                               "tflops": fl / us / 1e6, "frac_bf16_sustained": fl / us / 1e6 / tensor_peak,
+                               "launches": 4, "note": "graph replays back to back, inputs in L2"}}
     if ctx.device_status() != 0:
         raise RuntimeError("device status set during the benchmark")
 
@@ -404,6 +433,7 @@ def main():
                if args.layers else {}),
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+            **({"next": nxt} if nxt else {}),
         }
         print(json.dumps(line), flush=True)
     if graph is not None:

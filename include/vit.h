@@ -211,6 +211,34 @@ VIT_API vit_status vit_positions_from_grids(vit_ctx *ctx, const int32_t *grids_h
                                     int n_images, int32_t *cu_seqlens,
                                     int32_t *pos_rc, void *stream);
 
+/* ---- before the encoder: patch embedding + interpolated positions -------
+ * KLiteInfer README: section 精度与性能 (patch embedding, the first compared
+ * stage) and section 架构, paragraph 视觉算子 (bilinear position-embedding
+ * interpolation).  The pages give no patch or table size; both are
+ * parameters here.
+ *   pixels     images packed in order, image i [3, rows_i*patch,
+ *              cols_i*patch], channels first, ctx dtype
+ *   grids      HOST int32 [n_images, 2] = (rows, cols) in patches
+ *   w_pe       [C, 3*patch*patch]: a stride-patch Conv2d weight [C, 3, patch,
+ *              patch], flattened in (channel, y, x) order; b_pe [C]
+ *   pos_table  [table_h, table_w, C]
+ *   y          [T, C], T = sum rows*cols; token r*cols + c of image i
+ * y = patch(t) . w_pe^T + b_pe + table resized bilinearly (half-pixel
+ * centres, as PyTorch's align_corners = false) to (rows, cols) at (r, c).
+ * 1 <= patch <= 32, n_images <= 1024, C % 8 == 0; b_pe, pos_table, y and the
+ * workspace 16-byte aligned.  Workspace:
+ * vit_embed_workspace_bytes (patches, padded weight, interpolated table). */
+VIT_API size_t vit_embed_workspace_bytes(const vit_ctx *ctx, int total_tokens, int patch);
+VIT_API vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels,
+                                   const int32_t *grids_hw_host, int n_images, int patch,
+                                   const void *w_pe, const void *b_pe, const void *pos_table,
+                                   int table_h, int table_w, void *y, void *workspace,
+                                   size_t ws_bytes, void *stream);
+/* The interpolation alone: y [T, C] = resized pos_table per image (as above). */
+VIT_API vit_status vit_pos_interp(vit_ctx *ctx, const void *pos_table, int table_h, int table_w,
+                                  const int32_t *grids_hw_host, int n_images, void *y,
+                                  void *stream);
+
 /* ---- single steps of the layer, exposed for step-level use and testing --- */
 
 /* LayerNorm over the last axis ("视觉算子": LayerNorm), biased variance,
@@ -247,8 +275,9 @@ VIT_API vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc,
 typedef enum {
   VIT_K_LAYERNORM = 0, VIT_K_GEMM_QKV = 1, VIT_K_ROPE = 2, VIT_K_ATTENTION = 3,
   VIT_K_GEMM_OUT = 4, VIT_K_GEMM_FC1 = 5, VIT_K_GEMM_FC2 = 6, VIT_K_MERGE = 7,
-  VIT_K_POSITIONS = 8, VIT_K_GEMM = 9, /* vit_linear */
-  VIT_K_COUNT = 10
+  VIT_K_POSITIONS = 8, VIT_K_GEMM = 9, /* vit_linear, the patch projection */
+  VIT_K_EMBED = 10, /* patch extraction, weight padding, position interpolation */
+  VIT_K_COUNT = 11
 } vit_kernel_kind;
 
 /* enable != 0: every later kernel launch of this context is bracketed by two

@@ -222,3 +222,29 @@ def random_tensor(shape, seed: int, dtype: str, scale: float = 1.0) -> np.ndarra
     tests of single steps."""
     rng = np.random.Generator(np.random.PCG64(seed))
     return from_f64(scale * rng.standard_normal(shape), dtype)
+
+
+@dataclass
+class EmbedInputs:
+    """Inputs of the patch embedding (the step before the encoder)."""
+    grids: List[Tuple[int, int]]
+    patch: int
+    images: List[np.ndarray]   # per image [3, rows*patch, cols*patch], storage dtype
+    w_pe: np.ndarray           # [C, 3*patch*patch]
+    b_pe: np.ndarray           # [C]
+    table: np.ndarray          # [table_h, table_w, C]
+
+
+def make_embed_inputs(wl: Workload, patch: int = 14, table_hw: Tuple[int, int] = (27, 27),
+                      seed: Optional[int] = None) -> EmbedInputs:
+    """Seeded synthetic pixels (N(0, 1), as normalised images) and a random
+    patch projection (N(0, 0.02), bias N(0, 0.01)) and position table
+    (N(0, 0.02)) for the workload's image grids; draw order: images, w_pe,
+    b_pe, table."""
+    rng = np.random.Generator(np.random.PCG64(wl.seed + 1000 if seed is None else seed))
+    C = wl.hidden
+    imgs = [from_f64(rng.standard_normal((3, r * patch, c * patch)), wl.dtype) for r, c in wl.grids]
+    w = from_f64(0.02 * rng.standard_normal((C, 3 * patch * patch)), wl.dtype)
+    b = from_f64(0.01 * rng.standard_normal(C), wl.dtype)
+    t = from_f64(0.02 * rng.standard_normal((table_hw[0], table_hw[1], C)), wl.dtype)
+    return EmbedInputs(list(wl.grids), patch, imgs, w, b, t)

@@ -27,7 +27,7 @@ F32, BF16 = 0, 1
 FLAG_NO_ROPE, FLAG_NO_MLP = 0x1, 0x2
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_RESIDUAL = 0, 1, 2
 KERNEL_KINDS = ("layernorm", "gemm_qkv", "rope", "attention", "gemm_out", "gemm_fc1",
-                "gemm_fc2", "merge", "positions", "gemm")
+                "gemm_fc2", "merge", "positions", "gemm", "embed")
 STATUS = {0: "VIT_OK", 1: "VIT_ERR_INVALID_ARG", 2: "VIT_ERR_SHAPE", 3: "VIT_ERR_UNSUPPORTED",
           4: "VIT_ERR_WORKSPACE", 5: "VIT_ERR_CUDA", 6: "VIT_ERR_TIMEOUT",
           7: "VIT_ERR_DEVICE_BOUNDS"}
@@ -82,6 +82,10 @@ ABI_FUNCTIONS = {
     "vit_profile_enable": (_I, [_P, _I]),
     "vit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_longlong),
                               ctypes.POINTER(ctypes.c_double), _I]),
+    "vit_embed_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I]),
+    "vit_patch_embed": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32), _I, _I, _P, _P, _P, _I, _I,
+                             _P, _P, ctypes.c_size_t, _P]),
+    "vit_pos_interp": (_I, [_P, _P, _I, _I, ctypes.POINTER(ctypes.c_int32), _I, _P, _P]),
     "vit_graph_begin": (_I, [_P, ctypes.POINTER(_P)]),
     "vit_graph_end": (_I, [_P, ctypes.POINTER(_P)]),
     "vit_graph_launch": (_I, [_P, _P]),
@@ -262,6 +266,26 @@ class Context:
 
     def profile_enable(self, enable: bool = True):
         _check("vit_profile_enable", lib.vit_profile_enable(self._h, int(bool(enable))))
+
+    def embed_workspace_bytes(self, total_tokens: int, patch: int) -> int:
+        return int(lib.vit_embed_workspace_bytes(self._h, total_tokens, patch))
+
+    def patch_embed(self, pixels, grids, patch: int, w_pe, b_pe, pos_table, y, workspace,
+                    stream=None):
+        """Tokens y [T, C] of packed images (pixels: all images' [3, rows*patch,
+        cols*patch] back to back); pos_table [table_h, table_w, C]."""
+        arr, n = _grids_arr(grids)
+        th, tw = int(pos_table.shape[0]), int(pos_table.shape[1])
+        _check("vit_patch_embed", lib.vit_patch_embed(
+            self._h, _ptr(pixels), arr, n, patch, _ptr(w_pe), _ptr(b_pe), _ptr(pos_table), th, tw,
+            _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream)))
+
+    def pos_interp(self, pos_table, grids, y, stream=None):
+        arr, n = _grids_arr(grids)
+        _check("vit_pos_interp", lib.vit_pos_interp(
+            self._h, _ptr(pos_table), int(pos_table.shape[0]), int(pos_table.shape[1]), arr, n,
+            _ptr(y), _stream(stream)))
 
     def graph_begin(self) -> int:
         """Starts capturing this context's calls; returns the capture stream

@@ -1,0 +1,178 @@
+// k_embed.cu -- the steps before the encoder: patch extraction for the patch
+// embedding GEMM, and the bilinear interpolation of the position table.
+//
+// KLiteInfer README, section "精度与性能" (patch embedding is the first of
+// the compared stages) and section "架构", paragraph "视觉算子" (bilinear
+// position-embedding interpolation).  Image i is [3, rows*p, cols*p],
+// channels first, packed after image i-1; its tokens are its patches in
+// row-major order, token t of the packed sequence starting at base(i).  A
+// token's patch is flattened in (channel, y, x) order, as a Conv2d weight
+// [C, 3, p, p] is, so the embedding is one GEMM against the weight viewed as
+// [C, 3*p*p].  The table [gh, gw, C] is resized to (rows, cols) with
+// half-pixel centres (PyTorch's bilinear default, align_corners = false).
+#include "kernels.h"
+
+namespace vit {
+
+// ---------------------------------------------------------------- patches
+// patches [T, Kp] (Kp = 3*p*p rounded up to a multiple of 8, zero padded).
+// Block (x, image): kTokPerBlock tokens of the image, the threads across
+// each token's Kp entries.  Image i's pixels start at base(i) * 3 * p * p.
+constexpr int kTokPerBlock = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(256) patchify_kernel(const __grid_constant__ ImageTable tab,
+                                                        const T *__restrict__ px,
+                                                        T *__restrict__ out, int p, int kp) {
+  pdl_trigger();
+  pdl_wait();
+  const ImageEntry im = tab.img[blockIdx.y];
+  const int n_tok = im.rows * im.cols;
+  const int pp = p * p, k3 = 3 * pp;
+  const int W = im.cols * p, Hh = im.rows * p;
+  const T *img = px + (long long)im.base * k3;
+  for (int tt = 0; tt < kTokPerBlock; ++tt) {
+    const int tok = blockIdx.x * kTokPerBlock + tt;
+    if (tok >= n_tok) break;
+    const int r = tok / im.cols, c = tok - r * im.cols;
+    const T *src = img + (long long)(r * p) * W + c * p;
+    T *dst = out + (long long)(im.base + tok) * kp;
+    for (int k = threadIdx.x; k < kp; k += blockDim.x) {
+      T v = from_f32<T>(0.0f);
+      if (k < k3) {
+        const int ch = k / pp, rem = k - ch * pp, y = rem / p, x = rem - y * p;
+        v = src[((long long)ch * Hh + y) * W + x];
+      }
+      dst[k] = v;
+    }
+  }
+}
+
+// w [N, K] -> w_pad [N, Kp], zero columns K..Kp-1; block per row
+template <typename T>
+__global__ void __launch_bounds__(256) pad_cols_kernel(const T *__restrict__ w, T *__restrict__ out,
+                                                        int k, int kp) {
+  pdl_trigger();
+  pdl_wait();
+  const T *src = w + (long long)blockIdx.x * k;
+  T *dst = out + (long long)blockIdx.x * kp;
+  for (int col = threadIdx.x; col < kp; col += blockDim.x)
+    dst[col] = col < k ? src[col] : from_f32<T>(0.0f);
+}
+
+// ---------------------------------------------------------------- position table
+// Source index of output i of n along an axis of g table entries, with
+// half-pixel centres: s = (i + 1/2) g / n - 1/2 = ((2i + 1) g - n) / (2n),
+// clamped below at 0.  Integer floor, so the neighbours are exact.
+__device__ __forceinline__ void bilinear_axis(int i, int n, int g, int &i0, int &i1, float &w1) {
+  const long long num = (2LL * i + 1) * g - n, den = 2LL * n;
+  if (num <= 0) {
+    i0 = 0;
+    w1 = 0.0f;
+  } else {
+    i0 = int(num / den);
+    w1 = float(num - den * i0) / float(den);
+  }
+  i1 = min(i0 + 1, g - 1);
+}
+
+template <typename T>
+struct Vec8;  // eight elements, one or two aligned 16-byte loads
+template <>
+struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16 *q, float (&f)[8]) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(q);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16_lo(w[i]);
+      f[2 * i + 1] = bf16_hi(w[i]);
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *q, const float (&f)[8]) {
+    *reinterpret_cast<uint4 *>(q) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                               pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+  }
+};
+template <>
+struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float *q, float (&f)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(q), b = *reinterpret_cast<const float4 *>(q + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float *q, const float (&f)[8]) {
+    *reinterpret_cast<float4 *>(q) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4 *>(q + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  }
+};
+
+// y[base(i) + r*cols + c, :] = bilinear(table)[r, c, :]; block (token, image),
+// one thread per 8 channels (C % 8 == 0), fp32 arithmetic.
+template <typename T>
+__global__ void __launch_bounds__(128) pos_interp_kernel(const __grid_constant__ ImageTable tab,
+                                                          const T *__restrict__ table, int gh,
+                                                          int gw, int C, T *__restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
+  const ImageEntry im = tab.img[blockIdx.y];
+  const int tok = blockIdx.x;
+  if (tok >= im.rows * im.cols) return;
+  const int r = tok / im.cols, c = tok - r * im.cols;
+  int y0, y1, x0, x1;
+  float wy, wx;
+  bilinear_axis(r, im.rows, gh, y0, y1, wy);
+  bilinear_axis(c, im.cols, gw, x0, x1, wx);
+  const T *t00 = table + ((long long)y0 * gw + x0) * C, *t01 = table + ((long long)y0 * gw + x1) * C;
+  const T *t10 = table + ((long long)y1 * gw + x0) * C, *t11 = table + ((long long)y1 * gw + x1) * C;
+  T *out = y + (long long)(im.base + tok) * C;
+  for (int ch = threadIdx.x * 8; ch < C; ch += blockDim.x * 8) {
+    float a[8], b[8], d[8], f[8], o[8];
+    Vec8<T>::load(t00 + ch, a);
+    Vec8<T>::load(t01 + ch, b);
+    Vec8<T>::load(t10 + ch, d);
+    Vec8<T>::load(t11 + ch, f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float top = (1.0f - wx) * a[u] + wx * b[u];
+      const float bot = (1.0f - wx) * d[u] + wx * f[u];
+      o[u] = (1.0f - wy) * top + wy * bot;
+    }
+    Vec8<T>::store(out + ch, o);
+  }
+}
+
+cudaError_t launch_patchify(int dtype, const ImageTable &tab, int n_images, long long max_tokens,
+                            const void *px, void *out, int p, int kp, cudaStream_t st) {
+  if (n_images == 0 || max_tokens == 0) return cudaSuccess;
+  const dim3 grid(unsigned((max_tokens + kTokPerBlock - 1) / kTokPerBlock), n_images);
+  if (dtype == kF32)
+    return launch_pdl(patchify_kernel<float>, grid, dim3(256), 0, st, 1, tab,
+                      static_cast<const float *>(px), static_cast<float *>(out), p, kp);
+  return launch_pdl(patchify_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, 1, tab,
+                    static_cast<const __nv_bfloat16 *>(px), static_cast<__nv_bfloat16 *>(out), p,
+                    kp);
+}
+
+cudaError_t launch_pad_cols(int dtype, const void *w, void *out, int n, int k, int kp,
+                            cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  if (dtype == kF32)
+    return launch_pdl(pad_cols_kernel<float>, dim3(n), dim3(256), 0, st, 1,
+                      static_cast<const float *>(w), static_cast<float *>(out), k, kp);
+  return launch_pdl(pad_cols_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 1,
+                    static_cast<const __nv_bfloat16 *>(w), static_cast<__nv_bfloat16 *>(out), k, kp);
+}
+
+cudaError_t launch_pos_interp(int dtype, const ImageTable &tab, int n_images, long long max_tokens,
+                              const void *table, int gh, int gw, int C, void *y, cudaStream_t st) {
+  if (n_images == 0 || max_tokens == 0) return cudaSuccess;
+  const dim3 grid(unsigned(max_tokens), n_images);
+  if (dtype == kF32)
+    return launch_pdl(pos_interp_kernel<float>, grid, dim3(128), 0, st, 1, tab,
+                      static_cast<const float *>(table), gh, gw, C, static_cast<float *>(y));
+  return launch_pdl(pos_interp_kernel<__nv_bfloat16>, grid, dim3(128), 0, st, 1, tab,
+                    static_cast<const __nv_bfloat16 *>(table), gh, gw, C,
+                    static_cast<__nv_bfloat16 *>(y));
+}
+
+}  // namespace vit

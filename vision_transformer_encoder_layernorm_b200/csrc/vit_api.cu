@@ -271,6 +271,47 @@ vit_status check_layer_call(vit_ctx *ctx, const void *x, void *y, const vit_seqs
 
 }  // namespace
 
+// ---------------------------------------------------------------- embedding helpers
+namespace {
+
+int embed_kp(int patch) { return (3 * patch * patch + 7) & ~7; }  // TMA rows: 16-byte multiples
+
+// Validates the image grids (host) and packs them into launch tables of at
+// most kMaxImagesPerLaunch images; returns the total token count (or < 0).
+long long embed_tokens(const int32_t *grids, int n_images) {
+  if (!grids || n_images < 1 || n_images > 1024) return -1;
+  long long t = 0;
+  for (int i = 0; i < n_images; ++i) {
+    const int r = grids[2 * i], c = grids[2 * i + 1];
+    if (r <= 0 || c <= 0) return -2;
+    t += (long long)r * c;
+  }
+  return t > INT32_MAX ? -2 : t;
+}
+
+template <class F>
+cudaError_t for_image_tables(const int32_t *grids, int n_images, F &&f) {
+  long long base = 0;
+  for (int i0 = 0; i0 < n_images; i0 += kMaxImagesPerLaunch) {
+    const int n = std::min(kMaxImagesPerLaunch, n_images - i0);
+    ImageTable tab;
+    long long max_t = 0;
+    for (int i = 0; i < n; ++i) {
+      const int r = grids[2 * (i0 + i)], c = grids[2 * (i0 + i) + 1];
+      tab.img[i].rows = r;
+      tab.img[i].cols = c;
+      tab.img[i].base = int(base);
+      base += (long long)r * c;
+      max_t = std::max(max_t, (long long)r * c);
+    }
+    const cudaError_t e = f(tab, n, max_t);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *vit_status_string(vit_status s) {
@@ -508,6 +549,79 @@ vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w, const void *bi
   return cuda_status(run_linear(ctx, VIT_K_GEMM, x, w, bias,
                                 epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr, y, M, N, K,
                                 int(epi), static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- embedding
+size_t vit_embed_workspace_bytes(const vit_ctx *ctx, int total_tokens, int patch) {
+  if (!ctx || total_tokens < 0 || patch < 1 || patch > 32) return 0;
+  const size_t e = esize(ctx->cfg), kp = size_t(embed_kp(patch)), C = size_t(ctx->cfg.hidden);
+  return align256(size_t(total_tokens) * kp * e) + align256(C * kp * e) +
+         align256(size_t(total_tokens) * C * e);
+}
+
+vit_status vit_pos_interp(vit_ctx *ctx, const void *pos_table, int table_h, int table_w,
+                          const int32_t *grids_hw_host, int n_images, void *y, void *stream) {
+  if (!ctx || !pos_table || !y || table_h < 1 || table_w < 1) return VIT_ERR_INVALID_ARG;
+  const long long T = embed_tokens(grids_hw_host, n_images);
+  if (T == -1) return VIT_ERR_INVALID_ARG;
+  if (T < 0) return VIT_ERR_SHAPE;
+  const int C = ctx->cfg.hidden;
+  if (C % 8) return VIT_ERR_UNSUPPORTED;
+  if (!aligned16(pos_table) || !aligned16(y)) return VIT_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int dt = ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16;
+  return cuda_status(for_image_tables(grids_hw_host, n_images, [&](const ImageTable &tab, int n,
+                                                                  long long max_t) {
+    return counted(ctx, VIT_K_EMBED, st, [&] {
+      return launch_pos_interp(dt, tab, n, max_t, pos_table, table_h, table_w, C, y, st);
+    });
+  }));
+}
+
+vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels, const int32_t *grids_hw_host,
+                           int n_images, int patch, const void *w_pe, const void *b_pe,
+                           const void *pos_table, int table_h, int table_w, void *y,
+                           void *workspace, size_t ws_bytes, void *stream) {
+  if (!ctx || !pixels || !w_pe || !b_pe || !pos_table || !y || !workspace || table_h < 1 ||
+      table_w < 1 || patch < 1 || patch > 32)
+    return VIT_ERR_INVALID_ARG;
+  const long long T = embed_tokens(grids_hw_host, n_images);
+  if (T == -1) return VIT_ERR_INVALID_ARG;
+  if (T < 0) return VIT_ERR_SHAPE;
+  const int C = ctx->cfg.hidden;
+  if (C % 8) return VIT_ERR_UNSUPPORTED;
+  if (ws_bytes < vit_embed_workspace_bytes(ctx, int(T), patch)) return VIT_ERR_WORKSPACE;
+  {
+    const void *ps[4] = {b_pe, pos_table, y, workspace};
+    for (const void *q : ps)
+      if (!aligned16(q)) return VIT_ERR_INVALID_ARG;
+  }
+  const size_t e = esize(ctx->cfg);
+  const int k = 3 * patch * patch, kp = embed_kp(patch);
+  uint8_t *wsb = static_cast<uint8_t *>(workspace);
+  void *patches = wsb;
+  void *w_pad = wsb + align256(size_t(T) * kp * e);
+  void *pos = static_cast<uint8_t *>(w_pad) + align256(size_t(C) * kp * e);
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int dt = ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16;
+  cudaError_t err = for_image_tables(grids_hw_host, n_images, [&](const ImageTable &tab, int n,
+                                                                 long long max_t) {
+    cudaError_t r = counted(ctx, VIT_K_EMBED, st, [&] {
+      return launch_patchify(dt, tab, n, max_t, pixels, patches, patch, kp, st);
+    });
+    if (r != cudaSuccess) return r;
+    return counted(ctx, VIT_K_EMBED, st, [&] {
+      return launch_pos_interp(dt, tab, n, max_t, pos_table, table_h, table_w, C, pos, st);
+    });
+  });
+  if (err != cudaSuccess) return VIT_ERR_CUDA;
+  if (counted(ctx, VIT_K_EMBED, st, [&] { return launch_pad_cols(dt, w_pe, w_pad, C, k, kp, st); }))
+    return VIT_ERR_CUDA;
+  // tokens = patches . w_pad^T + b_pe + interpolated table (residual epilogue)
+  return cuda_status(run_linear(ctx, VIT_K_GEMM, patches, w_pad, b_pe, pos, y, int(T), C, kp,
+                                kEpiResidual, st));
 }
 
 vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc, int total_tokens,
