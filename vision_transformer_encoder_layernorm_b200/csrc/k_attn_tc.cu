@@ -614,27 +614,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const float m_loc = fmaxf(a0, a1) * sl2;
         xj[half * 128 + r] = m_loc;
         mbar_arrive(xb);
+        if (!warp_wait(xb, xj_ph & 1, abort_flag)) { ok = false; break; }
+        const float m_tile = fmaxf(xj[r], xj[128 + r]);
         // The row max only matters when it grows by more than 8 (log2 units)
-        // over the running max m; otherwise m stays (stale) and the final
-        // O / l division absorbs it exactly.  So unless this thread already
-        // sees such growth (or it is the first key tile), the exponentials
-        // start with m while the partner's max is on its way, and are redone
-        // in the rare case that the partner's half grows.
-        bool exchanged = false;
-        float m_tile = m;
-        auto take_max = [&]() -> bool {
-          if (!warp_wait(xb, xj_ph & 1, abort_flag)) return false;
-          m_tile = fmaxf(xj[r], xj[128 + r]);
-          exchanged = true;
-          return true;
-        };
-        // rescale O (and the row sum) to a running max that grew by more than 8
-        auto grow_to = [&]() -> bool {
+        // over the running max m: then O (and the row sum) is rescaled.
+        // Otherwise m stays (stale) and the final O / l division absorbs it
+        // exactly.  (Starting the exponentials with m before the partner's
+        // max arrives measured slower.)
+        if (j == 0) {
+          m = m_tile;
+        } else if (__any_sync(0xffffffffu, m_tile > m + 8.0f)) {
           const bool mine = m_tile > m + 8.0f;
           const float m_new = mine ? m_tile : m;
           const float factor = mine ? ex2_approx(m - m_new) : 1.0f;
           const uint64_t f2 = f2_pack(factor, factor);
-          if (!warp_wait(&bars->o_done[t], (tj - 1) & 1, abort_flag)) return false;
+          if (!warp_wait(&bars->o_done[t], (tj - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < kOC; ++c) {
@@ -658,15 +652,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 2; ++k) l2[k] = f2_mul(l2[k], f2);
           m = m_new;
-          return true;
-        };
-        if (j == 0 || __any_sync(0xffffffffu, m_loc > m + 8.0f)) {
-          if (!take_max()) { ok = false; break; }
-          if (j == 0) {
-            m = m_tile;
-          } else if (__any_sync(0xffffffffu, m_tile > m + 8.0f)) {
-            if (!grow_to()) { ok = false; break; }
-          }
         }
         // p = 2^(s*scale*log2e - m) two at a time, packed bf16 pairs; stored
         // to P_t in two pieces (the first once O_t += P_t V_{j-1} has read
@@ -700,14 +685,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           }
           return f2_add(lsum[0], lsum[1]);
         };
-        uint64_t part0 = exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
-        if (!exchanged) {
-          if (!take_max()) { ok = false; break; }
-          if (__any_sync(0xffffffffu, m_tile > m + 8.0f)) {  // the partner's half grew: redo
-            if (!grow_to()) { ok = false; break; }
-            part0 = exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
-          }
-        }
+        const uint64_t part0 =
+            exp_pairs(std::integral_constant<int, 0>{}, std::integral_constant<int, NP0>{});
         if (!kSumByMma) l2[0] = f2_add(l2[0], part0);
         if (j > 0 && !warp_wait(&bars->o_done[t], (tj - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
