@@ -126,6 +126,32 @@ def test_c2_full_stack_and_merge():
     assert_close(got, ref, 1.0, 0.999, "c2 27-layer stack + merge")
 
 
+def test_c2_one_layer():
+    # one 3900-token layer (the headline's size) against the oracle
+    wl = synth.get("c2").with_(layers=1)
+    inp = synth.make_inputs(wl, layers=1)
+    got = _device_run(wl, inp, merge=False)
+    ref = orun.run_layers(inp)
+    assert_close(got, ref, 2e-2, 0.9999, "c2 layer")
+
+
+def test_c2_one_layer_split_attention_schedule():
+    # the opt-in split schedule (key tiles shared evenly by the SMs, items
+    # split between CTAs combined by the last part): a child process, since
+    # the switch is read once per process
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    out = subprocess.run([sys.executable, os.path.join(here, "split_attention_check.py")],
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    rel, cos, status, ws = out.stdout.split()[-4:]
+    assert int(status) == 0
+    assert int(ws) > 20 << 20  # the split's scratch is part of the workspace
+    assert float(rel) <= 2e-2 and float(cos) >= 0.9999, (rel, cos)
+
+
 # ------------------------------------------------------------------ boundary
 def test_boundary_errors_launch_nothing():
     wl = synth.get("c1")

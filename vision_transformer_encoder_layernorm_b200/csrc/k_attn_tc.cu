@@ -37,6 +37,7 @@
 // in shared memory so the neighbouring head's values there contribute 0.
 #include <cstdlib>
 #include <type_traits>
+#include <vector>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -99,7 +100,10 @@ struct __align__(8) Bars {
   uint64_t k_full[5], v_full[5], kv_empty[5], k_ready[5], v_ready[5];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t xchg[2][4];  // per (query tile, lane quarter): the 64 threads of a row pair
+  uint64_t part_done;   // split units: all softmax warps wrote their partial rows
+  uint64_t part_flag[2];  // split units: the counter was read (per tile)
   uint64_t drain[2];
+  int part_last;        // split units: this CTA combines the parts
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -112,6 +116,23 @@ struct Params {
   const int32_t *pos;
   __nv_bfloat16 *o;
   int *status;
+  float *part;           // split work: per CTA 2 slots x 2 tiles x 128 rows x kPartStride fp32
+  int *cnt;              // split work: parts finished, per item (indexed by its first CTA)
+};
+
+// Split (stream-K) schedule, head_dim 72, one sequence: CTA c processes the
+// key tiles from position (bw[c], bj[c]) up to (bw[c+1], bj[c+1]) of the
+// item list (item, key tile), in item order.  n == 0: whole items
+// round-robin instead.
+constexpr int kMaxSkCtas = 160;
+// a partial row: O columns 0..79 (72 = row sum), the running max at column
+// kPartM; the stride keeps every row 16-byte aligned for the vector stores
+constexpr int kPartStride = 84, kPartM = 80;
+static_assert((kPartStride * 4) % 16 == 0 && kPartM % 4 == 0 && 72 % 4 == 0,
+              "partial rows, the max and the row sum must sit at 16-byte boundaries");
+struct SkTable {
+  int n;
+  int bw[kMaxSkCtas + 1], bj[kMaxSkCtas + 1];
 };
 
 // One work item: query tiles [q0, q0 + 256) of head h of sequence seq.
@@ -135,6 +156,38 @@ __device__ __forceinline__ bool decode_item(int w, const Params &prm, int bk, It
   const int n_pre = prm.P > 0 ? (prm.P + bk - 1) / bk : 0;
   it.n_kv = n_pre + (it.len + bk - 1) / bk;
   return true;
+}
+
+// A work unit: key tiles [j0, j1) of item w.
+struct Unit {
+  Item it;
+  int w, j0, j1;
+  bool whole;
+};
+
+// k-th unit of this CTA: 0 = no more units, 1 = unit, 2 = nothing to do for
+// this k (an empty pair slot)
+__device__ __forceinline__ int get_unit(int k, const Params &prm, const SkTable &sk, int bk,
+                                        Unit &u) {
+  const int c = blockIdx.x;
+  if (sk.n == 0) {
+    u.w = c + k * gridDim.x;
+    if (u.w >= prm.n_pairs * prm.H * prm.n_seqs) return 0;
+    if (!decode_item(u.w, prm, bk, u.it)) return 2;
+    u.j0 = 0;
+    u.j1 = u.it.n_kv;
+    u.whole = true;
+    return 1;
+  }
+  u.w = sk.bw[c] + k;
+  const int last = sk.bj[c + 1] > 0 ? sk.bw[c + 1] : sk.bw[c + 1] - 1;
+  if (u.w > last) return 0;
+  if (!decode_item(u.w, prm, bk, u.it)) return 2;
+  u.j0 = u.w == sk.bw[c] ? sk.bj[c] : 0;
+  u.j1 = u.w == sk.bw[c + 1] ? sk.bj[c + 1] : u.it.n_kv;
+  if (u.j1 <= u.j0) return 2;
+  u.whole = u.j0 == 0 && u.j1 == u.it.n_kv;
+  return 1;
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
@@ -247,6 +300,78 @@ __device__ __forceinline__ void store_o_half(uint32_t o_addr, float l_sum, __nv_
   }
 }
 
+// Partial rows of a split item: this half's O columns (fp32, unnormalised;
+// column 72 holds the row sum) and, from half 0, the running max m.
+template <int HD, int HALF>
+__device__ __forceinline__ void store_o_part(uint32_t o_addr, float *row, float m) {
+  constexpr int NC = Cfg<HD>::HDP / 16;
+  constexpr int C0 = HALF ? (NC + 1) / 2 : 0, C1 = HALF ? NC : (NC + 1) / 2;
+  uint32_t ov[NC][16];
+  __syncwarp();
+#pragma unroll
+  for (int c = C0; c < C1; ++c) tmem_ld16(o_addr + c * 16, ov[c]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int c = C0; c < C1; ++c)
+#pragma unroll
+    for (int i = 0; i < 16; i += 4)
+      *reinterpret_cast<float4 *>(row + c * 16 + i) =
+          make_float4(__uint_as_float(ov[c][i]), __uint_as_float(ov[c][i + 1]),
+                      __uint_as_float(ov[c][i + 2]), __uint_as_float(ov[c][i + 3]));
+  if (HALF == 0) row[kPartM] = m;
+}
+
+// Combines the parts of a split item held by CTAs c0..c1 for row r:
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (l_s = O_s
+// column 72); this half's 16-byte units of the output row, bf16.
+// Partial rows of CTA cc's part of item w, query tile t (slot 0: the CTA's
+// first unit, 1: its last).
+__device__ __forceinline__ const float *part_rows(const float *part, const SkTable &sk, int cc,
+                                                 int w, int t) {
+  return part + ((size_t(cc) * 2 + (w == sk.bw[cc] ? 0 : 1)) * 2 + t) * kBlockQ * kPartStride;
+}
+
+template <int HD, int HALF>
+__device__ __noinline__ void combine_parts(const float *part, const SkTable &sk, int w, int t,
+                                           int c0, int c1, int r, __nv_bfloat16 *orow) {
+  constexpr int NU = HD / 8;
+  constexpr int U0 = HALF ? (NU + 1) / 2 : 0, U1 = HALF ? NU : (NU + 1) / 2;
+  constexpr int NV = (U1 - U0) * 2;  // float4 vectors of this half's output columns
+  // rows of the other CTAs' parts: 16-byte loads through L2 (ld.global.cg)
+  auto rowv = [&](int cc) {
+    return reinterpret_cast<const float4 *>(part_rows(part, sk, cc, w, t) + size_t(r) * kPartStride);
+  };
+  float M = -INFINITY;
+  for (int c = c0; c <= c1; ++c) M = fmaxf(M, __ldcg(rowv(c) + kPartM / 4).x);
+  float acc[NV * 4], l = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NV * 4; ++i) acc[i] = 0.0f;
+  for (int c = c0; c <= c1; ++c) {
+    const float4 *v = rowv(c);
+    float4 d[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) d[i] = __ldcg(v + U0 * 2 + i);
+    const float e = ex2_approx(__ldcg(v + kPartM / 4).x - M);
+    l += e * __ldcg(v + HD / 4).x;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      acc[4 * i] += e * d[i].x;
+      acc[4 * i + 1] += e * d[i].y;
+      acc[4 * i + 2] += e * d[i].z;
+      acc[4 * i + 3] += e * d[i].w;
+    }
+  }
+  if (orow == nullptr) return;
+  const float inv = 1.0f / l;
+#pragma unroll
+  for (int u = U0; u < U1; ++u) {
+    const float *a = acc + (u - U0) * 8;
+    *reinterpret_cast<uint4 *>(orow + u * 8) =
+        make_uint4(pack_bf16x2(a[0] * inv, a[1] * inv), pack_bf16x2(a[2] * inv, a[3] * inv),
+                   pack_bf16x2(a[4] * inv, a[5] * inv), pack_bf16x2(a[6] * inv, a[7] * inv));
+  }
+}
+
 }  // namespace attn
 
 template <int HD, bool ROPE>
@@ -257,7 +382,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_k1,
                         const __grid_constant__ CUtensorMap tm_p0,
                         const __grid_constant__ CUtensorMap tm_p1, const attn::Params prm,
-                        const __grid_constant__ RopeFreqs fr) {
+                        const __grid_constant__ RopeFreqs fr,
+                        const __grid_constant__ attn::SkTable sk) {
   using namespace attn;
   using CF = Cfg<HD>;
   constexpr int NS = CF::kStages;
@@ -273,7 +399,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
   pdl_trigger();
   pdl_wait();
-  const int n_items = prm.n_pairs * prm.H * prm.n_seqs;
   const int n_pre = prm.P > 0 ? (prm.P + BK - 1) / BK : 0;
 
   if (threadIdx.x == 0) {
@@ -287,6 +412,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       mbar_init(&bars->o_done[t], 1);
       for (int q = 0; q < 4; ++q) mbar_init(&bars->xchg[t][q], 64);
       mbar_init(&bars->drain[t], 1);
+      mbar_init(&bars->part_flag[t], 1);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -295,6 +421,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       mbar_init(&bars->k_ready[s], 32);
       mbar_init(&bars->v_ready[s], 32);
     }
+    mbar_init(&bars->part_done, 16);  // lane 0 of each softmax warp (tile 0 twice when alone)
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -333,11 +460,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       uint32_t J = 0;                 // key tiles loaded so far (ring position)
       uint32_t act[2] = {0, 0};       // items in which each query tile was active
       uint32_t issued = 0, issued_par = 0, q_issued = 0;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-        Item it;
-        if (!decode_item(w, prm, BK, it)) continue;
+      for (int k = 0; ok; ++k) {
+        Unit u;
+        const int gu = get_unit(k, prm, sk, BK, u);
+        if (gu == 0) break;
+        if (gu == 2) continue;
+        const Item &it = u.it;
         for (int t = 0; t < it.n_tiles_q; ++t) {
-          // the previous item's S MMAs of this tile have finished reading Q_t
+          // the previous unit's S MMAs of this tile have finished reading Q_t
           if (act[t] > 0 && !mbar_wait(&bars->q_empty[t], (act[t] - 1) & 1, abort_flag)) {
             ok = false;
             break;
@@ -350,7 +480,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           q_issued = (q_issued & ~(3u << (2 * t))) | ((1u | ((act[t] & 1) << 1)) << (2 * t));
           ++act[t];
         }
-        for (int j = 0; j < it.n_kv && ok; ++j, ++J) {
+        for (int j = u.j0; j < u.j1 && ok; ++j, ++J) {
           const int st = J % NS;
           const uint32_t f = (J / NS) & 1;
           if (!mbar_wait(&bars->kv_empty[st], f ^ 1, abort_flag)) { ok = false; break; }
@@ -393,13 +523,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     if (elect_one()) {
       bool ok = true, any = false;
       const uint32_t qa = smem_u32(smem + CF::kQOff + t * CF::kQTile);
-      const uint32_t sk = smem_u32(smem + CF::kKOff);
+      const uint32_t k_ring = smem_u32(smem + CF::kKOff);
       const uint32_t sv = smem_u32(smem + CF::kVOff);
       const uint32_t s_tm = tmem + CF::tmem_s(t), p_tm = tmem + CF::tmem_p(t),
                      o_tm = tmem + CF::tmem_o(t);
       // S_t = Q_t K_j^T over HDP/16 k-steps
       auto issue_s = [&](int st) {
-        const uint32_t ka = sk + st * CF::kKTile;
+        const uint32_t ka = k_ring + st * CF::kKTile;
 #pragma unroll
         for (int k = 0; k < CF::HDP / 16; ++k) {
           uint64_t ad, bd;
@@ -438,15 +568,18 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       uint32_t J = 0;     // ring position (key tiles of all items so far)
       uint32_t tc = 0;    // key tiles processed by this query tile so far
       uint32_t act = 0;   // items in which this query tile was active
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-        Item it;
-        if (!decode_item(w, prm, BK, it)) continue;
+      for (int k = 0; ok; ++k) {
+        Unit u;
+        const int gu = get_unit(k, prm, sk, BK, u);
+        if (gu == 0) break;
+        if (gu == 2) continue;
+        const Item &it = u.it;
+        const int n_kv = u.j1 - u.j0;  // key tiles of this unit
         if (t >= it.n_tiles_q) {  // tile 0's issuer commits this tile's share of kv_empty
-          J += it.n_kv;
+          J += n_kv;
           continue;
         }
         const bool alone = it.n_tiles_q == 1;
-        const int n_kv = it.n_kv;
         // Q_t loaded and prepared; S_t of the previous item loaded by the softmax
         if (!mbar_wait(kPrep ? &bars->q_ready[t] : &bars->q_full[t], act & 1, abort_flag) ||
             (tc > 0 && !mbar_wait(&bars->s_free[t], (tc - 1) & 1, abort_flag)) || !wait_k(J)) {
@@ -472,7 +605,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           if (!mbar_wait(HD == 72 ? &bars->v_ready[st] : &bars->v_full[st], (Jj / NS) & 1, abort_flag) ||
               !mbar_wait(&bars->p_full[t], tj & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(st, j > 0);
+          issue_pv(st, j > 0);  // j counts this unit's tiles
           mma_commit(&bars->o_done[t]);
           mma_commit(&bars->kv_empty[st]);  // this tile is done with K_j and V_j
           if (alone) mma_commit(&bars->kv_empty[st]);
@@ -492,9 +625,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     uint32_t J = 0;
     uint32_t act[2] = {0, 0};
     bool ok = true;
-    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-      Item it;
-      if (!decode_item(w, prm, BK, it)) continue;
+    for (int k = 0; ok; ++k) {
+      Unit u;
+      const int gu = get_unit(k, prm, sk, BK, u);
+      if (gu == 0) break;
+      if (gu == 2) continue;
+      const Item &it = u.it;
       for (int t = 0; t < it.n_tiles_q; ++t) {
         if (!mbar_wait(&bars->q_full[t], act[t] & 1, abort_flag)) { ok = false; break; }
         uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
@@ -512,7 +648,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         mbar_arrive(&bars->q_ready[t]);
         ++act[t];
       }
-      for (int j = 0; j < it.n_kv && ok; ++j, ++J) {
+      for (int j = u.j0; j < u.j1 && ok; ++j, ++J) {
         const int st = J % NS;
         const uint32_t f = (J / NS) & 1;
         if (ROPE) {
@@ -575,12 +711,17 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     bool ok = true;
     uint32_t tc = 0;    // key tiles processed by this query tile so far
     uint32_t xc = 0;    // row-pair exchanges so far
-    uint32_t act = 0;   // items in which this query tile was active
-    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-      Item it;
-      if (!decode_item(w, prm, BK, it)) continue;
+    uint32_t act = 0;   // units in which this query tile was active
+    uint32_t pc = 0;    // split units in which this query tile was active
+    uint32_t pd = 0;    // split units (tile 0: phases of part_done)
+    for (int k = 0; ok; ++k) {
+      Unit u;
+      const int gu = get_unit(k, prm, sk, BK, u);
+      if (gu == 0) break;
+      if (gu == 2) continue;
+      const Item &it = u.it;
       if (t >= it.n_tiles_q) continue;
-      const int n_kv = it.n_kv, len = it.len;
+      const int n_kv = u.j1 - u.j0, len = it.len;  // n_kv: this unit's key tiles
       const int qrow = it.q0 + t * kBlockQ + r;  // row inside the sequence
       float m = -INFINITY;
       uint64_t l2[2] = {0, 0};  // packed partial row sums (head_dim 128)
@@ -588,7 +729,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const uint32_t tj = tc + j, xj_ph = xc + j;
         if (!warp_wait(&bars->s_full[t], tj & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const int nvalid = (j < n_pre ? min(BK, prm.P - j * BK) : min(BK, len - (j - n_pre) * BK)) -
+        const int ja = u.j0 + j;  // key tile of the item
+        const int nvalid = (ja < n_pre ? min(BK, prm.P - ja * BK) : min(BK, len - (ja - n_pre) * BK)) -
                            half * HC;  // valid keys among this thread's columns
         uint32_t s[HC];
         __syncwarp();
@@ -718,6 +860,59 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
       __nv_bfloat16 *orow =
           qrow < len ? prm.o + size_t(it.seg0 + qrow) * prm.C + size_t(it.h) * HD : nullptr;
+      if constexpr (HD == 72) {
+        if (!u.whole) {
+          // part of a split item: unnormalised O (column 72 = row sum) and the
+          // running max go to this CTA's slot; the last part to finish
+          // combines all parts of the item
+          const int c = blockIdx.x;
+          float *mine = const_cast<float *>(part_rows(prm.part, sk, c, u.w, t)) + size_t(r) * kPartStride;
+          if (half == 0)
+            store_o_part<HD, 0>(o_addr, mine, m);
+          else
+            store_o_part<HD, 1>(o_addr, mine, m);
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cnt(&bars->part_done, it.n_tiles_q == 1 ? 2u : 1u);
+          // first and last CTA holding a part of this item
+          int c0 = c, c1 = c;
+          while (c0 > 0 && !(sk.bw[c0] < u.w || (sk.bw[c0] == u.w && sk.bj[c0] == 0))) --c0;
+          while (c1 + 1 < sk.n && (sk.bw[c1 + 1] < u.w || (sk.bw[c1 + 1] == u.w && sk.bj[c1 + 1] < it.n_kv)))
+            ++c1;
+          if (warp == 4 && lane == 0) {
+            bool okp = mbar_wait(&bars->part_done, pd & 1, abort_flag);
+            int last = 0;
+            if (okp) {
+              // part_done ordered every thread's partial rows before this
+              // point; the GPU-scope fence releases them (cumulatively)
+              // before the count
+              __threadfence();
+              const int old = atomicAdd(prm.cnt + c0, 1);
+              last = old == c1 - c0;
+              if (last) {
+                prm.cnt[c0] = 0;  // every part has arrived: ready for the next launch
+                __threadfence();  // order the other parts' rows before the reads below
+              }
+            }
+            bars->part_last = last;
+            for (int tt = 0; tt < it.n_tiles_q; ++tt) mbar_arrive(&bars->part_flag[tt]);
+          }
+          ++pd;
+          if (!warp_wait(&bars->part_flag[t], pc & 1, abort_flag)) { ok = false; break; }
+          ++pc;
+          if (*reinterpret_cast<volatile int *>(&bars->part_last)) {
+            // the counting thread's fence acquired the other parts' rows and
+            // part_flag passed that on; they are read through L2
+            if (half == 0)
+              combine_parts<HD, 0>(prm.part, sk, u.w, t, c0, c1, r, orow);
+            else
+              combine_parts<HD, 1>(prm.part, sk, u.w, t, c0, c1, r, orow);
+          }
+          tc += n_kv;
+          xc += n_kv;
+          ++act;
+          continue;
+        }
+      }
       if (half == 0)
         store_o_half<HD, 0>(o_addr, l, orow);
       else
@@ -740,19 +935,90 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 // ---------------------------------------------------------------- host side
 template <int HD, bool ROPE>
 static cudaError_t launch_hd(const CUtensorMap *maps, const attn::Params &prm, int grid,
-                             const RopeFreqs &fr, cudaStream_t st) {
+                             const RopeFreqs &fr, const attn::SkTable &sk, cudaStream_t st) {
   using CF = attn::Cfg<HD>;
   auto kern = attention_tc_kernel<HD, ROPE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmem));
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(attn::kThreads), CF::kSmem, st, 1, maps[0], maps[1],
-                    maps[2], maps[3], maps[4], maps[5], prm, fr);
+                    maps[2], maps[3], maps[4], maps[5], prm, fr, sk);
+}
+
+int attn_split_max_ctas() { return attn::kMaxSkCtas; }
+
+// The split schedule is opt-in (VIT_ATTN_SPLIT=1): it balances the SMs, but
+// the partial rows' round trip and the combine cost more than the balance
+// gains at the c2 size (measured 139 against 126 us per launch).
+bool attn_split_enabled() {
+  static const bool on = [] {
+    const char *e = getenv("VIT_ATTN_SPLIT");
+    return e != nullptr && atoi(e) != 0;
+  }();
+  return on;
+}
+
+// Whether one sequence of T tokens (no prefix) takes the split schedule at
+// head_dim 72 on `grid` CTAs: the same size rules as build_split_table.
+bool attn_split_possible(int T, int H, int grid) {
+  constexpr int BK = attn::Cfg<72>::BK;
+  const long long n_kv = (T + BK - 1) / BK;
+  const long long n_pairs = (T + 2 * attn::kBlockQ - 1) / (2 * attn::kBlockQ);
+  if (grid <= 0 || grid > attn::kMaxSkCtas || n_kv < 8) return false;
+  return n_pairs * H * 4 * n_kv / grid >= 8 * 3;  // upper bound of the real weight
+}
+size_t attn_split_part_bytes() { return size_t(2) * 2 * attn::kBlockQ * attn::kPartStride * 4; }
+
+// Split schedule for one sequence at head_dim 72 (see SkTable): equal shares
+// of the key-tile work (a tile of a two-query-tile item weighs 4, of a
+// one-tile item 3, their measured cost ratio), boundaries snapped to item
+// edges when within 3 tiles of one.  false: use whole items.
+static bool build_split_table(const SeqArgs &s, int H, int n_pairs, int grid, attn::SkTable &sk) {
+  constexpr int BK = attn::Cfg<72>::BK;
+  const int len = s.total_tokens, P = s.prefix_kv ? s.prefix_len : 0;
+  const int n_pre = P > 0 ? (P + BK - 1) / BK : 0;
+  const int n_kv = n_pre + (len + BK - 1) / BK;
+  const int N = n_pairs * H;
+  if (grid > attn::kMaxSkCtas || n_kv < 8) return false;
+  std::vector<long long> cum(N + 1, 0);
+  for (int w = 0; w < N; ++w) {
+    const int q0 = (w / H) * 2 * attn::kBlockQ;
+    const int tw = len - q0 > attn::kBlockQ ? 4 : 3;
+    cum[w + 1] = cum[w] + (long long)tw * n_kv;
+  }
+  const long long W = cum[N];
+  if (W / grid < 8 * 3) return false;  // shares of at least ~8 key tiles
+  sk.n = grid;
+  int w = 0;
+  for (int c = 0; c <= grid; ++c) {
+    const long long B = (long long)c * W / grid;
+    while (w < N && cum[w + 1] <= B) ++w;
+    int bw = w, bj = 0;
+    if (w < N && c < grid) {
+      const long long tw = (cum[w + 1] - cum[w]) / n_kv;
+      bj = int((B - cum[w] + tw - 1) / tw);
+      if (bj < 3) bj = 0;
+      if (bj > n_kv - 3) bj = n_kv;
+      if (bj >= n_kv) {
+        bw = w + 1;
+        bj = 0;
+      }
+    } else {
+      bw = N;
+      bj = 0;
+    }
+    sk.bw[c] = bw;
+    sk.bj[c] = bj;
+  }
+  for (int c = 0; c < grid; ++c)  // every share non-empty
+    if (!(sk.bw[c] < sk.bw[c + 1] || (sk.bw[c] == sk.bw[c + 1] && sk.bj[c] < sk.bj[c + 1])))
+      return false;
+  return true;
 }
 
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,
                                 float scale, const RopeFreqs &fr, int num_sms, int *status,
-                                cudaStream_t st) {
+                                float *part, int *cnt, cudaStream_t st) {
   if (s.total_tokens == 0 || s.max_seqlen == 0) return cudaSuccess;
   const int C = H * d;
   const int Hkv = s.kv_heads > 0 ? s.kv_heads : H;
@@ -799,6 +1065,8 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
   prm.pos = s.pos;
   prm.o = static_cast<__nv_bfloat16 *>(o);
   prm.status = status;
+  prm.part = part;
+  prm.cnt = cnt;
   const int n_items = prm.n_pairs * H * s.n_seqs;
   // persistent (one CTA per SM walking the items) or one CTA per item
   static const int grid_mode = [] {
@@ -806,13 +1074,19 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
     return e ? atoi(e) : 0;
   }();
   const bool persistent = grid_mode == 1 || (grid_mode == 0 && d == 72);
-  const int grid = (persistent && n_items > num_sms) ? num_sms : n_items;
+  int grid = (persistent && n_items > num_sms) ? num_sms : n_items;
+  attn::SkTable sk;
+  sk.n = 0;
+  if (d == 72 && s.n_seqs == 1 && part && cnt && persistent && attn_split_enabled() &&
+      !build_split_table(s, H, prm.n_pairs, std::min(num_sms, attn::kMaxSkCtas), sk))
+    sk.n = 0;
+  if (sk.n) grid = sk.n;
   const bool rope = s.pos != nullptr;
   if (d == 72)
-    return rope ? launch_hd<72, true>(maps, prm, grid, fr, st)
-                : launch_hd<72, false>(maps, prm, grid, fr, st);
-  return rope ? launch_hd<128, true>(maps, prm, grid, fr, st)
-              : launch_hd<128, false>(maps, prm, grid, fr, st);
+    return rope ? launch_hd<72, true>(maps, prm, grid, fr, sk, st)
+                : launch_hd<72, false>(maps, prm, grid, fr, sk, st);
+  return rope ? launch_hd<128, true>(maps, prm, grid, fr, sk, st)
+              : launch_hd<128, false>(maps, prm, grid, fr, sk, st);
 }
 
 }  // namespace vit

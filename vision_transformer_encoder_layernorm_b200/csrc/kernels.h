@@ -95,8 +95,15 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
                            cudaStream_t st, const RopeEpi *rope = nullptr);
 
 // tcgen05 flash attention, bf16, head_dim 72 or 128.
+// Split (stream-K) attention schedule: most CTAs it uses, and the bytes of
+// partial rows each of them needs in the workspace.
+int attn_split_max_ctas();
+bool attn_split_possible(int T, int H, int grid);
+bool attn_split_enabled();
+size_t attn_split_part_bytes();
 cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int H, int d,
                                 float scale, const RopeFreqs &fr, int num_sms, int *status,
+                                float *part, int *cnt,
                                 cudaStream_t st);
 
 // Launches `kern` with programmatic dependent launch allowed (and a cluster

@@ -155,35 +155,46 @@ cudaError_t run_linear(vit_ctx *ctx, int kind, const void *x, const void *w, con
 }
 
 cudaError_t run_attention(vit_ctx *ctx, const void *qkv, void *o, const SeqArgs &s, float scale,
-                          cudaStream_t st) {
+                          cudaStream_t st, float *part = nullptr, int *cnt = nullptr) {
   const vit_config &c = ctx->cfg;
   return counted(ctx, VIT_K_ATTENTION, st, [&] {
     if (c.dtype == VIT_F32)
       return launch_attention_simt(kF32, qkv, o, s, c.heads, c.head_dim, scale, ctx->fr,
                                    ctx->d_status, st);
     return launch_attention_tc(qkv, o, s, c.heads, c.head_dim, scale, ctx->fr, ctx->num_sms,
-                               ctx->d_status, st);
+                               ctx->d_status, part, cnt, st);
   });
 }
 
 struct Workspace {
   void *h, *qkv, *attn, *x1, *g, *act[2];
+  void *part, *cnt;  // split attention: partial rows and per-item counters (or null)
 };
 
-size_t workspace_layout(const vit_config &c, int T, Workspace *w, void *base) {
+// CTAs of the split attention schedule whose scratch the workspace holds
+// for T tokens (bf16 at head_dim 72, large enough to split; 0 = none)
+int split_ctas(const vit_ctx *ctx, int T) {
+  if (ctx->cfg.dtype != VIT_BF16 || ctx->cfg.head_dim != 72 || !attn_split_enabled()) return 0;
+  const int g = std::min(ctx->num_sms, attn_split_max_ctas());
+  return attn_split_possible(T, ctx->cfg.heads, g) ? g : 0;
+}
+
+size_t workspace_layout(const vit_config &c, int T, Workspace *w, void *base, int sk_ctas) {
   const size_t es = esize(c);
   const size_t C = size_t(c.hidden);
   const size_t F = (c.flags & VIT_FLAG_NO_MLP) ? 0 : size_t(c.mlp);
-  const size_t sizes[7] = {T * C * es, T * 3 * C * es, T * C * es, T * C * es,
-                           T * F * es, T * C * es, T * C * es};
+  const size_t sizes[9] = {T * C * es, T * 3 * C * es, T * C * es, T * C * es,
+                           T * F * es, T * C * es, T * C * es,
+                           size_t(sk_ctas) * attn_split_part_bytes(), size_t(sk_ctas) * 4};
   size_t off = 0;
-  void **slots[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  void **slots[9] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   if (w) {
     slots[0] = &w->h; slots[1] = &w->qkv; slots[2] = &w->attn; slots[3] = &w->x1;
     slots[4] = &w->g; slots[5] = &w->act[0]; slots[6] = &w->act[1];
+    slots[7] = &w->part; slots[8] = &w->cnt;
   }
-  for (int i = 0; i < 7; ++i) {
-    if (w) *slots[i] = static_cast<char *>(base) + off;
+  for (int i = 0; i < 9; ++i) {
+    if (w) *slots[i] = sizes[i] ? static_cast<char *>(base) + off : nullptr;
     off += align256(sizes[i]);
   }
   return off;
@@ -234,7 +245,9 @@ vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, v
       }))
     return VIT_ERR_CUDA;
   const SeqArgs sa = to_seq_args(seqs, false);
-  if (run_attention(ctx, ws.qkv, ws.attn, sa, scale, st)) return VIT_ERR_CUDA;
+  if (run_attention(ctx, ws.qkv, ws.attn, sa, scale, st, static_cast<float *>(ws.part),
+                    static_cast<int *>(ws.cnt)))
+    return VIT_ERR_CUDA;
   if (c.flags & VIT_FLAG_NO_MLP) {
     if (run_linear(ctx, VIT_K_GEMM_OUT, ws.attn, w->w_o, w->b_o, x, y, T, C, C, kEpiResidual, st))
       return VIT_ERR_CUDA;
@@ -263,7 +276,7 @@ vit_status check_layer_call(vit_ctx *ctx, const void *x, void *y, const vit_seqs
   if (ctx->cfg.dtype == VIT_BF16 && (!aligned16(x) || !aligned16(y))) return VIT_ERR_INVALID_ARG;
   if (seqs->total_tokens > 0 && !(ctx->cfg.flags & VIT_FLAG_NO_ROPE) && !seqs->pos_rc)
     return VIT_ERR_INVALID_ARG;
-  const size_t need = workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr);
+  const size_t need = workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr, split_ctas(ctx, seqs->total_tokens));
   if (!workspace || ws_bytes < need) return VIT_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return VIT_ERR_WORKSPACE;
   return VIT_OK;
@@ -462,7 +475,7 @@ void vit_destroy(vit_ctx *ctx) {
 
 size_t vit_workspace_bytes(const vit_ctx *ctx, int total_tokens) {
   if (!ctx || total_tokens < 0) return 0;
-  return workspace_layout(ctx->cfg, total_tokens, nullptr, nullptr);
+  return workspace_layout(ctx->cfg, total_tokens, nullptr, nullptr, split_ctas(ctx, total_tokens));
 }
 
 vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const void *x, void *y,
@@ -474,8 +487,12 @@ vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const voi
   if (seqs->total_tokens == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
   Workspace ws;
-  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, workspace);
-  return layer_impl(ctx, w, x, y, seqs, ws, static_cast<cudaStream_t>(stream));
+  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, workspace, split_ctas(ctx, seqs->total_tokens));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the split attention's counters start at zero; each launch leaves them so
+  if (ws.cnt && cudaMemsetAsync(ws.cnt, 0, size_t(split_ctas(ctx, seqs->total_tokens)) * 4, st) != cudaSuccess)
+    return VIT_ERR_CUDA;
+  return layer_impl(ctx, w, x, y, seqs, ws, st);
 }
 
 vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, int n_layers,
@@ -489,8 +506,11 @@ vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, in
   if (seqs->total_tokens == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
   Workspace ws;
-  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, workspace);
+  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, workspace, split_ctas(ctx, seqs->total_tokens));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the split attention's counters start at zero; each launch leaves them so
+  if (ws.cnt && cudaMemsetAsync(ws.cnt, 0, size_t(split_ctas(ctx, seqs->total_tokens)) * 4, st) != cudaSuccess)
+    return VIT_ERR_CUDA;
   for (int i = 0; i < n_layers; ++i) {
     const void *in = i == 0 ? x : ws.act[(i - 1) & 1];
     void *out = i == n_layers - 1 ? y : ws.act[i & 1];
@@ -791,7 +811,7 @@ extern "C" vit_status vit_layer_forward_noalloc(vit_ctx *ctx, const vit_layer_we
   if (!ctx || !seqs) return VIT_ERR_INVALID_ARG;
   if (seqs->total_tokens < 0) return VIT_ERR_INVALID_ARG;
   // size check first, against the fixed scratch, before any device work
-  if (workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr) > kStaticScratchBytes)
+  if (workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr, 0) > kStaticScratchBytes)
     return VIT_ERR_WORKSPACE;
   DeviceGuard g(ctx->device);
   void *scratch = nullptr;
@@ -801,7 +821,7 @@ extern "C" vit_status vit_layer_forward_noalloc(vit_ctx *ctx, const vit_layer_we
   if ((s = check_layer_weights(ctx->cfg, w)) != VIT_OK) return s;
   if (seqs->total_tokens == 0) return VIT_OK;
   Workspace ws;
-  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, scratch);
+  workspace_layout(ctx->cfg, seqs->total_tokens, &ws, scratch, 0);
   // launch counts only: no timing events are created during this call
   const bool prof_on = ctx->prof.on;
   ctx->prof.on = false;
