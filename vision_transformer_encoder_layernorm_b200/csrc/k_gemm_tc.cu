@@ -127,20 +127,26 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, in
 // epilogue warp e (= warp - 2) drains TMEM lane quarter (warp & 3), i.e. one
 // row per thread, and column half (e >> 2) of the tile.  The warp's half of
 // the tile bias was staged in its shared-memory slot (bias_w).
-template <int BN, int EPI>
+template <int BN, int EPI, int TS = BN>
 __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int lane, int row,
                                               bool row_ok, int n0, int N, const RopeEpi &re,
                                               const __nv_bfloat16 *bias_w,
+                                              const __nv_bfloat16 *__restrict__ bias,
                                               const __nv_bfloat16 *__restrict__ res,
                                               __nv_bfloat16 *__restrict__ y) {
   constexpr int kChunks = BN / 64;  // 32-column chunks per half
   const int quarter = warp & 3, half = (warp - 2) >> 2;
   if constexpr (EPI == kEpiRope) {
-    // one whole head (BN/2 columns) per warp: bias, then the 2D rotation of
-    // Q/K pairs (j, j + HD/4) in each half of the head, in fp32
-    constexpr int HD = BN / 2, Q4 = HD / 4, NF = HD / 32;
-    const int col0 = n0 + half * HD;
-    const uint32_t base = tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(half * HD);
+    // whole heads: the tile holds HPT heads of HD columns (TS = HPT * HD;
+    // the MMA width BN may round TS up); warp `half` of a lane quarter takes
+    // heads half, half + 2, ...: bias, then the 2D rotation of Q/K pairs
+    // (j, j + HD/4) in each half of the head, in fp32
+    constexpr int HPT = TS == 216 ? 3 : 2, HD = TS / HPT, Q4 = HD / 4, NF = HD / 32;
+    static_assert(HPT * HD == TS && TS <= BN, "RoPE tile of whole heads");
+#pragma unroll 1
+    for (int hh = half; hh < HPT; hh += 2) {
+    const int col0 = n0 + hh * HD;
+    const uint32_t base = tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(hh * HD);
     uint32_t r[NF][32];
     uint32_t r8[8];
     __syncwarp();
@@ -148,19 +154,25 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
     for (int c = 0; c < NF; ++c) tmem_ld32(base + c * 32, r[c]);
     if (HD % 32) tmem_ld8(base + NF * 32, r8);
     tmem_ld_wait();
-    if (!(row_ok && col0 < N)) return;
+    if (!(row_ok && col0 < N)) continue;
     float v[HD];
 #pragma unroll
     for (int i = 0; i < HD; ++i) {
       const uint32_t bits = i < NF * 32 ? r[i / 32][i % 32] : r8[i - NF * 32];
       v[i] = __uint_as_float(bits);
     }
-    const uint32_t *bw = reinterpret_cast<const uint32_t *>(bias_w);
+    if (bias != nullptr) {  // the head's bias (the same for the whole warp: broadcast loads)
+      const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
 #pragma unroll
-    for (int i = 0; i < HD / 2; ++i) {
-      const uint32_t b2 = bw[i];
-      v[2 * i] += bf16_lo(b2);
-      v[2 * i + 1] += bf16_hi(b2);
+      for (int u = 0; u < HD / 8; ++u) {
+        const uint4 b4 = __ldg(bp + u);
+        const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * u + 2 * e] += bf16_lo(bb[e]);
+          v[8 * u + 2 * e + 1] += bf16_hi(bb[e]);
+        }
+      }
     }
     if (col0 < re.rot_cols) {
       const int2 pr = reinterpret_cast<const int2 *>(re.pos)[row];
@@ -186,6 +198,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
       o.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
       o.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
       yp[u] = o;
+    }
     }
   } else {
 #pragma unroll 1
@@ -352,7 +365,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       tc_fence_after();
       const int row = mb * BM + row_in_tile;
       epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, re,
-                             bias_w, res, y);
+                             bias_w, bias, res, y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
@@ -394,7 +407,7 @@ struct Cfg2 {
 };
 }  // namespace gemm
 
-template <int BN, int EPI>
+template <int BN, int EPI, int TS = BN>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
@@ -412,7 +425,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const uint32_t rank = cluster_cta_rank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-  const int num_m = (M + 2 * BM - 1) / (2 * BM), num_n = (N + BN - 1) / BN;
+  // tiles step TS columns (TS <= BN, the MMA width: a RoPE tile of three
+  // 72-wide heads computes 224 columns and keeps 216)
+  const int num_m = (M + 2 * BM - 1) / (2 * BM), num_n = (N + TS - 1) / TS;
   const int num_tiles = num_m * num_n;
   const int k_blocks = (K + BK - 1) / BK;
 
@@ -460,7 +475,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const uint32_t full_leader = map_to_cta(&bars->full[stage], 0);
           tma_load_2d_pair(sa, &tmA, full_leader, kb * BK, mb * 2 * BM + int(rank) * BM);
           tma_load_2d_pair(sa + kATileBytes, &tmB, full_leader, kb * BK,
-                           nb * BN + int(rank) * (BN / 2));
+                           nb * TS + int(rank) * (BN / 2));
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == CF::kStages) { stage = 0; phase ^= 1; }
@@ -523,12 +538,12 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      stage_bias_warp<BN>(bias_w, bias, nb * BN, N, warp, lane);
+      if (EPI != kEpiRope) stage_bias_warp<BN>(bias_w, bias, nb * TS, N, warp, lane);
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * 2 * BM + row_in_tile;
-      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, re,
-                             bias_w, res, y);
+      epilogue_tile<BN, EPI, TS>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * TS, N, re,
+                                 bias_w, bias, res, y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_cta(&bars->acc_empty[a], 0));
@@ -598,12 +613,12 @@ static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap 
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int TS = BN>
 static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
                                const void *res, void *y, int M, int N, int K, int num_sms,
                                int *status, cudaStream_t st, const RopeEpi &re) {
   using CF = gemm::Cfg2<BN>;
-  auto kern = gemm_tc2_kernel<BN, EPI>;
+  auto kern = gemm_tc2_kernel<BN, EPI, TS>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmemBytes));
   if (e != cudaSuccess) return e;
@@ -629,7 +644,7 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
     }
     max_clusters = n;
   }
-  const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + BN - 1) / BN);
+  const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + TS - 1) / TS);
   return launch_pdl(kern, dim3(2 * std::max(1, std::min(tiles, max_clusters))),
                     dim3(gemm::kThreads), CF::kSmemBytes, st, 2, ta, tb,
                     static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
@@ -692,9 +707,9 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
                            cudaStream_t st, const RopeEpi *rope) {
   if (M == 0 || N == 0) return cudaSuccess;
   GemmVariant v = choose_variant(M, N, K, num_sms);
-  if (epi == kEpiRope) {  // tiles of two whole heads on a CTA pair
+  if (epi == kEpiRope) {  // tiles of whole heads on a CTA pair: 3 x 72 (MMA N = 224) or 2 x 128
     if (rope == nullptr || (rope->head_dim != 72 && rope->head_dim != 128)) return cudaErrorInvalidValue;
-    v = {2, 2 * rope->head_dim};
+    v = {2, rope->head_dim == 72 ? 224 : 256};
   }
   const int b_rows = v.pair == 2 ? v.bn / 2 : v.bn;
   CUtensorMap ta, tb;
@@ -705,9 +720,9 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
                            gemm::BK, b_rows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (epi == kEpiRope) {
-    if (v.bn == 144)
-      return launch_pair<144, kEpiRope>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
-    return launch_pair<256, kEpiRope>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
+    if (v.bn == 224)
+      return launch_pair<224, kEpiRope, 216>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
+    return launch_pair<256, kEpiRope, 256>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
   }
   if (v.pair == 2) {
     if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
