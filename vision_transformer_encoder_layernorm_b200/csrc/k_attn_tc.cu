@@ -300,6 +300,35 @@ __device__ __forceinline__ void store_o_half(uint32_t o_addr, float l_sum, __nv_
   }
 }
 
+// Maximum of the first `nvalid` of N consecutive TMEM columns of this
+// thread's lane (N % 8 == 0), read in pieces of at most 32 columns.
+template <int N>
+__device__ __forceinline__ float tmem_rowmax(uint32_t addr, int nvalid) {
+  float mx = -INFINITY;
+  int base = 0;
+  auto piece = [&](auto wc) {
+    constexpr int W = decltype(wc)::value;
+    uint32_t q[W];
+    __syncwarp();
+    tmem_ld_cols<W>(addr + base, q);
+    tmem_ld_wait();
+    if (nvalid - base < W) {
+#pragma unroll
+      for (int i = 0; i < W; ++i)
+        if (base + i >= nvalid) q[i] = 0xFF800000u;
+    }
+#pragma unroll
+    for (int i = 0; i + 1 < W; i += 2)
+      mx = fmax3(mx, __uint_as_float(q[i]), __uint_as_float(q[i + 1]));
+    base += W;
+  };
+  if constexpr (N >= 32) piece(std::integral_constant<int, 32>{});
+  if constexpr (N % 32 >= 16) piece(std::integral_constant<int, 16>{});
+  if constexpr (N % 16 >= 8) piece(std::integral_constant<int, 8>{});
+  static_assert(N <= 56 && N % 8 == 0, "row pieces");
+  return mx;
+}
+
 // Partial rows of a split item: this half's O columns (fp32, unnormalised;
 // column 72 holds the row sum) and, from half 0, the running max m.
 template <int HD, int HALF>
@@ -689,6 +718,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const int r = quarter * 32 + lane;   // query row inside the tile
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + CF::tmem_s(t) + half * HC;
+    const uint32_t s_other = tmem + lane_base + CF::tmem_s(t) + (half ^ 1) * HC;
     const uint32_t p_addr = tmem + lane_base + CF::tmem_p(t) + half * (HC / 2);
     const uint32_t o_addr = tmem + lane_base + CF::tmem_o(t);
     float *xv = reinterpret_cast<float *>(smem + CF::kXOff) + t * 256;  // [phase&1][t][half][row]
@@ -726,12 +756,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       float m = -INFINITY;
       uint64_t l2[2] = {0, 0};  // packed partial row sums (head_dim 128)
       for (int j = 0; j < n_kv; ++j) {
-        const uint32_t tj = tc + j, xj_ph = xc + j;
+        const uint32_t tj = tc + j;
         if (!warp_wait(&bars->s_full[t], tj & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int ja = u.j0 + j;  // key tile of the item
-        const int nvalid = (ja < n_pre ? min(BK, prm.P - ja * BK) : min(BK, len - (ja - n_pre) * BK)) -
-                           half * HC;  // valid keys among this thread's columns
+        const int nv_tile = ja < n_pre ? min(BK, prm.P - ja * BK) : min(BK, len - (ja - n_pre) * BK);
+        const int nvalid = nv_tile - half * HC;  // valid keys among this thread's columns
+        // the row max needs the other half's scores too: read them from TMEM
+        // in pieces and keep only their maximum (cheaper than a hand-off
+        // between the two threads of the row)
+        const float m_other = tmem_rowmax<HC>(s_other, nv_tile - (half ^ 1) * HC);
         uint32_t s[HC];
         __syncwarp();
         tmem_ld_cols<HC>(s_addr, s);
@@ -751,13 +785,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
         if constexpr ((HC - 2) % 4 != 0)
           a0 = fmax3(a0, __uint_as_float(s[HC - 2]), __uint_as_float(s[HC - 1]));
-        // swap partial maxima with the thread that holds the row's other half
-        float *xj = xv + (xj_ph & 1) * 512;
-        const float m_loc = fmaxf(a0, a1) * sl2;
-        xj[half * 128 + r] = m_loc;
-        mbar_arrive(xb);
-        if (!warp_wait(xb, xj_ph & 1, abort_flag)) { ok = false; break; }
-        const float m_tile = fmaxf(xj[r], xj[128 + r]);
+        const float m_tile = fmax3(a0, a1, m_other) * sl2;
         // The row max only matters when it grows by more than 8 (log2 units)
         // over the running max m: then O (and the row sum) is rescaled.
         // Otherwise m stays (stale) and the final O / l division absorbs it
@@ -852,10 +880,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         float a, b, c2, d2;
         f2_unpack(l2[0], a, b);
         f2_unpack(l2[1], c2, d2);
-        float *xj = xv + ((xc + n_kv) & 1) * 512;
+        float *xj = xv + (xc & 1) * 512;
         xj[half * 128 + r] = (a + b) + (c2 + d2);
         mbar_arrive(xb);
-        if (!warp_wait(xb, (xc + n_kv) & 1, abort_flag)) { ok = false; break; }
+        if (!warp_wait(xb, xc & 1, abort_flag)) { ok = false; break; }
         l = xj[r] + xj[128 + r];
       }
       __nv_bfloat16 *orow =
@@ -908,7 +936,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
               combine_parts<HD, 1>(prm.part, sk, u.w, t, c0, c1, r, orow);
           }
           tc += n_kv;
-          xc += n_kv;
           ++act;
           continue;
         }
@@ -918,7 +945,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       else
         store_o_half<HD, 1>(o_addr, l, orow);
       tc += n_kv;
-      xc += n_kv + (kSumByMma ? 0 : 1);
+      xc += kSumByMma ? 0 : 1;  // the head_dim 128 epilogue swaps the halves' row sums
       ++act;
     }
   }
