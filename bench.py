@@ -447,6 +447,53 @@ def main():
                            "L2 flushed before every step (inside the region)",
                "serial": {"value": world * T / (s_ms / 1e3), "ms_per_step": s_ms,
                           "schedule": "upload, step, download in line on one stream"}}
+    # ---- the 27-layer stack without the merge, on the workload's other grid
+    # (the same 3900 patches as a 60 x 65 image): same inputs and weights,
+    # positions and segment table rebuilt for that grid, L2 flushed before
+    # every step
+    enc_only = None
+    if not args.layers:
+        g2 = [(60, 65)]
+        cu2 = torch.empty(2, dtype=torch.int32, device="cuda")
+        pos2 = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+        ctx.positions_from_grids(g2, cu2, pos2)
+        sq2 = vit.seqs(T, 1, T, cu2, pos2)
+        y2 = torch.empty_like(x)
+
+        def enc_step(st=stream):
+            ctx.encoder_forward(lw_structs, x, y2, sq2, ws, st)
+
+        g_enc = None
+        if graph is not None:
+            cs = ctx.graph_begin()
+            enc_step(cs)
+            g_enc = ctx.graph_end()
+
+        def enc_launch():
+            if g_enc is not None:
+                g_enc.launch(stream)
+            else:
+                enc_step()
+
+        for _ in range(args.warmup):
+            enc_launch()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.zero_()
+            ev2[k][0].record(stream)
+            enc_launch()
+            ev2[k][1].record(stream)
+        torch.cuda.synchronize()
+        if g_enc is not None:
+            g_enc.close()
+        enc_ms = replicas.max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev2])),
+                                         device="cuda")
+        enc_only = {"value": world * T / (enc_ms / 1e3), "unit": UNIT, "ms_per_step": enc_ms,
+                    "grid": "60x65", "merge": False,
+                    "tflops": flops["total"] / (enc_ms / 1e3) / 1e12}
     # ---- beyond the encoder: patch embedding of the same image (50 x 78
     # patches of 14 x 14 pixels, 27 x 27 position table), timed on its own
     nxt = None
@@ -504,6 +551,7 @@ def main():
                if args.layers else {}),
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+            **({"encoder_only": enc_only} if enc_only else {}),
             **({"next": nxt} if nxt else {}),
         }
         print(json.dumps(line), flush=True)

@@ -126,13 +126,15 @@ def test_c2_full_stack_and_merge():
     assert_close(got, ref, 1.0, 0.999, "c2 27-layer stack + merge")
 
 
-def test_c2_one_layer():
-    # one 3900-token layer (the headline's size) against the oracle
-    wl = synth.get("c2").with_(layers=1)
+@pytest.mark.parametrize("grid", [(50, 78), (60, 65)])
+def test_c2_one_layer(grid):
+    # one 3900-token layer (the headline's size) against the oracle, on both
+    # grids of the workload (the merged image and the encoder-only one)
+    wl = synth.get("c2").with_(layers=1, grids=[grid])
     inp = synth.make_inputs(wl, layers=1)
     got = _device_run(wl, inp, merge=False)
     ref = orun.run_layers(inp)
-    assert_close(got, ref, 2e-2, 0.9999, "c2 layer")
+    assert_close(got, ref, 2e-2, 0.9999, f"c2 layer, grid {grid}")
 
 
 def test_c2_one_layer_split_attention_schedule():
