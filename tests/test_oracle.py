@@ -441,3 +441,130 @@ def test_embed_images_packs_images_in_order():
     first = E.patch_embed(imgs[0], w, b, p) + E.bilinear_resize(t, 2, 3).reshape(6, C)
     second = E.patch_embed(imgs[1], w, b, p) + E.bilinear_resize(t, 1, 2).reshape(2, C)
     np.testing.assert_array_equal(got, np.concatenate([first, second]))
+
+
+# ------------------------------------------------------------------ MXFP8 (block-scaled 8-bit)
+from oracle import mxfp8_ref as MX  # noqa: E402
+
+
+def _torch_e4m3(x):
+    """PyTorch's float8_e4m3fn conversion (round to nearest even, no clamp)."""
+    return torch.tensor(np.asarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_table_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.tensor(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = MX.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+    # the definition's landmarks: 1.0, largest normal, smallest normal and subnormal
+    assert MX.e4m3_decode([0x38, 0x7E, 0x08, 0x01]).tolist() == [1.0, 448.0, 2.0 ** -6, 2.0 ** -9]
+
+
+def test_e4m3_round_trip_of_every_code():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    assert np.array_equal(MX.e4m3_encode(MX.e4m3_decode(codes)), codes)
+
+
+def test_e4m3_rounding_matches_torch():
+    # every midpoint between neighbouring values (ties), points just off them,
+    # and random values over the whole range, up to 464 (torch does not clamp)
+    v = np.unique(MX.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8)))
+    mids = (v[1:] + v[:-1]) / 2
+    pts = np.concatenate([v, mids, mids * (1 + 2.0 ** -12), mids * (1 - 2.0 ** -12),
+                          [464.0, 460.0, 449.0]])
+    r = rng(40)
+    pts = np.concatenate([pts, np.exp2(r.uniform(-12, np.log2(464), 4000))])
+    pts = np.concatenate([pts, -pts]).astype(np.float32).astype(np.float64)
+    assert np.array_equal(MX.e4m3_encode(pts), _torch_e4m3(pts))
+
+
+def test_e4m3_clamps_above_the_largest_normal():
+    x = np.array([465.0, 480.0, 1e6, -500.0, np.inf])
+    assert MX.e4m3_encode(x).tolist() == [0x7E, 0x7E, 0x7E, 0xFE, 0x7E]
+    assert MX.e4m3_encode([np.nan]).tolist() == [0x7F]
+
+
+def test_mx_block_exponent_closed_form():
+    # amax = f * 2^k with f in [1, 2) gives X = k - 8: the scaled maximum lands in [256, 512)
+    r = rng(41)
+    k = r.integers(-100, 100, 64)
+    f = r.uniform(1.0, 2.0, 64)
+    x = np.zeros((64, 40))
+    x[:, 0] = -f * np.exp2(k)           # the block maximum, negative on purpose
+    x[:, 1:32] = r.uniform(-1, 1, (64, 31)) * np.exp2(k)[:, None]
+    x[:, 32:] = 3.0                     # second block: 8 elements (K = 40)
+    X = MX.mx_block_exponents(x)
+    assert X.shape == (64, 2)
+    assert np.array_equal(X[:, 0], k - 8)
+    assert np.all(X[:, 1] == 1 - 8)     # log2(3) = 1.58: only the block's own elements count
+    assert MX.mx_block_exponents(np.zeros((1, 32)))[0, 0] == -127
+    assert MX.mx_block_exponents(np.full((1, 32), 2.0 ** 200))[0, 0] == 127
+
+
+def test_mx_quantize_exact_on_representable_blocks():
+    # elements that are E4M3 values times the block's own scale survive exactly
+    r = rng(42)
+    codes = r.integers(0, 0x7F, (16, 96)).astype(np.uint8) | (r.integers(0, 2, (16, 96)) << 7).astype(np.uint8)
+    codes[:, ::32] = 0x78 | (codes[:, ::32] & 0x80)       # each block holds +-256: X is the block's own
+    X = r.integers(-20, 20, (16, 3))
+    x = MX.e4m3_decode(codes) * np.exp2(np.repeat(X, 32, axis=1).astype(np.float64))
+    q, s = MX.mx_quantize(x)
+    assert np.array_equal(s.astype(np.int64) - 127, X)
+    assert np.array_equal(MX.mx_dequantize(q, s), x)
+
+
+def test_mx_quantize_error_bound():
+    # round to nearest: |x - deq| <= half the E4M3 spacing at x, times 2^X,
+    # except where the clamp at 448 * 2^X applies
+    r = rng(43)
+    x = r.standard_normal((32, 128)) * np.exp2(r.integers(-10, 10, (32, 1)))
+    q, s = MX.mx_quantize(x)
+    d = MX.mx_dequantize(q, s)
+    X = np.repeat(s.astype(np.int64) - 127, 32, axis=1).astype(np.float64)
+    sx = np.abs(x) / np.exp2(X)
+    clamp = sx > 448
+    spacing = np.exp2(np.maximum(np.floor(np.log2(np.maximum(sx, 2.0 ** -30))), -6) - 3)
+    err = np.abs(d - x) / np.exp2(X)
+    assert np.all(err[~clamp] <= spacing[~clamp] / 2)
+    assert np.all(np.abs(d[clamp]) == 448 * np.exp2(X[clamp]))
+    assert np.all(np.sign(d[d != 0]) == np.sign(x[d != 0]))
+
+
+def test_mx_linear_integer_closed_form():
+    # integer E4M3 values with scale 2^0: deq(A).deq(W)^T is an integer matmul
+    r = rng(44)
+    vals = np.arange(-16, 17)
+    a = r.choice(vals, (9, 70))
+    w = r.choice(vals, (13, 70))
+    a[:, [0, 32, 64]] = 288             # E4M3 block maxima in [256, 512) keep X = 0
+    w[:, [0, 32, 64]] = -256
+    qa, sa = MX.mx_quantize(a.astype(np.float64))
+    qw, sw = MX.mx_quantize(w.astype(np.float64))
+    assert np.all(sa == 127) and np.all(sw == 127)
+    b = r.integers(-5, 5, 13)
+    ref = (a.astype(np.int64) @ w.astype(np.int64).T + b).astype(np.float64)
+    assert np.array_equal(MX.mx_linear(qa, sa, qw, sw, b), ref)
+    res = r.standard_normal((9, 13))
+    assert np.array_equal(MX.mx_linear(qa, sa, qw, sw, b, "residual", res), ref + res)
+    g = MX.mx_linear(qa, sa, qw, sw, b, "gelu")
+    np.testing.assert_allclose(g, R.gelu_tanh(ref), rtol=0, atol=0)
+
+
+def test_mx_linear_power_of_two_rescaling():
+    # raising one block's scale byte by n multiplies exactly that block's
+    # contribution by 2^n
+    r = rng(45)
+    qa, sa = MX.mx_quantize(r.standard_normal((5, 64)))
+    qw, sw = MX.mx_quantize(r.standard_normal((7, 64)))
+    y = MX.mx_linear(qa, sa, qw, sw)
+    sa2 = sa.copy()
+    sa2[:, 1] += 3
+    y2 = MX.mx_linear(qa, sa2, qw, sw)
+    da = MX.mx_dequantize(qa, sa)
+    dw = MX.mx_dequantize(qw, sw)
+    part = da[:, 32:] @ dw[:, 32:].T
+    np.testing.assert_allclose(y2, y + 7 * part, rtol=1e-12, atol=1e-12)
