@@ -269,6 +269,44 @@ VIT_API vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w,
 VIT_API vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc,
                       int total_tokens, void *stream);
 
+/* ---- MXFP8 (block-scaled 8-bit) linear layer ----
+ * The pages name 8-bit inference as a next step without fixing a format (the
+ * NEO++ launcher page lists fp8 variants of its dense checkpoints; KLiteInfer
+ * README, section "已知限制与后续": FP16 / INT8 after CUDA Graph and operator
+ * fusion).  The format here is OCP Microscaling v1.0 MXFP8: E4M3 elements
+ * (bias 7, max 448, no infinity), one E8M0 scale 2^(s-127) per 32
+ * consecutive elements of a row.  bf16 contexts only.
+ *
+ * codes  : [rows, vit_mx8_row_bytes(K)] bytes, element (r, k) at
+ *          r * row_bytes + k (bytes past K are never read).
+ * scales : vit_mx8_scale_bytes(rows, K) bytes of 512-byte blocks, block
+ *          (rb, kb) = rows [128 rb, 128 rb + 128) x columns [128 kb, 128 kb +
+ *          128) at (rb * ceil(K/128) + kb) * 512; inside it the scale of row
+ *          128 rb + r0 + 32 r1 (r0 < 32, r1 < 4) and of its 32-column group j
+ *          (< 4) at byte 16 r0 + 4 r1 + j (the tensor core's scale-copy
+ *          shape).  Bytes of rows or groups past the matrix hold 127 (2^0).
+ * All buffers belong to the caller; device pointers 16-byte aligned. */
+VIT_API size_t vit_mx8_row_bytes(int K);
+VIT_API size_t vit_mx8_scale_bytes(int rows, int K);
+
+/* x bf16 [rows, K] (row stride K) -> codes, scales.  Per 32-element group:
+ * X = floor(log2 max|x|) - 8 clamped to [-127, 127] (-127 for an all-zero
+ * group), code = E4M3(x / 2^X) rounded to nearest even, magnitudes above 448
+ * clamped to 448.  Errors: VIT_ERR_INVALID_ARG (null or misaligned pointer,
+ * negative size), VIT_ERR_UNSUPPORTED (fp32 context). */
+VIT_API vit_status vit_mx8_quantize(vit_ctx *ctx, const void *x, int rows, int K,
+                                    void *codes, void *scales, void *stream);
+
+/* y bf16 [M, N] = epi(deq(A) deq(W)^T + bias) with A = (a_codes, a_scales)
+ * [M, K] and W = (w_codes, w_scales) [N, K] (a PyTorch Linear weight,
+ * quantised along K); bias bf16 [N] or NULL; residual bf16 [M, N] for
+ * VIT_EPI_BIAS_RESIDUAL.  fp32 accumulation on the tensor core (block-scaled
+ * MMA).  N a multiple of 8.  Errors as vit_linear. */
+VIT_API vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void *a_scales,
+                                  const void *w_codes, const void *w_scales, const void *bias,
+                                  const void *residual, void *y, int M, int N, int K,
+                                  vit_epilogue epi, void *stream);
+
 /* ---- launch accounting and per-kernel timing ---- */
 
 /* Kernel kinds counted by the context (one count per kernel launch). */
@@ -277,7 +315,8 @@ typedef enum {
   VIT_K_GEMM_OUT = 4, VIT_K_GEMM_FC1 = 5, VIT_K_GEMM_FC2 = 6, VIT_K_MERGE = 7,
   VIT_K_POSITIONS = 8, VIT_K_GEMM = 9, /* vit_linear, the patch projection */
   VIT_K_EMBED = 10, /* patch extraction, weight padding, position interpolation */
-  VIT_K_COUNT = 11
+  VIT_K_MX8_QUANTIZE = 11, VIT_K_GEMM_MX8 = 12, /* vit_mx8_quantize, vit_linear_mx8 */
+  VIT_K_COUNT = 13
 } vit_kernel_kind;
 
 /* enable != 0: every later kernel launch of this context is bracketed by two

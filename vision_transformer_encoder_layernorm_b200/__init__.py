@@ -27,7 +27,7 @@ F32, BF16 = 0, 1
 FLAG_NO_ROPE, FLAG_NO_MLP = 0x1, 0x2
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_RESIDUAL = 0, 1, 2
 KERNEL_KINDS = ("layernorm", "gemm_qkv", "rope", "attention", "gemm_out", "gemm_fc1",
-                "gemm_fc2", "merge", "positions", "gemm", "embed")
+                "gemm_fc2", "merge", "positions", "gemm", "embed", "mx8_quantize", "gemm_mx8")
 STATUS = {0: "VIT_OK", 1: "VIT_ERR_INVALID_ARG", 2: "VIT_ERR_SHAPE", 3: "VIT_ERR_UNSUPPORTED",
           4: "VIT_ERR_WORKSPACE", 5: "VIT_ERR_CUDA", 6: "VIT_ERR_TIMEOUT",
           7: "VIT_ERR_DEVICE_BOUNDS"}
@@ -91,6 +91,10 @@ ABI_FUNCTIONS = {
     "vit_graph_launch": (_I, [_P, _P]),
     "vit_graph_kernels": (ctypes.c_longlong, [_P]),
     "vit_graph_destroy": (None, [_P]),
+    "vit_mx8_row_bytes": (ctypes.c_size_t, [_I]),
+    "vit_mx8_scale_bytes": (ctypes.c_size_t, [_I, _I]),
+    "vit_mx8_quantize": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "vit_linear_mx8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "vit_get_last_device_status": (_I, [_P]),
     "vit_status_string": (ctypes.c_char_p, [_I]),
     "vit_version": (ctypes.c_char_p, []),
@@ -133,6 +137,16 @@ def _stream(stream) -> Optional[int]:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def mx8_row_bytes(K: int) -> int:
+    """Bytes per row of an MXFP8 code matrix with K columns."""
+    return int(lib.vit_mx8_row_bytes(K))
+
+
+def mx8_scale_bytes(rows: int, K: int) -> int:
+    """Bytes of the E8M0 scale blocks of a [rows, K] MXFP8 matrix."""
+    return int(lib.vit_mx8_scale_bytes(rows, K))
 
 
 def _grids_arr(grids: Sequence[Sequence[int]]):
@@ -256,6 +270,21 @@ class Context:
         N = w.shape[0]
         _check("vit_linear", lib.vit_linear(self._h, _ptr(x), _ptr(w), _ptr(bias), _ptr(residual),
                                             _ptr(y), M, N, K, epi, _stream(stream)))
+
+    def mx8_quantize(self, x, codes, scales, stream=None):
+        """bf16 x [rows, K] -> MXFP8 codes [rows, mx8_row_bytes(K)] (uint8) and
+        scales [mx8_scale_bytes(rows, K)] (uint8), see vit_mx8_quantize."""
+        rows, K = x.shape
+        _check("vit_mx8_quantize", lib.vit_mx8_quantize(self._h, _ptr(x), rows, K, _ptr(codes),
+                                                        _ptr(scales), _stream(stream)))
+
+    def linear_mx8(self, a, w, bias, y, K, epi=EPI_BIAS, residual=None, stream=None):
+        """y = epi(deq(A) deq(W)^T + bias) with a = (codes, scales) [M, K] and
+        w = (codes, scales) [N, K] from mx8_quantize."""
+        M, N = y.shape
+        _check("vit_linear_mx8", lib.vit_linear_mx8(self._h, _ptr(a[0]), _ptr(a[1]), _ptr(w[0]),
+                                                    _ptr(w[1]), _ptr(bias), _ptr(residual), _ptr(y),
+                                                    M, N, K, epi, _stream(stream)))
 
     def rope2d(self, qkv, pos_rc, stream=None):
         _check("vit_rope2d", lib.vit_rope2d(self._h, _ptr(qkv), _ptr(pos_rc), qkv.shape[0],

@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libvit.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["vit_api.cu", "k_rows.cu", "k_simt.cu", "k_gemm_tc.cu", "k_attn_tc.cu", "k_embed.cu"]
+SOURCES = ["vit_api.cu", "k_rows.cu", "k_simt.cu", "k_gemm_tc.cu", "k_attn_tc.cu", "k_embed.cu", "k_mx8.cu"]
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

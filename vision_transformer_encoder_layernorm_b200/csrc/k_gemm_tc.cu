@@ -23,7 +23,9 @@
 #include <stdlib.h>
 
 #include "kernels.h"
+#include "mx8.h"
 #include "sm100.cuh"
+#include "sm100_mx8.cuh"
 
 namespace vit {
 
@@ -731,6 +733,232 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
   }
   if (v.bn == 256) return launch_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
   return launch_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+}
+
+// ---------------------------------------------------------------- MXFP8 GEMM
+// The same persistent structure as gemm_tc_kernel with E4M3 operands and E8M0
+// block scales (OCP Microscaling v1.0): per 128-column k-block, the producer
+// brings a 128x128-byte tile of A codes and a BNx128 tile of W codes (the
+// same 128-byte swizzle atom as 64 bf16), plus the 512-byte scale blocks of
+// A's 128 rows and W's BN rows.  The MMA lane copies the scale blocks into
+// TMEM (tcgen05.cp, one copy per 128 rows), then issues four K = 32 block-
+// scaled MMAs; MMA k reads byte k of each row's scale word.  The scale
+// columns are rewritten every k-block: the tensor core runs copies and MMAs
+// of one thread in issue order.
+namespace gemm {
+constexpr int kMxBK = 128;                      // E4M3 elements (bytes) per k-block
+constexpr uint32_t kMxATileBytes = BM * kMxBK;  // 16 KB
+constexpr uint32_t kMxSfBlock = 512;            // scales of 128 rows x 128 columns
+template <int BN>
+struct CfgMx {
+  static constexpr uint32_t kBTileBytes = BN * kMxBK;
+  static constexpr int kSfbBlocks = BN / 128;
+  static constexpr uint32_t kSfOff = kMxATileBytes + kBTileBytes;
+  static constexpr uint32_t kStageBytes = kSfOff + kMxSfBlock * (1 + kSfbBlocks);
+  static constexpr int kStages = 6;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kSfaCol = 2 * BN;      // 4 columns
+  static constexpr uint32_t kSfbCol = 2 * BN + 4;  // 4 columns per 128 rows of W
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 2048 + 1024;
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KB alignment of the swizzled tiles");
+  static_assert(kSfbCol + 4 * kSfbBlocks <= kTmemCols, "TMEM columns");
+  static_assert(kStages <= 8, "barrier slots");
+};
+}  // namespace gemm
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(gemm::kThreads, 1)
+    gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfb,
+                    const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
+                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status) {
+  using namespace gemm;
+  using CF = CfgMx<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  Bars *bars = reinterpret_cast<Bars *>(smem + size_t(CF::kStages) * CF::kStageBytes);
+  volatile int *abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int k_blocks = (K + kMxBK - 1) / kMxBK;
+
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CF::kStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], kEpiWarps);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, CF::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  pdl_wait();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile % num_m, nb = tile / num_m;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t *sa = smem + size_t(stage) * CF::kStageBytes;
+          mbar_arrive_expect_tx(&bars->full[stage], CF::kStageBytes);
+          tma_load_2d(sa, &tmA, &bars->full[stage], kb * kMxBK, mb * BM);
+          tma_load_2d(sa + kMxATileBytes, &tmB, &bars->full[stage], kb * kMxBK, nb * BN);
+          bulk_load(sa + CF::kSfOff, sfa + (size_t(mb) * k_blocks + kb) * kMxSfBlock, kMxSfBlock,
+                    &bars->full[stage]);
+#pragma unroll
+          for (int i = 0; i < CF::kSfbBlocks; ++i)
+            bulk_load(sa + CF::kSfOff + kMxSfBlock * (1 + i),
+                      sfb + (size_t(nb * CF::kSfbBlocks + i) * k_blocks + kb) * kMxSfBlock,
+                      kMxSfBlock, &bars->full[stage]);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == CF::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < CF::kStages; ++s)
+          if (issued_mask & (1u << s)) drain_wait(&bars->full[s], (issued_parity >> s) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool any_mma = false;
+      const uint32_t sfa_t = tmem + CF::kSfaCol, sfb_t = tmem + CF::kSfbCol;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int a = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&bars->acc_empty[a], aphase ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + uint32_t(a * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&bars->full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + size_t(stage) * CF::kStageBytes);
+          const uint32_t sb = sa + kMxATileBytes;
+          const uint32_t ssf = sa + CF::kSfOff;
+          tmem_cp_32x128b_x4(sfa_t, smem_desc(ssf, 0, 128, 0));
+#pragma unroll
+          for (int i = 0; i < CF::kSfbBlocks; ++i)
+            tmem_cp_32x128b_x4(sfb_t + 4 * i, smem_desc(ssf + kMxSfBlock * (1 + i), 0, 128, 0));
+#pragma unroll
+          for (int k = 0; k < kMxBK / 32; ++k) {
+            const uint64_t ad = smem_desc(sa + k * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(sb + k * 32, 16, 1024, 2);
+            mma_mx8_ss(d_tmem, ad, bd, idesc_mx8(BM, BN, k, k), sfa_t | (uint32_t(k) << 30),
+                       sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+          }
+          any_mma = true;
+          mma_commit(&bars->empty[stage]);
+          if (++stage == CF::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&bars->acc_full[a]);
+      }
+      if (!ok && any_mma) {
+        mma_commit(&bars->drain);
+        drain_wait(&bars->drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int row_in_tile = (warp & 3) * 32 + lane;
+    __nv_bfloat16 *bias_w = reinterpret_cast<__nv_bfloat16 *>(bars + 1) + (warp - 2) * 128;
+    const RopeEpi none{};
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int a = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      stage_bias_warp<BN>(bias_w, bias, nb * BN, N, warp, lane);
+      if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
+      tc_fence_after();
+      const int row = mb * BM + row_in_tile;
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, none,
+                             bias_w, bias, res, y);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, CF::kTmemCols);
+  }
+  if (threadIdx.x == 0 && bars->abort_flag) report_status(status, kDevTimeout);
+}
+
+template <int BN, int EPI>
+static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb, const uint8_t *sfa,
+                                 const uint8_t *sfb, const void *b, const void *res, void *y, int M,
+                                 int N, int K, int num_sms, int *status, cudaStream_t st) {
+  using CF = gemm::CfgMx<BN>;
+  auto kern = gemm_mx8_kernel<BN, EPI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + BN - 1) / BN);
+  const int grid = std::max(1, std::min(tiles, num_sms));
+  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb, sfa, sfb,
+                    static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
+                    static_cast<__nv_bfloat16 *>(y), M, N, K, status);
+}
+
+cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes,
+                            const uint8_t *w_scales, const void *b, const void *res, void *y, int M,
+                            int N, int K, int epi, int num_sms, int *status, cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  constexpr int BN = 128;
+  CUtensorMap ta, tb;
+  if (encode_tensor_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K, M, mx8_row_bytes(K),
+                           gemm::kMxBK, gemm::BM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (encode_tensor_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K, N, mx8_row_bytes(K),
+                           gemm::kMxBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  switch (epi) {
+    case kEpiGelu:
+      return launch_mx8_bn<BN, kEpiGelu>(ta, tb, a_scales, w_scales, b, res, y, M, N, K, num_sms,
+                                         status, st);
+    case kEpiResidual:
+      return launch_mx8_bn<BN, kEpiResidual>(ta, tb, a_scales, w_scales, b, res, y, M, N, K,
+                                             num_sms, status, st);
+    default:
+      return launch_mx8_bn<BN, kEpiBias>(ta, tb, a_scales, w_scales, b, res, y, M, N, K, num_sms,
+                                         status, st);
+  }
 }
 
 }  // namespace vit

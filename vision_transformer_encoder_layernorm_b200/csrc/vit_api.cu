@@ -22,6 +22,7 @@
 
 #include "../../include/vit.h"
 #include "kernels.h"
+#include "mx8.h"
 
 // Launch accounting: a count per kernel kind, and (while enabled) a pair of
 // CUDA events around every launch.
@@ -642,6 +643,54 @@ vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels, const int32_t *grid
   // tokens = patches . w_pad^T + b_pe + interpolated table (residual epilogue)
   return cuda_status(run_linear(ctx, VIT_K_GEMM, patches, w_pad, b_pe, pos, y, int(T), C, kp,
                                 kEpiResidual, st));
+}
+
+// ---------------------------------------------------------------- MXFP8
+size_t vit_mx8_row_bytes(int K) { return K < 0 ? 0 : mx8_row_bytes(K); }
+size_t vit_mx8_scale_bytes(int rows, int K) {
+  return rows < 0 || K < 0 ? 0 : mx8_scale_bytes(rows, K);
+}
+
+vit_status vit_mx8_quantize(vit_ctx *ctx, const void *x, int rows, int K, void *codes,
+                            void *scales, void *stream) {
+  if (!ctx || !x || !codes || !scales || rows < 0 || K < 0) return VIT_ERR_INVALID_ARG;
+  if (ctx->cfg.dtype != VIT_BF16) return VIT_ERR_UNSUPPORTED;
+  if (!aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(x) & 1u))
+    return VIT_ERR_INVALID_ARG;
+  if (rows == 0 || K == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(counted(ctx, VIT_K_MX8_QUANTIZE, st, [&] {
+    return launch_mx8_quantize(x, rows, K, static_cast<uint8_t *>(codes),
+                               static_cast<uint8_t *>(scales), st);
+  }));
+}
+
+vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void *a_scales,
+                          const void *w_codes, const void *w_scales, const void *bias,
+                          const void *residual, void *y, int M, int N, int K, vit_epilogue epi,
+                          void *stream) {
+  if (!ctx || !a_codes || !a_scales || !w_codes || !w_scales || !y || M < 0 || N <= 0 || K <= 0)
+    return VIT_ERR_INVALID_ARG;
+  if (epi != VIT_EPI_BIAS && epi != VIT_EPI_BIAS_GELU && epi != VIT_EPI_BIAS_RESIDUAL)
+    return VIT_ERR_INVALID_ARG;
+  if (epi == VIT_EPI_BIAS_RESIDUAL && !residual) return VIT_ERR_INVALID_ARG;
+  if (ctx->cfg.dtype != VIT_BF16) return VIT_ERR_UNSUPPORTED;
+  if (N % 8) return VIT_ERR_UNSUPPORTED;
+  const void *ps[7] = {a_codes, a_scales, w_codes, w_scales, bias, residual, y};
+  for (const void *p : ps)
+    if (p && !aligned16(p)) return VIT_ERR_INVALID_ARG;
+  if (M == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(counted(ctx, VIT_K_GEMM_MX8, st, [&] {
+    return launch_gemm_mx8(static_cast<const uint8_t *>(a_codes),
+                           static_cast<const uint8_t *>(a_scales),
+                           static_cast<const uint8_t *>(w_codes),
+                           static_cast<const uint8_t *>(w_scales), bias,
+                           epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr, y, M, N, K, int(epi),
+                           ctx->num_sms, ctx->d_status, st);
+  }));
 }
 
 vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc, int total_tokens,
