@@ -151,6 +151,10 @@ def test_mx8_errors_launch_nothing(ctx):
     with pytest.raises(vit.VitError) as e:
         ctx.linear_mx8((a[0].view(-1)[1:], a[1]), a, None, y, K)      # misaligned codes
     assert e.value.code == 1
+    with pytest.raises(vit.VitError) as e:                         # misaligned input rows
+        xm = torch.empty(M * K + 8, dtype=torch.bfloat16, device="cuda")[1:1 + M * K].view(M, K)
+        ctx.mx8_quantize(xm, a[0], a[1])
+    assert e.value.code == 1
     f32 = vit.Context(256, 4, 64, 1024, vit.F32)
     try:
         with pytest.raises(vit.VitError) as e:

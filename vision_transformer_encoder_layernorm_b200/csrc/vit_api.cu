@@ -655,8 +655,7 @@ vit_status vit_mx8_quantize(vit_ctx *ctx, const void *x, int rows, int K, void *
                             void *scales, void *stream) {
   if (!ctx || !x || !codes || !scales || rows < 0 || K < 0) return VIT_ERR_INVALID_ARG;
   if (ctx->cfg.dtype != VIT_BF16) return VIT_ERR_UNSUPPORTED;
-  if (!aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(x) & 1u))
-    return VIT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return VIT_ERR_INVALID_ARG;
   if (rows == 0 || K == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
