@@ -104,3 +104,35 @@ def test_structs_keep_their_tensors_alive():
     del w
     gc.collect()
     assert wref() is not None and lw.w_qkv == wref().data_ptr() and lw.w_o is None
+
+
+def test_mx8_sizes_and_null_arguments_without_gpu():
+    # MXFP8 buffer sizes: rows of ceil(K/16)*16 code bytes; one 512-byte scale
+    # block per (128 rows, 128 columns), each holding 128 rows x 4 groups of 32
+    import vision_transformer_encoder_layernorm_b200 as vit
+    L = vit.lib
+    for K, rb in [(1, 16), (16, 16), (17, 32), (1152, 1152), (4304, 4304), (4305, 4320)]:
+        assert vit.mx8_row_bytes(K) == rb
+    for rows, K in [(1, 1), (128, 128), (129, 128), (3900, 1152), (4304, 4304), (0, 64)]:
+        assert vit.mx8_scale_bytes(rows, K) == -(-rows // 128) * -(-K // 128) * 512
+    assert L.vit_mx8_row_bytes(-1) == 0 and L.vit_mx8_scale_bytes(-1, 8) == 0
+    assert L.vit_mx8_quantize(None, None, 0, 0, None, None, None) == 1
+    assert L.vit_linear_mx8(None, None, None, None, None, None, None, None, 0, 0, 0, 0, None) == 1
+
+
+def test_mx8_scale_layout_is_a_bijection():
+    # the documented block layout (include/vit.h, vit_mx8_quantize) gives every
+    # (row, 32-column group) its own byte inside the buffer; what is left over
+    # is the padding of the last row block and column block
+    import vision_transformer_encoder_layernorm_b200 as vit
+    import numpy as np
+    for rows, K in [(300, 1152), (130, 4304), (5, 48), (257, 200)]:
+        nkb = -(-K // 128)
+        r = np.arange(rows)[:, None]
+        j = np.arange(-(-K // 32))[None, :]
+        off = ((r // 128) * nkb + j // 4) * 512 + (r % 32) * 16 + (r % 128 // 32) * 4 + j % 4
+        assert off.min() >= 0 and off.max() < vit.mx8_scale_bytes(rows, K)
+        assert np.unique(off).size == off.size
+        # a full 128-row x 128-column block uses each of its 512 bytes once
+        if rows >= 128 and K >= 128:
+            assert np.array_equal(np.sort(off[:128, :4].ravel()), np.arange(512))
