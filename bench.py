@@ -141,6 +141,40 @@ def oracle_step_time(max_seconds=15.0):
     return step, f"{n} of {wl.layers} layers of the 3900-token stack in fp64 (x{wl.layers / n:.1f}) + merge"
 
 
+def cpu_fp32_step_time(max_seconds=8.0):
+    """The same stack at the pages' own precision (fp32) on the host cores,
+    through the PyTorch CPU restatement of the layer that pins the oracle:
+    layers of the 3900-token stack until ``max_seconds`` (at least one),
+    scaled to all 27 layers.  Returns (seconds per step, sample text,
+    threads)."""
+    import torch
+
+    import synth
+    from oracle import run as orun
+    from oracle import vit_ref as R
+    from tests import torch_fp64_layer as TL
+
+    wl = synth.get(WORKLOAD)
+    inp = synth.make_inputs(wl, layers=3)
+    cu, pos = R.positions_from_grids(wl.grids)
+    ws = [{k: torch.as_tensor(v, dtype=torch.float32) for k, v in orun.layer_f64(inp, i).items()}
+          for i in range(3)]
+    x = torch.as_tensor(synth.to_f64(inp.x, wl.dtype), dtype=torch.float32)
+    n = 0
+    with torch.no_grad():
+        t0 = time.perf_counter()
+        while True:
+            x = torch.as_tensor(TL.layer(x, ws[n % 3], cu, pos, wl.heads, wl.head_dim, wl.ln_eps,
+                                         wl.rope_theta, dtype=torch.float32))
+            n += 1
+            if time.perf_counter() - t0 >= max_seconds or n >= wl.layers:
+                break
+        t = time.perf_counter() - t0
+    return (t / n * wl.layers,
+            f"{n} of {wl.layers} layers of the 3900-token stack in fp32 (x{wl.layers / n:.1f}), "
+            "no merge", torch.get_num_threads())
+
+
 def cpu_cores():
     try:
         from threadpoolctl import threadpool_info
@@ -582,6 +616,13 @@ def main():
         t_cpu, sample = oracle_step_time(max_seconds=15.0)
         cpu = {"value": T / t_cpu, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                "sample": sample}
+        try:  # context only: the pages' precision on the same host cores
+            t32, s32, th32 = cpu_fp32_step_time(8.0)
+            cpu["fp32_restatement"] = {"value": T / t32, "unit": UNIT, "threads": th32,
+                                       "kind": "PyTorch fp32 CPU restatement of the layer",
+                                       "sample": s32}
+        except Exception as e:  # never lose the bench line to the context figure
+            cpu["fp32_restatement"] = {"error": f"{type(e).__name__}: {e}"[:200]}
 
     if rank == 0:
         tflops = flops["total"] / (t_ms / 1e3) / 1e12
