@@ -15,6 +15,11 @@
  * spatial merge).  The prefix K/V segment follows the LightX2V NeoPP README,
  * section "KV file layout" (online layout [layers, 2, seq, kv_heads, d]).
  *
+ * Around the stack: patch embedding and bilinear position-table
+ * interpolation (the steps before it), a CUDA-graph capture of any sequence
+ * of calls, and an MXFP8 block-scaled linear layer (E4M3 codes, one E8M0
+ * scale per 32 elements) with its quantiser.
+ *
  * Conventions (all entry points):
  *  - Every tensor pointer is a DEVICE pointer owned by the caller, unless the
  *    parameter name ends in _host.  The library never allocates or frees
@@ -22,7 +27,8 @@
  *    by vit_init, freed by vit_destroy).
  *  - Activations are row-major [tokens, features] with contiguous rows.
  *    Weights use the [out_features, in_features] row-major layout.
- *  - Element type of every floating tensor = vit_config.dtype (fp32 or bf16).
+ *  - Element type of every floating tensor = vit_config.dtype (fp32 or bf16);
+ *    the MXFP8 entry points take byte codes and scales as documented there.
  *    bf16 runs tcgen05 tensor-core kernels with fp32 accumulation; fp32 runs
  *    SIMT FFMA kernels (no TF32).
  *  - Streams are passed as void* (a cudaStream_t; NULL = legacy stream).  All
