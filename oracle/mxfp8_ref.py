@@ -29,19 +29,27 @@ design notes):
     A is [M, K] (activations, blocks along each row); W is [N, K] (a
     PyTorch Linear weight, blocks along each row, i.e. per output column
     of y).
+16. An FP8 encoder layer runs the four projections (QKV, output, fc1, fc2)
+    in MXFP8: each projection's input activation and weight are quantised
+    along K, then multiplied as in 15.  LayerNorm, RoPE, attention, GELU
+    and the residual adds are those of the bf16 layer (vit_ref).
 
 Parity status: pinned by tests/test_oracle.py -- the E4M3 table and the
 rounding against PyTorch's float8_e4m3fn conversion, round trips of every
 code, the block exponent's closed form, exactness on representable blocks,
-the error bound of round-to-nearest, and the layer against an integer matmul
-and under power-of-two rescaling.
+the error bound of round-to-nearest, the linear layer against an integer
+matmul and under power-of-two rescaling, and the FP8 encoder layer against
+the fp64 layer (equal with the projections unquantised; every projection
+routed through the quantised product; bounded error when quantised).
 """
 from __future__ import annotations
 
 import numpy as np
 
+from . import vit_ref as R
+
 __all__ = ["E4M3_MAX", "BLOCK", "e4m3_decode", "e4m3_encode", "mx_block_exponents",
-           "mx_quantize", "mx_dequantize", "mx_linear"]
+           "mx_quantize", "mx_dequantize", "mx_linear", "mx_project", "layer_forward_mx8"]
 
 E4M3_MAX = 448.0
 BLOCK = 32
@@ -132,3 +140,28 @@ def mx_linear(a_codes, a_scales, w_codes, w_scales, bias=None, epilogue="none", 
     elif epilogue != "none":
         raise ValueError(epilogue)
     return y
+
+
+def mx_project(x, w, b=None):
+    """One projection of the FP8 layer: x [M, K] and w [N, K] each quantised
+    along K, then deq(x)·deq(w)^T + b (readings 13, 15, 16)."""
+    qa, sa = mx_quantize(x)
+    qw, sw = mx_quantize(w)
+    return mx_linear(qa, sa, qw, sw, b)
+
+
+def layer_forward_mx8(x, w, cu_seqlens, pos_rc, heads, head_dim, eps=1e-6, theta=10000.0,
+                      prefix_kv=None, attn_only=False, project=mx_project):
+    """The pre-LN encoder layer of vit_ref.layer_forward with its four
+    projections computed by ``project`` (MXFP8 by default, reading 16)."""
+    x = np.asarray(x, dtype=np.float64)
+    T = x.shape[0]
+    h = R.layernorm(x, w["ln1_g"], w["ln1_b"], eps)
+    q, k, v = R.split_qkv(project(h, w["w_qkv"], w["b_qkv"]), heads, head_dim)
+    o = R.attention(q, k, v, cu_seqlens, pos_rc, prefix_kv, None, theta)
+    x1 = x + project(o.reshape(T, heads * head_dim), w["w_o"], w["b_o"])
+    if attn_only:
+        return x1
+    h2 = R.layernorm(x1, w["ln2_g"], w["ln2_b"], eps)
+    g = R.gelu_tanh(project(h2, w["w_fc1"], w["b_fc1"]))
+    return x1 + project(g, w["w_fc2"], w["b_fc2"])

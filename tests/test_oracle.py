@@ -568,3 +568,50 @@ def test_mx_linear_power_of_two_rescaling():
     dw = MX.mx_dequantize(qw, sw)
     part = da[:, 32:] @ dw[:, 32:].T
     np.testing.assert_allclose(y2, y + 7 * part, rtol=1e-12, atol=1e-12)
+
+
+def _small_layer(seed, C=64, H=2, F=96, T=70):
+    r = rng(seed)
+    w = {"ln1_g": 1 + 0.02 * r.standard_normal(C), "ln1_b": 0.01 * r.standard_normal(C),
+         "w_qkv": 0.05 * r.standard_normal((3 * C, C)), "b_qkv": 0.01 * r.standard_normal(3 * C),
+         "w_o": 0.05 * r.standard_normal((C, C)), "b_o": 0.01 * r.standard_normal(C),
+         "ln2_g": 1 + 0.02 * r.standard_normal(C), "ln2_b": 0.01 * r.standard_normal(C),
+         "w_fc1": 0.05 * r.standard_normal((F, C)), "b_fc1": 0.01 * r.standard_normal(F),
+         "w_fc2": 0.05 * r.standard_normal((C, F)), "b_fc2": 0.01 * r.standard_normal(C)}
+    x = r.standard_normal((T, C))
+    cu = np.array([0, 40, T])
+    pos = np.stack([np.arange(T) // 7, np.arange(T) % 7], axis=1)
+    return x, w, cu, pos, H, C // H
+
+
+def test_mx_layer_with_plain_projections_is_the_fp64_layer():
+    x, w, cu, pos, H, d = _small_layer(46)
+    got = MX.layer_forward_mx8(x, w, cu, pos, H, d, project=R.linear)
+    assert np.array_equal(got, R.layer_forward(x, w, cu, pos, H, d))
+    got = MX.layer_forward_mx8(x, w, cu, pos, H, d, attn_only=True, project=R.linear)
+    assert np.array_equal(got, R.layer_forward(x, w, cu, pos, H, d, attn_only=True))
+
+
+def test_mx_layer_routes_every_projection_through_the_quantised_product():
+    x, w, cu, pos, H, d = _small_layer(47)
+    seen = []
+
+    def spy(a, wt, b=None):
+        seen.append((a.shape, wt.shape))
+        return MX.mx_project(a, wt, b)
+
+    MX.layer_forward_mx8(x, w, cu, pos, H, d, project=spy)
+    T, C = x.shape
+    F = w["w_fc1"].shape[0]
+    assert seen == [((T, C), (3 * C, C)), ((T, C), (C, C)), ((T, C), (F, C)), ((T, F), (C, F))]
+
+
+def test_mx_layer_error_is_bounded():
+    # E4M3 rounding of every projection's operands: well below the signal,
+    # but not zero
+    x, w, cu, pos, H, d = _small_layer(48)
+    ref = R.layer_forward(x, w, cu, pos, H, d)
+    got = MX.layer_forward_mx8(x, w, cu, pos, H, d)
+    dy, dr = got - x, ref - x          # the layer's own contribution, without the residual
+    cos = float(np.sum(dy * dr) / np.sqrt(np.sum(dy * dy) * np.sum(dr * dr)))
+    assert 0.99 <= cos < 1.0, cos
