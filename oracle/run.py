@@ -23,17 +23,33 @@ def sequence_args(wl):
     return cu, (pos if wl.rope else None)
 
 
+class _LazyLayers:
+    """Layers ``[0, n)`` of a workload's inputs, each widened to fp64 only
+    when the stack reaches it (27 fp64 layers of the 1152-wide model would
+    hold 3.3 GB at once)."""
+
+    def __init__(self, inputs, n):
+        self.inputs, self.n = inputs, n
+
+    def __len__(self):
+        return self.n
+
+    def __getitem__(self, i):
+        if not 0 <= i < self.n:
+            raise IndexError(i)
+        return layer_f64(self.inputs, i)
+
+
 def run_layers(inputs, x=None, n_layers=None):
-    """The layer stack of a workload on its seeded inputs (or on ``x``)."""
+    """The layer stack of a workload (``vit_ref.encoder_forward``) on its
+    seeded inputs, or on ``x``."""
     wl = inputs.workload
     cu, pos = sequence_args(wl)
     y = synth.to_f64(inputs.x, wl.dtype) if x is None else np.asarray(x, np.float64)
     pkv = None if inputs.prefix_kv is None else synth.to_f64(inputs.prefix_kv, wl.dtype)
     n = len(inputs.layers) if n_layers is None else n_layers
-    for i in range(n):
-        y = R.layer_forward(y, layer_f64(inputs, i), cu, pos, wl.heads, wl.head_dim,
-                            wl.ln_eps, wl.rope_theta, pkv, wl.attn_only)
-    return y
+    return R.encoder_forward(y, _LazyLayers(inputs, n), cu, pos, wl.heads, wl.head_dim,
+                             wl.ln_eps, wl.rope_theta, pkv, wl.attn_only)
 
 
 def run_workload(inputs, n_layers=None):

@@ -204,14 +204,13 @@ def layer_forward(x, w, cu_seqlens, pos_rc, heads, head_dim, eps=1e-6,
 def encoder_forward(x, layer_weights, cu_seqlens, pos_rc, heads, head_dim,
                     eps=1e-6, theta=10000.0, prefix_kv=None, attn_only=False):
     """The layer stack: each layer's output feeds the next (intro bullet:
-    27 layers).  ``layer_weights`` is a sequence of per-layer dicts (or a
-    callable returning the dict of layer i, to bound memory)."""
+    27 layers).  ``layer_weights`` is a sequence of per-layer dicts; anything
+    with ``len()`` and indexing will do, so a caller can widen each layer's
+    parameters only when the stack reaches it."""
     y = np.asarray(x, dtype=np.float64)
-    n = len(layer_weights)
-    for i in range(n):
-        w = layer_weights[i]
-        y = layer_forward(y, w, cu_seqlens, pos_rc, heads, head_dim, eps, theta,
-                          prefix_kv, attn_only)
+    for i in range(len(layer_weights)):
+        y = layer_forward(y, layer_weights[i], cu_seqlens, pos_rc, heads, head_dim, eps,
+                          theta, prefix_kv, attn_only)
     return y
 
 

@@ -345,14 +345,33 @@ def test_layer_matches_torch_restatement(P, attn_only):
     np.testing.assert_allclose(y, ref, atol=1e-12)
 
 
-def test_encoder_is_layer_composition():
-    wl, inp = _small_layer_inputs(51, [(4, 4)])
-    y2 = orun.run_layers(inp)
-    y1 = orun.run_layers(inp, n_layers=1)
+@pytest.mark.parametrize("P,attn_only", [(0, False), (3, True)])
+def test_stack_matches_torch_restatement_layer_by_layer(P, attn_only):
+    # The stack oracle (vit_ref.encoder_forward, reached through
+    # oracle.run.run_layers as every stack-level GPU test reaches it) against
+    # the independent PyTorch restatement applied once per layer, with each
+    # layer's own weights, over two packed images: a stack that reused one
+    # layer's weights, dropped or repeated a layer, or fed a layer the wrong
+    # input would differ.
+    wl = synth.Workload("t", 51, "f32", 64, 4, 16, 96, 3, ((3, 4), (2, 5)), prefix_len=P,
+                        kv_heads=(2 if P else 0), attn_only=attn_only)
+    inp = synth.make_inputs(wl)
+    got = orun.run_layers(inp)
     cu, pos = R.positions_from_grids(wl.grids)
-    np.testing.assert_allclose(
-        y2, R.layer_forward(y1, orun.layer_f64(inp, 1), cu, pos, wl.heads, wl.head_dim),
-        atol=1e-13)
+    pkv = None if inp.prefix_kv is None else synth.to_f64(inp.prefix_kv, wl.dtype)
+    ref = synth.to_f64(inp.x, wl.dtype)
+    outs = []
+    for i in range(wl.layers):
+        ref = torch_fp64_layer.layer(ref, orun.layer_f64(inp, i), cu, pos, wl.heads, wl.head_dim,
+                                     wl.ln_eps, wl.rope_theta, pkv, attn_only)
+        outs.append(ref)
+    np.testing.assert_allclose(got, ref, atol=1e-11)
+    # every layer changes the activations, so the comparison above covers
+    # each layer of the chain
+    for a, b in zip(outs, outs[1:]):
+        assert np.max(np.abs(a - b)) > 1e-3
+    # a shorter stack stops after its own last layer
+    np.testing.assert_allclose(orun.run_layers(inp, n_layers=2), outs[1], atol=1e-11)
 
 
 def test_c1_layer_matches_torch_restatement():
