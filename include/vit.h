@@ -148,12 +148,17 @@ VIT_API vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w,
  * it until the process exits).  The call allocates nothing: no cudaMalloc,
  * cudaFree or allocating library routine.  The caller still passes x, y and
  * the weights, as for vit_layer_forward.
- *  - Size limit: vit_workspace_bytes(ctx, total_tokens) must be <= 32 MiB
- *    (e.g. up to 1,240 tokens at hidden 1152 / MLP 4304); larger calls return
- *    VIT_ERR_WORKSPACE before anything is launched.
+ *  - Size limit: the layer's intermediates (LayerNorm output, qkv, attention
+ *    output, x1, MLP hidden; no split-attention scratch, which this call
+ *    never uses) must fit in 32 MiB: up to 1,240 tokens at hidden 1152 /
+ *    MLP 4304.  Larger calls return VIT_ERR_WORKSPACE before anything is
+ *    launched.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, once per device); make that first call before any
- *    stream capture.
+ *    (cudaGetSymbolAddress, once per device) and keeps it; make that first
+ *    call before any stream capture.  The kept address belongs to the
+ *    device's primary context: after cudaDeviceReset on that device (which
+ *    reloads the library's device code) the process must not call this
+ *    entry point again on that device.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents.  Nothing in it has to start at zero (every intermediate is
  *    written before it is read), so nothing is cleared.  Calls whose work
@@ -343,6 +348,17 @@ VIT_API vit_status vit_profile_read(vit_ctx *ctx, int kind, long long *launches,
  * it and returns VIT_OK, VIT_ERR_TIMEOUT or VIT_ERR_DEVICE_BOUNDS (or
  * VIT_ERR_CUDA when the device reports an error). */
 VIT_API vit_status vit_get_last_device_status(vit_ctx *ctx);
+
+/* Fault injection for tests of the bounded waits; the pages have no
+ * counterpart.  With bytes > 0, every later one-CTA GEMM launch of this
+ * context (vit_linear with at most 128 rows always takes that kernel)
+ * announces `bytes` more per pipeline stage than its copies deliver, so the
+ * stage barrier never completes.  The kernel's waits are bounded (2 s): it
+ * winds down, waits for its copies, frees its tensor memory and records
+ * VIT_ERR_TIMEOUT, which vit_get_last_device_status() returns; the context
+ * stays usable.  bytes = 0 (the default) turns the injection off; values
+ * above 65536 return VIT_ERR_INVALID_ARG. */
+VIT_API vit_status vit_debug_lost_tx(vit_ctx *ctx, unsigned bytes);
 
 /* Static string for a status code. */
 VIT_API const char *vit_status_string(vit_status s);

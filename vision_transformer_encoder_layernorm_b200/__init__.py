@@ -96,6 +96,7 @@ ABI_FUNCTIONS = {
     "vit_mx8_quantize": (_I, [_P, _P, _I, _I, _P, _P, _P]),
     "vit_linear_mx8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "vit_get_last_device_status": (_I, [_P]),
+    "vit_debug_lost_tx": (_I, [_P, ctypes.c_uint]),
     "vit_status_string": (ctypes.c_char_p, [_I]),
     "vit_version": (ctypes.c_char_p, []),
 }
@@ -289,6 +290,10 @@ class Context:
     def rope2d(self, qkv, pos_rc, stream=None):
         _check("vit_rope2d", lib.vit_rope2d(self._h, _ptr(qkv), _ptr(pos_rc), qkv.shape[0],
                                             _stream(stream)))
+
+    def debug_lost_tx(self, nbytes: int):
+        """Fault injection for the watchdog tests (vit_debug_lost_tx)."""
+        _check("vit_debug_lost_tx", lib.vit_debug_lost_tx(self._h, nbytes))
 
     def device_status(self) -> int:
         return lib.vit_get_last_device_status(self._h)

@@ -22,6 +22,8 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <atomic>
+
 #include "kernels.h"
 #include "mx8.h"
 #include "sm100.cuh"
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status,
-                   const __grid_constant__ RopeEpi re) {
+                   const __grid_constant__ RopeEpi re, uint32_t lost_tx) {
   using namespace gemm;
   using CF = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -301,7 +303,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           uint8_t *sa = smem + size_t(stage) * CF::kStageBytes;
-          mbar_arrive_expect_tx(&bars->full[stage], CF::kStageBytes);
+          // lost_tx > 0 only under fault injection (vit_debug_lost_tx): the
+          // stage then waits for bytes no copy delivers, and the bounded
+          // waits end the kernel with VIT_ERR_TIMEOUT
+          mbar_arrive_expect_tx(&bars->full[stage], CF::kStageBytes + lost_tx);
           tma_load_2d(sa, &tmA, &bars->full[stage], kb * BK, mb * BM);
           tma_load_2d(sa + kATileBytes, &tmB, &bars->full[stage], kb * BK, nb * BN);
           issued_mask |= 1u << stage;
@@ -562,25 +567,32 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+constexpr int kMaxDevices = 64;  // per-device caches of launch properties
+
+// cuTensorMapEncodeTiled, resolved once per process (thread-safe static init)
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
 
 CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
                               uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
                               uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
-  if (g_encode == nullptr) {
-    cudaDriverEntryPointQueryResult q;
-    void *fn = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        fn == nullptr)
-      return CUDA_ERROR_NOT_FOUND;
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return CUDA_ERROR_NOT_FOUND;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+  return encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
@@ -588,7 +600,8 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const vo
 template <int BN, int EPI>
 static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
                              const void *res, void *y, int M, int N, int K, int num_sms,
-                             int *status, cudaStream_t st, const RopeEpi &re) {
+                             int *status, cudaStream_t st, const RopeEpi &re,
+                             uint32_t lost_tx) {
   using CF = gemm::Cfg<BN>;
   auto kern = gemm_tc_kernel<BN, EPI>;
   cudaError_t e =
@@ -598,20 +611,23 @@ static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const
   const int grid = std::max(1, std::min(tiles, num_sms));
   return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb,
                     static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-                    static_cast<__nv_bfloat16 *>(y), M, N, K, status, re);
+                    static_cast<__nv_bfloat16 *>(y), M, N, K, status, re, lost_tx);
 }
 
 template <int BN>
 static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
                               const void *b, const void *res, void *y, int M, int N, int K,
-                              int num_sms, int *status, cudaStream_t st) {
+                              int num_sms, int *status, cudaStream_t st, uint32_t lost_tx) {
   switch (epi) {
     case kEpiGelu:
-      return launch_bn<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{});
+      return launch_bn<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{},
+                                     lost_tx);
     case kEpiResidual:
-      return launch_bn<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{});
+      return launch_bn<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st,
+                                         RopeEpi{}, lost_tx);
     default:
-      return launch_bn<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{});
+      return launch_bn<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{},
+                                     lost_tx);
   }
 }
 
@@ -635,9 +651,14 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // SM pairs that can hold one CTA pair each (clusters live inside a GPC)
-  static int max_clusters = -1;
-  if (max_clusters < 0) {
+  // SM pairs that can hold one CTA pair each (clusters live inside a GPC),
+  // queried once per device and kernel (0 = not yet known; concurrent first
+  // calls compute the same value)
+  static std::atomic<int> cached[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  int max_clusters = dev < kMaxDevices ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (max_clusters <= 0) {
     cfg.gridDim = dim3(2 * (num_sms / 2));
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
@@ -645,6 +666,7 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
       n = num_sms / 2;
     }
     max_clusters = n;
+    if (dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
   }
   const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + TS - 1) / TS);
   return launch_pdl(kern, dim3(2 * std::max(1, std::min(tiles, max_clusters))),
@@ -706,7 +728,7 @@ static GemmVariant choose_variant(int M, int N, int K, int num_sms) {
 
 cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
                            int M, int N, int K, int epi, int num_sms, int *status,
-                           cudaStream_t st, const RopeEpi *rope) {
+                           cudaStream_t st, const RopeEpi *rope, uint32_t lost_tx) {
   if (M == 0 || N == 0) return cudaSuccess;
   GemmVariant v = choose_variant(M, N, K, num_sms);
   if (epi == kEpiRope) {  // tiles of whole heads on a CTA pair: 3 x 72 (MMA N = 224) or 2 x 128
@@ -731,8 +753,9 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
     if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
     return launch_pair_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
   }
-  if (v.bn == 256) return launch_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
-  return launch_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+  if (v.bn == 256)
+    return launch_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st, lost_tx);
+  return launch_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st, lost_tx);
 }
 
 // ---------------------------------------------------------------- MXFP8 GEMM

@@ -90,9 +90,12 @@ cudaError_t launch_attention_simt(int dtype, const void *qkv, void *o, const Seq
 
 // tcgen05 GEMM, bf16 in / bf16 out, fp32 accumulation in TMEM.
 struct GemmPlan;
+// lost_tx: fault injection for the watchdog tests (0 in normal use): the
+// one-CTA kernel's stage barriers expect this many bytes more than arrive.
 cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
                            int M, int N, int K, int epi, int num_sms, int *status,
-                           cudaStream_t st, const RopeEpi *rope = nullptr);
+                           cudaStream_t st, const RopeEpi *rope = nullptr,
+                           uint32_t lost_tx = 0);
 
 // tcgen05 flash attention, bf16, head_dim 72 or 128.
 // Split (stream-K) attention schedule: most CTAs it uses, and the bytes of

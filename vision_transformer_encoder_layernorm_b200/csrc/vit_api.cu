@@ -71,6 +71,9 @@ struct vit_ctx {
   cudaStream_t cap_stream = nullptr;
   bool cap_prof_on = false;
   long long cap_launches0 = 0;
+  // fault injection (vit_debug_lost_tx): extra bytes the one-CTA GEMM's
+  // stage barriers wait for; 0 in normal use
+  uint32_t debug_lost_tx = 0;
 };
 
 struct vit_graph {
@@ -151,7 +154,8 @@ cudaError_t run_linear(vit_ctx *ctx, int kind, const void *x, const void *w, con
                        const RopeEpi *rope = nullptr) {
   return counted(ctx, kind, st, [&] {
     if (ctx->cfg.dtype == VIT_F32) return launch_gemm_simt(kF32, x, w, b, res, y, M, N, K, epi, st);
-    return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st, rope);
+    return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st, rope,
+                          ctx->debug_lost_tx);
   });
 }
 
@@ -267,8 +271,10 @@ vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, v
   return VIT_OK;
 }
 
+// sk_ctas: CTAs of the split attention schedule whose scratch the caller's
+// workspace layout holds (split_ctas(), or 0 where the split is never used)
 vit_status check_layer_call(vit_ctx *ctx, const void *x, void *y, const vit_seqs *seqs,
-                            void *workspace, size_t ws_bytes) {
+                            void *workspace, size_t ws_bytes, int sk_ctas) {
   if (!ctx) return VIT_ERR_INVALID_ARG;
   vit_status s = check_seqs(ctx, seqs, true);
   if (s != VIT_OK) return s;
@@ -277,7 +283,7 @@ vit_status check_layer_call(vit_ctx *ctx, const void *x, void *y, const vit_seqs
   if (ctx->cfg.dtype == VIT_BF16 && (!aligned16(x) || !aligned16(y))) return VIT_ERR_INVALID_ARG;
   if (seqs->total_tokens > 0 && !(ctx->cfg.flags & VIT_FLAG_NO_ROPE) && !seqs->pos_rc)
     return VIT_ERR_INVALID_ARG;
-  const size_t need = workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr, split_ctas(ctx, seqs->total_tokens));
+  const size_t need = workspace_layout(ctx->cfg, seqs->total_tokens, nullptr, nullptr, sk_ctas);
   if (!workspace || ws_bytes < need) return VIT_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return VIT_ERR_WORKSPACE;
   return VIT_OK;
@@ -482,7 +488,8 @@ size_t vit_workspace_bytes(const vit_ctx *ctx, int total_tokens) {
 vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const void *x, void *y,
                              const vit_seqs *seqs, void *workspace, size_t ws_bytes,
                              void *stream) {
-  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes);
+  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes,
+                                  seqs ? split_ctas(ctx, seqs->total_tokens) : 0);
   if (s != VIT_OK) return s;
   if ((s = check_layer_weights(ctx->cfg, w)) != VIT_OK) return s;
   if (seqs->total_tokens == 0) return VIT_OK;
@@ -499,7 +506,8 @@ vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const voi
 vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, int n_layers,
                                const void *x, void *y, const vit_seqs *seqs, void *workspace,
                                size_t ws_bytes, void *stream) {
-  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes);
+  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes,
+                                  seqs ? split_ctas(ctx, seqs->total_tokens) : 0);
   if (s != VIT_OK) return s;
   if (!layers || n_layers < 1) return VIT_ERR_INVALID_ARG;
   for (int i = 0; i < n_layers; ++i)
@@ -800,6 +808,12 @@ vit_status vit_profile_read(vit_ctx *ctx, int kind, long long *launches, double 
   return VIT_OK;
 }
 
+vit_status vit_debug_lost_tx(vit_ctx *ctx, unsigned bytes) {
+  if (!ctx || bytes > 65536u) return VIT_ERR_INVALID_ARG;  // keeps the tx count in range
+  ctx->debug_lost_tx = bytes;
+  return VIT_OK;
+}
+
 vit_status vit_get_last_device_status(vit_ctx *ctx) {
   if (!ctx) return VIT_ERR_INVALID_ARG;
   DeviceGuard g(ctx->device);
@@ -865,7 +879,9 @@ extern "C" vit_status vit_layer_forward_noalloc(vit_ctx *ctx, const vit_layer_we
   void *scratch = nullptr;
   vit_status s = static_scratch(ctx->device, &scratch);
   if (s != VIT_OK) return s;
-  if ((s = check_layer_call(ctx, x, y, seqs, scratch, kStaticScratchBytes)) != VIT_OK) return s;
+  // the layout below holds no split-attention scratch (part and cnt stay
+  // null, so attention takes the whole-item schedule): size it the same way
+  if ((s = check_layer_call(ctx, x, y, seqs, scratch, kStaticScratchBytes, 0)) != VIT_OK) return s;
   if ((s = check_layer_weights(ctx->cfg, w)) != VIT_OK) return s;
   if (seqs->total_tokens == 0) return VIT_OK;
   Workspace ws;
