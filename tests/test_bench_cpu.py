@@ -31,6 +31,10 @@ def test_reference_arm_prints_one_json_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert "workload" in d["config"]
+    # what was timed: a sample of layers per step, scaled to the full step
+    assert 1 <= d["extrapolated_from_layers"] <= 27
+    assert d["ms_per_full_step_estimate"] >= d["ms_per_step"] * 0.5
+    assert abs(3900.0 / (d["ms_per_full_step_estimate"] / 1e3) - d["value"]) < 1e-6 * d["value"]
 
 
 def test_reference_arm_runs_on_rank_zero_only():
