@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ln", default="plain", choices=["plain", "folded"],
+                    help="LayerNorm as its own kernel (plain) or folded into the next GEMM")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the timing of the c1, c3 and c4 workloads")
     ap.add_argument("--no-graph", action="store_true",
@@ -290,7 +292,17 @@ def main():
 
     ctx = vit.Context(C, wl.heads, wl.head_dim, wl.mlp, vit.BF16, device=local_rank)
     layers = [{k: dev(v) for k, v in lw.items()} for lw in inp.layers]
-    lw_structs = [vit.layer_weights(l) for l in layers]
+    # --ln folded: weights prepared once, as a model is when it is loaded,
+    # each layer's LayerNorms folded into the projection after them
+    # (vit_fold_layernorm), so a layer runs 5 kernels and no LayerNorm pass;
+    # --ln plain: the layer as written (LayerNorm kernels).  The other one is
+    # timed too, as `ln_other`.
+    folded = [ctx.fold_layernorm(l) for l in layers]
+    torch.cuda.synchronize()
+    fold_structs = [vit.layer_weights(l) for l in folded]
+    plain_structs = [vit.layer_weights(l) for l in layers]
+    lw_structs, other_structs = ((fold_structs, plain_structs) if args.ln == "folded"
+                                 else (plain_structs, fold_structs))
     x = dev(inp.x)
     cu = torch.empty(2, dtype=torch.int32, device="cuda")
     pos = torch.empty((T, 2), dtype=torch.int32, device="cuda")
@@ -365,6 +377,7 @@ def main():
         "gemm_fc1": (2.0 * T * Fm * C, None), "gemm_fc2": (2.0 * T * C * Fm, None),
         "attention": (4.0 * T * T * C, None),
         "layernorm": (None, 2.0 * T * C * 2 + 2 * C * 2),
+        "rowstats": (None, 1.0 * T * C * 2 + T * ((C + 63) // 64) * 8),
         "rope": (None, 2.0 * T * 2 * C * 2 + T * 8), "merge": (None, 2.0 * T * C * 2),
     }
     pk, pk_src = peaks()
@@ -565,6 +578,35 @@ def main():
             ms = replicas.max_over_ranks(float(np.mean(r["ms"])), device="cuda")
             enc_only["%dx%d" % r["grid"]] = {"value": world * T / (ms / 1e3), "ms_per_step": ms,
                                              "tflops": flops["total"] / (ms / 1e3) / 1e12}
+    # ---- the same step with the other LayerNorm variant (--ln), for
+    # comparison with the step above: graph replays, L2 flushed before each
+    plain = None
+    if not args.layers and graph is not None:
+        cs = ctx.graph_begin()
+        ctx.encoder_forward(other_structs, x, y, sq, ws, cs)
+        ctx.spatial_merge_2x2(y, out, wl.grids, C, cs)
+        pg = ctx.graph_end()
+        for _ in range(args.warmup):
+            pg.launch(stream)
+        pev = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            pg.launch(stream)
+            e1.record(stream)
+            pev.append((e0, e1))
+        torch.cuda.synchronize()
+        pg.close()
+        p_ms = replicas.max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in pev])),
+                                       device="cuda")
+        plain = {"ln": "plain" if args.ln == "folded" else "folded",
+                 "value": world * T / (p_ms / 1e3), "ms_per_step": p_ms,
+                 "note": "the same step with the other LayerNorm variant: plain = a LayerNorm "
+                         "kernel before every QKV and fc1 GEMM; folded = LayerNorms folded into "
+                         "those GEMMs (one row-statistics launch per step in place of 54 "
+                         "LayerNorm launches)"}
+
     # ---- the workload's other configurations, each timed as graph replays
     # (3 warm-ups, then `steps` replays with the L2 flushed before each and
     # events around each), plus a profiled direct pass for the attention
@@ -630,6 +672,8 @@ def main():
         wl1 = synth.get("c1")
         in1 = synth.make_inputs(wl1)
         l1 = [{k: dev(v) for k, v in in1.layers[0].items()}]
+        if args.ln == "folded":
+            l1 = [ctx.fold_layernorm(l1[0])]
         l1s = [vit.layer_weights(l1[0])]
         x1c = dev(in1.x)
         y1c = torch.empty_like(x1c)
@@ -643,7 +687,7 @@ def main():
         ws3 = torch.empty(ctx.workspace_bytes(wl3.tokens), dtype=torch.uint8, device="cuda")
         time_config("c3", ctx, lambda st: ctx.encoder_forward(lw_structs, x3c, y3c, sq3, ws3, st),
                     wl3)
-        other["c3"]["weights"] = "the c2 stack's 27 layers (same shapes)"
+        other["c3"]["weights"] = f"the c2 stack's 27 layers (same shapes), LayerNorm {args.ln}"
         del ws3
         # c4
         wl4 = synth.get("c4")
@@ -651,6 +695,8 @@ def main():
         ctx4 = vit.Context(wl4.hidden, wl4.heads, wl4.head_dim, 0, vit.BF16,
                            flags=vit.FLAG_NO_MLP, device=local_rank)
         l4 = {k: (dev(v) if v.size else None) for k, v in in4.layers[0].items()}
+        if args.ln == "folded":
+            l4 = ctx4.fold_layernorm(l4)
         l4s = [vit.layer_weights(l4)]
         x4c = dev(in4.x)
         y4c = torch.empty_like(x4c)
@@ -694,6 +740,31 @@ def main():
                                            "27x27 position table", "us": us,
                                "tflops": fl / us / 1e6, "frac_bf16": fl / us / 1e6 / tensor_peak,
                                "launches": 4, "note": "graph replays back to back, inputs in L2"}}
+        # the projector composition after the merge (LayerNorm over 4C,
+        # linear + GELU, linear) on the merged c2 tokens, widths 4608 -> 4608
+        # -> 1024 (the pages give none), graph replays
+        pj = {k: dev(v) for k, v in synth.make_projector_weights(4 * C, 4 * C, 1024, 5, "bf16").items()}
+        pj_y = torch.empty((T // 4, 1024), dtype=torch.bfloat16, device="cuda")
+        pj_ws = torch.empty(ctx.projector_workspace_bytes(T // 4, 4 * C, 4 * C), dtype=torch.uint8,
+                            device="cuda")
+        cs = ctx.graph_begin()
+        ctx.projector(pj, out, pj_y, pj_ws, cs)
+        pg2 = ctx.graph_end()
+        for _ in range(3):
+            pg2.launch(stream)
+        flush.zero_()
+        e0.record(stream)
+        for _ in range(n_rep):
+            pg2.launch(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pg2.close()
+        pus = e0.elapsed_time(e1) * 1e3 / n_rep
+        pfl = 2.0 * (T // 4) * 4 * C * (4 * C + 1024)
+        nxt["projector"] = {"workload": "975 merged tokens, LayerNorm over 4608, 4608 -> 4608 "
+                                        "(GELU) -> 1024", "us": pus, "tflops": pfl / pus / 1e6,
+                            "frac_bf16": pfl / pus / 1e6 / tensor_peak, "launches": 3,
+                            "note": "graph replays back to back, inputs in L2"}
         # MXFP8 block-scaled GEMM on fc1's shape (3900 x 4304 x 1152, bias +
         # GELU) with layer 0's fc1 weights quantised once outside the timed
         # region; the activations' quantisation is timed on its own
@@ -755,6 +826,10 @@ def main():
             "dtype": "bf16", "data": "synthetic (seeded, synth.c2; random-init weights)",
             "config": {"workload": "c2: 27-layer ViT encoder, 3900 patches (50x78 grid), "
                                    "hidden 1152, 16x72 heads, MLP 4304, + 2x2 merge to 975x4608",
+                       "weights": ("random-init (seeded), LayerNorms folded into the next "
+                                   "projection once before timing (vit_fold_layernorm)"
+                                   if args.ln == "folded" else "random-init (seeded)"),
+                       "layernorm": args.ln,
                        "global_batch": world, "seq_len": T,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every timed step (256 MiB write)",
@@ -768,6 +843,7 @@ def main():
             "e2e": e2e, "gpu_launches": launches, "clocks": clk,
             **({"encoder_only": enc_only} if enc_only else {}),
             **({"configs": other} if other else {}),
+            **({"ln_other": plain} if plain else {}),
             **({"next": nxt} if nxt else {}),
         }
         print(json.dumps(line), flush=True)

@@ -90,10 +90,19 @@ typedef struct {
 /* One layer's parameters; all device pointers of cfg.dtype.
  * w_qkv [3C, C] (output rows: Q heads 0..H-1, then K, then V; d each),
  * w_o [C, C], w_fc1 [F, C], w_fc2 [C, F]; biases and LayerNorm vectors 1-D.
- * The ln2 / fc pointers may be NULL with VIT_FLAG_NO_MLP. */
+ * The ln2 / fc pointers may be NULL with VIT_FLAG_NO_MLP.
+ *
+ * LayerNorm folded into the projection after it (bf16 only; see
+ * vit_fold_layernorm): when qkv_fold is not NULL, w_qkv must be the folded
+ * weight W_qkv diag(ln1_g) and qkv_fold points to fp32 [2][3C] = (s, c) of
+ * that fold; ln1_g, ln1_b and b_qkv are then not read (may be NULL).  The
+ * layer then launches no LayerNorm: the QKV GEMM reads the raw x and its
+ * epilogue applies the normalisation.  fc1_fold likewise for LN2 and fc1
+ * (fp32 [2][F]; ln2_g, ln2_b, b_fc1 not read).  Both NULL: the plain layer. */
 typedef struct {
   const void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o;
   const void *ln2_g, *ln2_b, *w_fc1, *b_fc1, *w_fc2, *b_fc2;
+  const void *qkv_fold, *fc1_fold;
 } vit_layer_weights;
 
 /* Packed variable-length sequences (images).  Tokens of sequence s are rows
@@ -129,6 +138,30 @@ VIT_API void vit_destroy(vit_ctx *ctx);
  * total_tokens tokens (256-byte aligned base required). */
 VIT_API size_t vit_workspace_bytes(const vit_ctx *ctx, int total_tokens);
 
+/* Folds each pre-LayerNorm into the projection that reads its output
+ * (KLiteInfer README, 架构 / 视觉算子: LayerNorm, then GEMM + bias, over
+ * the same rows).  For a row x with mean m and r = 1/sqrt(var + eps):
+ *   LN(x) W^T + b = r (x W'^T - m s) + c,
+ *   W' = W diag(gamma),  s_n = sum_k W'_nk,  c = b + W beta,
+ * an exact identity; the folded GEMM needs only each row's m and r, which
+ * the kernel that wrote the row supplies (see vit_layer_weights), so the
+ * LayerNorm kernel and its round trip through memory disappear.
+ * Rounding: W' is rounded once to bf16 (in place of the LayerNorm output);
+ * s is summed from the rounded W' and c from W and beta, in fp32.
+ *   in       the layer's plain weights (ln1_g, ln1_b, w_qkv, b_qkv read for
+ *            the QKV fold; ln2_g, ln2_b, w_fc1, b_fc1 for the fc1 fold)
+ *   w_qkv_out  [3C, C] bf16 folded weight (may equal in->w_qkv: in place)
+ *   qkv_fold   fp32 [2][3C]: s, then c
+ *   w_fc1_out  [F, C] bf16 (may equal in->w_fc1),  fc1_fold fp32 [2][F]
+ * Either output pair may be NULL to skip that fold (both NULL: nothing is
+ * done).  bf16 contexts only (else VIT_ERR_UNSUPPORTED); pointers 16-byte
+ * aligned.  Weights of a model are folded once, when they are loaded; the
+ * caller then fills a vit_layer_weights with w_qkv = w_qkv_out,
+ * qkv_fold = qkv_fold, and so on. */
+VIT_API vit_status vit_fold_layernorm(vit_ctx *ctx, const vit_layer_weights *in,
+                                      void *w_qkv_out, void *qkv_fold, void *w_fc1_out,
+                                      void *fc1_fold, void *stream);
+
 /* One pre-LN encoder layer (reading: x1 = x + Wo Attn(RoPE(Wqkv LN1(x))) + bo;
  * y = x1 + W2 GELU(W1 LN2(x1) + b1) + b2).  x, y: [T, C]; y may not alias x.
  * With VIT_FLAG_NO_MLP y = x1 (DiT-style attention half-layer). */
@@ -149,10 +182,10 @@ VIT_API vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w,
  * cudaFree or allocating library routine.  The caller still passes x, y and
  * the weights, as for vit_layer_forward.
  *  - Size limit: the layer's intermediates (LayerNorm output, qkv, attention
- *    output, x1, MLP hidden; no split-attention scratch, which this call
- *    never uses) must fit in 32 MiB: up to 1,240 tokens at hidden 1152 /
- *    MLP 4304.  Larger calls return VIT_ERR_WORKSPACE before anything is
- *    launched.
+ *    output, x1, MLP hidden, row statistics; no split-attention scratch,
+ *    which this call never uses) must fit in 32 MiB: up to 1,227 tokens at
+ *    hidden 1152 / MLP 4304.  Larger calls return VIT_ERR_WORKSPACE before
+ *    anything is launched.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, once per device) and keeps it; make that first
  *    call before any stream capture.  The kept address belongs to the
@@ -250,11 +283,38 @@ VIT_API vit_status vit_pos_interp(vit_ctx *ctx, const void *pos_table, int table
                                   const int32_t *grids_hw_host, int n_images, void *y,
                                   void *stream);
 
+/* ---- projector after the merge ------------------------------------------
+ * The KLiteInfer README's intro bullet names the projector only as the 2x2
+ * spatial merge (vit_spatial_merge_2x2).  For models that follow the merge
+ * with a LayerNorm and a two-layer GELU MLP mapping the merged tokens to the
+ * decoder's width, this call runs that composition with caller-chosen
+ * widths:
+ *   y = GELU_tanh(LN(x) W1^T + b1) W2^T + b2
+ * x [M, d_in] (merged tokens, d_in = 4C), LayerNorm over d_in (biased
+ * variance, eps = cfg.ln_eps), W1 [d_hidden, d_in], W2 [d_out, d_hidden],
+ * y [M, d_out].  Launches: the LayerNorm (a block per row above 4096
+ * columns), then two GEMMs (vit_linear's kernels, bias + GELU and bias
+ * epilogues).  Workspace: vit_projector_workspace_bytes (LN output and the
+ * hidden activations, 256-byte aligned).  bf16: d_in, d_hidden, d_out
+ * multiples of 8; d_in <= 16384.  No trained projector is available, so
+ * parity is with the fp64 composition only. */
+typedef struct {
+  const void *ln_g, *ln_b;  /* [d_in] */
+  const void *w1, *b1;      /* [d_hidden, d_in], [d_hidden] */
+  const void *w2, *b2;      /* [d_out, d_hidden], [d_out] */
+} vit_projector_weights;
+VIT_API size_t vit_projector_workspace_bytes(const vit_ctx *ctx, int M, int d_in, int d_hidden);
+VIT_API vit_status vit_projector(vit_ctx *ctx, const vit_projector_weights *w, const void *x,
+                                 void *y, int M, int d_in, int d_hidden, int d_out,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
 /* ---- single steps of the layer, exposed for step-level use and testing --- */
 
 /* LayerNorm over the last axis ("视觉算子": LayerNorm), biased variance,
  * y = (x - mean)/sqrt(var + eps) * gamma + beta.  x, y [rows, cols];
- * y may alias x. */
+ * y may alias x.  cols a multiple of 4, at most 16384 (rows of up to 4096
+ * columns take one warp each, wider rows one block each), else
+ * VIT_ERR_UNSUPPORTED. */
 VIT_API vit_status vit_layernorm(vit_ctx *ctx, const void *x, void *y,
                          const void *gamma, const void *beta, int rows,
                          int cols, float eps, void *stream);
@@ -327,7 +387,9 @@ typedef enum {
   VIT_K_POSITIONS = 8, VIT_K_GEMM = 9, /* vit_linear, the patch projection */
   VIT_K_EMBED = 10, /* patch extraction, weight padding, position interpolation */
   VIT_K_MX8_QUANTIZE = 11, VIT_K_GEMM_MX8 = 12, /* vit_mx8_quantize, vit_linear_mx8 */
-  VIT_K_COUNT = 13
+  VIT_K_ROWSTATS = 13, /* row statistics of a stack's input (folded LayerNorm) */
+  VIT_K_FOLD = 14,     /* vit_fold_layernorm */
+  VIT_K_COUNT = 15
 } vit_kernel_kind;
 
 /* enable != 0: every later kernel launch of this context is bracketed by two

@@ -49,7 +49,7 @@ import numpy as np
 __all__ = [
     "layernorm", "linear", "gelu_tanh", "rope2d_frequencies", "rope2d",
     "attention", "attention_segment", "layer_forward", "encoder_forward",
-    "spatial_merge_2x2", "positions_from_grids", "split_qkv",
+    "spatial_merge_2x2", "positions_from_grids", "split_qkv", "projector",
 ]
 
 
@@ -212,6 +212,18 @@ def encoder_forward(x, layer_weights, cu_seqlens, pos_rc, heads, head_dim,
         y = layer_forward(y, layer_weights[i], cu_seqlens, pos_rc, heads, head_dim, eps,
                           theta, prefix_kv, attn_only)
     return y
+
+
+# ------------------------------------------------------------------ projector
+def projector(x, w, eps=1e-6):
+    """The projector that may follow the 2x2 merge, as a composition of the
+    steps above with caller-chosen widths (the intro bullet names the
+    projector only as the 2x2 spatial merge; a LayerNorm and a two-layer
+    GELU MLP after it is the reading taken for models that add one):
+    y = GELU_tanh(LN(x) W1^T + b1) W2^T + b2.  ``w`` maps ln_g, ln_b, w1,
+    b1, w2, b2 to fp64 arrays."""
+    h = layernorm(x, w["ln_g"], w["ln_b"], eps)
+    return linear(gelu_tanh(linear(h, w["w1"], w["b1"])), w["w2"], w["b2"])
 
 
 # ------------------------------------------------------------------ merge

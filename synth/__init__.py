@@ -41,7 +41,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "get", "make_inputs", "make_layer_weights",
     "round_bf16_bits", "bf16_bits_to_f64", "to_f64", "from_f64",
-    "grid_tokens", "LAYER_KEYS",
+    "grid_tokens", "LAYER_KEYS", "make_projector_weights",
 ]
 
 LAYER_KEYS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
@@ -222,6 +222,27 @@ def random_tensor(shape, seed: int, dtype: str, scale: float = 1.0) -> np.ndarra
     tests of single steps."""
     rng = np.random.Generator(np.random.PCG64(seed))
     return from_f64(scale * rng.standard_normal(shape), dtype)
+
+
+def make_projector_weights(d_in: int, d_hidden: int, d_out: int, seed: int,
+                           dtype: str) -> Dict[str, np.ndarray]:
+    """Seeded weights of a LayerNorm + two-layer MLP projector (draw order
+    ln_g, ln_b, w1, b1, w2, b2; scales as for the encoder layers:
+    gamma = 1 + N(0, 0.02), beta and biases N(0, 0.01), weights N(0, 0.02))."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    shapes = {"ln_g": (d_in,), "ln_b": (d_in,), "w1": (d_hidden, d_in), "b1": (d_hidden,),
+              "w2": (d_out, d_hidden), "b2": (d_out,)}
+    out = {}
+    for k, shp in shapes.items():
+        z = rng.standard_normal(shp)
+        if k == "ln_g":
+            v = 1.0 + 0.02 * z
+        elif k in ("ln_b", "b1", "b2"):
+            v = 0.01 * z
+        else:
+            v = 0.02 * z
+        out[k] = from_f64(v, dtype)
+    return out
 
 
 @dataclass

@@ -15,8 +15,10 @@ pytestmark = pytest.mark.gpu
 vit = pytest.importorskip("vision_transformer_encoder_layernorm_b200")
 
 
-def _device_run(wl, inputs, n_layers=None, merge=None):
-    """Runs the workload's stack (and merge) on the GPU; returns fp64 numpy."""
+def _device_run(wl, inputs, n_layers=None, merge=None, fold=False):
+    """Runs the workload's stack (and merge) on the GPU; returns fp64 numpy.
+    fold: every layer's LayerNorms folded into the projections after them
+    (vit_fold_layernorm), the path the benchmark times."""
     ctx = context_for(wl)
     T, C = wl.tokens, wl.hidden
     cu_r, pos_r = R.positions_from_grids(wl.grids)
@@ -29,6 +31,8 @@ def _device_run(wl, inputs, n_layers=None, merge=None):
                   pos if wl.rope else None, pkv, wl.prefix_len, wl.prefix_heads)
     n = len(inputs.layers) if n_layers is None else n_layers
     layers = [layer_dev(inputs, i) for i in range(n)]
+    if fold:
+        layers = [ctx.fold_layernorm(lw) for lw in layers]
     ws = torch.empty(ctx.workspace_bytes(T), dtype=torch.uint8, device="cuda")
     y = torch.empty_like(x)
     ctx.encoder_forward(layers, x, y, sq, ws)
@@ -41,6 +45,17 @@ def _device_run(wl, inputs, n_layers=None, merge=None):
     res = from_dev(out)
     ctx.close()
     return res
+
+
+_ORACLE = {}  # workload name -> (inputs, oracle output): each stack oracle runs once
+
+
+def _stack_case(name):
+    if name not in _ORACLE:
+        wl = synth.get(name)
+        inp = synth.make_inputs(wl)
+        _ORACLE[name] = (wl, inp, orun.run_workload(inp))
+    return _ORACLE[name]
 
 
 def test_c0_fp32_layer_and_merge():
@@ -98,12 +113,11 @@ def test_encoder_one_layer_equals_layer_forward():
 
 
 @pytest.mark.slow
-def test_c4_attention_half_layer():
-    wl = synth.get("c4")
-    inp = synth.make_inputs(wl)
-    got = _device_run(wl, inp)
-    ref = orun.run_workload(inp)
-    assert_close(got, ref, 2e-2, 0.9999, "c4 attention half-layer")
+@pytest.mark.parametrize("fold", [False, True], ids=["plain", "folded_ln"])
+def test_c4_attention_half_layer(fold):
+    wl, inp, ref = _stack_case("c4")
+    got = _device_run(wl, inp, fold=fold)
+    assert_close(got, ref, 2e-2, 0.9999, f"c4 attention half-layer (fold {fold})")
 
 
 @pytest.mark.slow
@@ -124,29 +138,28 @@ STACK_REL = 0.1
 
 
 @pytest.mark.slow
-def test_c2_full_stack_and_merge():
-    # the headline workload: 27 layers over 3900 tokens, then the 2x2 merge
-    wl = synth.get("c2")
-    inp = synth.make_inputs(wl)
-    got = _device_run(wl, inp)
-    ref = orun.run_workload(inp)
+@pytest.mark.parametrize("fold", [False, True], ids=["plain", "folded_ln"])
+def test_c2_full_stack_and_merge(fold):
+    # the headline workload: 27 layers over 3900 tokens, then the 2x2 merge;
+    # plain layers, and layers with folded LayerNorms (the benchmark's path)
+    wl, inp, ref = _stack_case("c2")
+    got = _device_run(wl, inp, fold=fold)
     assert got.shape == (975, 4608)
-    rel, cos = assert_close(got, ref, STACK_REL, 0.999, "c2 27-layer stack + merge")
-    print(f"c2 27-layer stack + merge: rel {rel:.4e} cos {cos:.7f}")
+    rel, cos = assert_close(got, ref, STACK_REL, 0.999, f"c2 27-layer stack + merge (fold {fold})")
+    print(f"c2 27-layer stack + merge, fold {fold}: rel {rel:.4e} cos {cos:.7f}")
 
 
 @pytest.mark.slow
-def test_c3_full_packed_stack():
+@pytest.mark.parametrize("fold", [False, True], ids=["plain", "folded_ln"])
+def test_c3_full_packed_stack(fold):
     # 27 layers over 5 packed images (780 + 888 + 960 + 3900 + 4408 tokens):
     # block-diagonal attention through cu_seqlens, per-image RoPE positions
     # and 27 layers of error growth together
-    wl = synth.get("c3")
-    inp = synth.make_inputs(wl)
-    got = _device_run(wl, inp)
-    ref = orun.run_layers(inp)
+    wl, inp, ref = _stack_case("c3")
+    got = _device_run(wl, inp, fold=fold)
     assert got.shape == (10936, 1152)
-    rel, cos = assert_close(got, ref, STACK_REL, 0.999, "c3 27-layer packed stack")
-    print(f"c3 27-layer packed stack: rel {rel:.4e} cos {cos:.7f}")
+    rel, cos = assert_close(got, ref, STACK_REL, 0.999, f"c3 27-layer packed stack (fold {fold})")
+    print(f"c3 27-layer packed stack, fold {fold}: rel {rel:.4e} cos {cos:.7f}")
 
 
 @pytest.mark.parametrize("grid", [(50, 78), (60, 65)])

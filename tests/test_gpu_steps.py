@@ -98,7 +98,10 @@ def test_linear_f32(ctx_f32, epi):
 
 # ------------------------------------------------------------------ LayerNorm
 @pytest.mark.parametrize("rows,cols,dt", [(1000, 1152, "bf16"), (77, 3072, "bf16"),
-                                          (300, 256, "f32"), (5, 4096, "f32")])
+                                          (300, 256, "f32"), (5, 4096, "f32"),
+                                          # rows wider than a warp holds: a block per row
+                                          (975, 4608, "bf16"), (3, 16384, "f32"),
+                                          (7, 4100, "bf16")])
 def test_layernorm(ctx_bf16, ctx_f32, rows, cols, dt):
     ctx = ctx_bf16 if dt == "bf16" else ctx_f32
     _, x, xr = _t((rows, cols), 11, dt, 2.0)

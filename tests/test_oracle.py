@@ -374,6 +374,23 @@ def test_stack_matches_torch_restatement_layer_by_layer(P, attn_only):
     np.testing.assert_allclose(orun.run_layers(inp, n_layers=2), outs[1], atol=1e-11)
 
 
+def test_projector_matches_torch_restatement():
+    # the composition LN -> linear + GELU -> linear against PyTorch's routines,
+    # with ragged widths; and its two closed-form cases
+    w = {k: synth.to_f64(v, "f32") for k, v in
+         synth.make_projector_weights(40, 24, 12, 55, "f32").items()}
+    x = rng(56).standard_normal((7, 40)) * 3.0 + 1.0
+    np.testing.assert_allclose(R.projector(x, w, 1e-6), torch_fp64_layer.projector(x, w, 1e-6),
+                               atol=1e-12)
+    # zero second weight: y = b2 for every row
+    w0 = dict(w, w2=np.zeros_like(w["w2"]))
+    np.testing.assert_allclose(R.projector(x, w0), np.broadcast_to(w["b2"], (7, 12)), atol=0)
+    # a constant row normalises to beta: y = W2 GELU(W1 beta + b1) + b2
+    xc = np.full((1, 40), 2.5)
+    want = R.linear(R.gelu_tanh(R.linear(w["ln_b"][None, :], w["w1"], w["b1"])), w["w2"], w["b2"])
+    np.testing.assert_allclose(R.projector(xc, w), want, atol=1e-12)
+
+
 def test_c1_layer_matches_torch_restatement():
     wl = synth.get("c1")
     inp = synth.make_inputs(wl)

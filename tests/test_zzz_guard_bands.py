@@ -122,6 +122,39 @@ def test_guard_layer_and_workspace():
     c.close()
 
 
+def test_guard_folded_layernorm_layer():
+    # the fold's outputs, and a folded two-layer stack whose row statistics
+    # live in the workspace (written by GEMM epilogues and the row-statistics
+    # kernel)
+    wl = synth.get("c1")
+    inp = synth.make_inputs(wl, layers=1)
+    c = context_for(wl)
+    T, C, Fm = wl.tokens, wl.hidden, wl.mlp
+    lw = layer_dev(inp, 0)
+    wq, sq_ = Band((3 * C, C), torch.bfloat16), Band((2, 3 * C), torch.float32)
+    w1, s1 = Band((Fm, C), torch.bfloat16), Band((2, Fm), torch.float32)
+    import ctypes
+    lws = vit.layer_weights(lw)
+    assert vit.lib.vit_fold_layernorm(c.handle, ctypes.byref(lws), wq.t.data_ptr(), sq_.t.data_ptr(),
+                                      w1.t.data_ptr(), s1.t.data_ptr(), None) == 0
+    for band, what in [(wq, "folded w_qkv"), (sq_, "qkv s, c"), (w1, "folded w_fc1"), (s1, "fc1 s, c")]:
+        band.check(what)
+    f = dict(lw, w_qkv=wq.t, qkv_fold=sq_.t, w_fc1=w1.t, fc1_fold=s1.t, ln1_g=None, ln1_b=None,
+             b_qkv=None, ln2_g=None, ln2_b=None, b_fc1=None)
+    x = to_dev(inp.x, "bf16")
+    cu = torch.empty(len(wl.grids) + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+    c.positions_from_grids(wl.grids, cu, pos)
+    sq = vit.seqs(T, len(wl.grids), max(r * q for r, q in wl.grids), cu, pos)
+    ws = Band((c.workspace_bytes(T),), torch.uint8, poison=False)
+    y = Band((T, C), torch.bfloat16)
+    c.encoder_forward([f, f], x, y.t, sq, ws.t)
+    y.check("folded two-layer encoder output")
+    ws.check("folded encoder workspace")
+    assert c.device_status() == 0
+    c.close()
+
+
 def test_guard_merge_and_positions(ctx):
     grids = [(26, 30), (24, 36), (2, 2)]
     T = sum(r * q for r, q in grids)

@@ -55,3 +55,12 @@ def layer(x, w, cu_seqlens, pos_rc, heads, head_dim, eps, theta,
     h2 = F.layer_norm(x1, (C,), t["ln2_g"], t["ln2_b"], eps)
     g = F.gelu(F.linear(h2, t["w_fc1"], t["b_fc1"]), approximate="tanh")
     return (x1 + F.linear(g, t["w_fc2"], t["b_fc2"])).numpy()
+
+
+def projector(x, w, eps, dtype=torch.float64):
+    # LayerNorm, linear + GELU (tanh), linear, with PyTorch's library routines
+    t = {k: torch.as_tensor(v, dtype=dtype) for k, v in w.items()}
+    x = torch.as_tensor(x, dtype=dtype)
+    h = F.layer_norm(x, (x.shape[1],), t["ln_g"], t["ln_b"], eps)
+    g = F.gelu(F.linear(h, t["w1"], t["b1"]), approximate="tanh")
+    return F.linear(g, t["w2"], t["b2"]).numpy()

@@ -16,7 +16,8 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "lib", "LIB_PATH", "VitError", "VitConfig", "VitLayerWeights", "VitSeqs", "Context",
+    "lib", "LIB_PATH", "VitError", "VitConfig", "VitLayerWeights", "VitProjectorWeights",
+    "VitSeqs", "Context",
     "F32", "BF16", "FLAG_NO_ROPE", "FLAG_NO_MLP", "EPI_BIAS", "EPI_BIAS_GELU",
     "EPI_BIAS_RESIDUAL", "STATUS", "ABI_FUNCTIONS", "KERNEL_KINDS", "Graph",
 ]
@@ -27,7 +28,8 @@ F32, BF16 = 0, 1
 FLAG_NO_ROPE, FLAG_NO_MLP = 0x1, 0x2
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_RESIDUAL = 0, 1, 2
 KERNEL_KINDS = ("layernorm", "gemm_qkv", "rope", "attention", "gemm_out", "gemm_fc1",
-                "gemm_fc2", "merge", "positions", "gemm", "embed", "mx8_quantize", "gemm_mx8")
+                "gemm_fc2", "merge", "positions", "gemm", "embed", "mx8_quantize", "gemm_mx8",
+                "rowstats", "fold")
 STATUS = {0: "VIT_OK", 1: "VIT_ERR_INVALID_ARG", 2: "VIT_ERR_SHAPE", 3: "VIT_ERR_UNSUPPORTED",
           4: "VIT_ERR_WORKSPACE", 5: "VIT_ERR_CUDA", 6: "VIT_ERR_TIMEOUT",
           7: "VIT_ERR_DEVICE_BOUNDS"}
@@ -46,11 +48,15 @@ class VitConfig(ctypes.Structure):
 
 
 _WKEYS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
-          "ln2_g", "ln2_b", "w_fc1", "b_fc1", "w_fc2", "b_fc2")
+          "ln2_g", "ln2_b", "w_fc1", "b_fc1", "w_fc2", "b_fc2", "qkv_fold", "fc1_fold")
 
 
 class VitLayerWeights(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in _WKEYS]
+
+
+class VitProjectorWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("ln_g", "ln_b", "w1", "b1", "w2", "b2")]
 
 
 class VitSeqs(ctypes.Structure):
@@ -67,6 +73,7 @@ ABI_FUNCTIONS = {
     "vit_init": (_I, [ctypes.POINTER(VitConfig), _I, ctypes.POINTER(_P)]),
     "vit_destroy": (None, [_P]),
     "vit_workspace_bytes": (ctypes.c_size_t, [_P, _I]),
+    "vit_fold_layernorm": (_I, [_P, ctypes.POINTER(VitLayerWeights), _P, _P, _P, _P, _P]),
     "vit_layer_forward": (_I, [_P, ctypes.POINTER(VitLayerWeights), _P, _P,
                                ctypes.POINTER(VitSeqs), _P, ctypes.c_size_t, _P]),
     "vit_layer_forward_noalloc": (_I, [_P, ctypes.POINTER(VitLayerWeights), _P, _P,
@@ -83,6 +90,9 @@ ABI_FUNCTIONS = {
     "vit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_longlong),
                               ctypes.POINTER(ctypes.c_double), _I]),
     "vit_embed_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I]),
+    "vit_projector_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I, _I]),
+    "vit_projector": (_I, [_P, ctypes.POINTER(VitProjectorWeights), _P, _P, _I, _I, _I, _I, _P,
+                           ctypes.c_size_t, _P]),
     "vit_patch_embed": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32), _I, _I, _P, _P, _P, _I, _I,
                              _P, _P, ctypes.c_size_t, _P]),
     "vit_pos_interp": (_I, [_P, _P, _I, _I, ctypes.POINTER(ctypes.c_int32), _I, _P, _P]),
@@ -156,9 +166,10 @@ def _grids_arr(grids: Sequence[Sequence[int]]):
 
 
 def layer_weights(d) -> VitLayerWeights:
-    """A VitLayerWeights from a mapping of the 12 parameter names to tensors
-    (missing or None entries become NULL).  The struct keeps the tensors
-    alive: it holds raw device pointers."""
+    """A VitLayerWeights from a mapping of the parameter names (the 12 of a
+    layer, plus qkv_fold / fc1_fold of folded LayerNorms) to tensors (missing
+    or None entries become NULL).  The struct keeps the tensors alive: it
+    holds raw device pointers."""
     lw = VitLayerWeights(*[_ptr(d.get(k)) for k in _WKEYS])
     lw._tensors = dict(d)
     return lw
@@ -226,6 +237,31 @@ class Context:
 
     def workspace_bytes(self, total_tokens: int) -> int:
         return lib.vit_workspace_bytes(self._h, total_tokens)
+
+    def fold_layernorm(self, weights, in_place: bool = False, stream=None):
+        """vit_fold_layernorm: returns a copy of the layer's weight mapping
+        whose w_qkv / w_fc1 are the LayerNorm-folded weights, with the
+        qkv_fold / fc1_fold vectors (new tensors; with in_place the folded
+        weights overwrite w_qkv / w_fc1 of ``weights``)."""
+        import torch
+        w_qkv, w_fc1 = weights["w_qkv"], weights.get("w_fc1")
+        mlp = w_fc1 is not None and not (self.cfg.flags & FLAG_NO_MLP)
+        out = dict(weights)
+        out["w_qkv"] = w_qkv if in_place else torch.empty_like(w_qkv)
+        out["qkv_fold"] = torch.empty((2, w_qkv.shape[0]), dtype=torch.float32,
+                                      device=w_qkv.device)
+        if mlp:
+            out["w_fc1"] = w_fc1 if in_place else torch.empty_like(w_fc1)
+            out["fc1_fold"] = torch.empty((2, w_fc1.shape[0]), dtype=torch.float32,
+                                          device=w_fc1.device)
+        lw = layer_weights(weights)
+        _check("vit_fold_layernorm", lib.vit_fold_layernorm(
+            self._h, ctypes.byref(lw), _ptr(out["w_qkv"]), _ptr(out["qkv_fold"]),
+            _ptr(out.get("w_fc1") if mlp else None), _ptr(out.get("fc1_fold")),
+            _stream(stream)))
+        for k in ("ln1_g", "ln1_b", "b_qkv") + (("ln2_g", "ln2_b", "b_fc1") if mlp else ()):
+            out[k] = None  # not read by a folded layer
+        return out
 
     def layer_forward(self, weights, x, y, sq: VitSeqs, workspace, stream=None):
         lw = layer_weights(weights) if not isinstance(weights, VitLayerWeights) else weights
@@ -300,6 +336,20 @@ class Context:
 
     def profile_enable(self, enable: bool = True):
         _check("vit_profile_enable", lib.vit_profile_enable(self._h, int(bool(enable))))
+
+    def projector_workspace_bytes(self, M: int, d_in: int, d_hidden: int) -> int:
+        return int(lib.vit_projector_workspace_bytes(self._h, M, d_in, d_hidden))
+
+    def projector(self, weights, x, y, workspace, stream=None):
+        """vit_projector: y = GELU(LN(x) W1^T + b1) W2^T + b2; ``weights``
+        maps ln_g, ln_b, w1, b1, w2, b2 to tensors."""
+        M, d_in = x.shape
+        d_hidden, d_out = weights["w1"].shape[0], weights["w2"].shape[0]
+        pw = VitProjectorWeights(*[_ptr(weights.get(k)) for k in
+                                   ("ln_g", "ln_b", "w1", "b1", "w2", "b2")])
+        _check("vit_projector", lib.vit_projector(
+            self._h, ctypes.byref(pw), _ptr(x), _ptr(y), M, d_in, d_hidden, d_out,
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
     def embed_workspace_bytes(self, total_tokens: int, patch: int) -> int:
         return int(lib.vit_embed_workspace_bytes(self._h, total_tokens, patch))

@@ -80,30 +80,81 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 
 }  // namespace gemm
 
-// One 32-column slice of one output row: fp32 accumulators r + bias (from
-// shared memory) -> epilogue op (+ residual rv, already loaded) -> bf16 stores
-// (columns at or past N are skipped; N % 8 == 0).
+// Mean and 1/sqrt(var + eps) of row `row` of a LayerNorm input of K
+// columns, from its slice statistics (Chan's pairwise update, slice order).
+__device__ __forceinline__ void ln_row_stats(const EpiArgs &ea, int row, int K, float &mu,
+                                             float &rstd) {
+  const SliceStats &st = ea.stats_in;
+  const float2 *p = st.p + size_t(row) * st.parts;
+  float n_a = 0.f, mean = 0.f, m2 = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < st.parts; ++j) {
+    const float2 e = __ldg(p + j);
+    const float nb = float(min(st.w, K - j * st.w));
+    const float n = n_a + nb;
+    const float f = nb / n;
+    const float d = e.x - mean;
+    mean = fmaf(d, f, mean);
+    m2 += e.y + d * d * n_a * f;
+    n_a = n;
+  }
+  mu = mean;
+  rstd = 1.0f / sqrtf(m2 / float(K) + ea.ln_eps);
+}
+
+// Running (count, mean, M2) of a row slice, merged chunk by chunk.
+struct RunStats {
+  float n = 0.f, mean = 0.f, m2 = 0.f;
+  __device__ __forceinline__ void merge(float nb, float mb, float m2b) {
+    const float nn = n + nb;
+    const float f = nb / nn;
+    const float d = mb - mean;
+    mean = fmaf(d, f, mean);
+    m2 += m2b + d * d * n * f;
+    n = nn;
+  }
+};
+
+// One 32-column slice of one output row: fp32 accumulators r, then either
+// + bias (from shared memory) or, with the LayerNorm folded in,
+// rstd (r - mu s) + c (s, c already loaded); then the epilogue op (GELU, or
+// + residual rv, already loaded) and bf16 stores (columns at or past N are
+// skipped; N % 8 == 0).  With kEpiStats, adds the stored (rounded) values'
+// mean and M2 to `rs`.
 template <int EPI>
 __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, int col0, int N,
                                             const __nv_bfloat16 *bias_s, const uint4 (&rv)[4],
-                                            __nv_bfloat16 *__restrict__ y) {
+                                            const float4 (&sv)[8], const float4 (&cv)[8], float mu,
+                                            float rstd, __nv_bfloat16 *__restrict__ y,
+                                            RunStats &rs) {
+  constexpr int OP = EPI & kEpiOpMask;
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  const uint4 *bp = reinterpret_cast<const uint4 *>(bias_s);
+  if constexpr ((EPI & kEpiLn) != 0) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 b4 = bp[q];
-    v[8 * q + 0] += bf16_lo(b4.x); v[8 * q + 1] += bf16_hi(b4.x);
-    v[8 * q + 2] += bf16_lo(b4.y); v[8 * q + 3] += bf16_hi(b4.y);
-    v[8 * q + 4] += bf16_lo(b4.z); v[8 * q + 5] += bf16_hi(b4.z);
-    v[8 * q + 6] += bf16_lo(b4.w); v[8 * q + 7] += bf16_hi(b4.w);
+    for (int q = 0; q < 8; ++q) {
+      const float sq[4] = {sv[q].x, sv[q].y, sv[q].z, sv[q].w};
+      const float cq[4] = {cv[q].x, cv[q].y, cv[q].z, cv[q].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[4 * q + e] = fmaf(rstd, fmaf(-mu, sq[e], v[4 * q + e]), cq[e]);
+    }
+  } else {
+    const uint4 *bp = reinterpret_cast<const uint4 *>(bias_s);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 b4 = bp[q];
+      v[8 * q + 0] += bf16_lo(b4.x); v[8 * q + 1] += bf16_hi(b4.x);
+      v[8 * q + 2] += bf16_lo(b4.y); v[8 * q + 3] += bf16_hi(b4.y);
+      v[8 * q + 4] += bf16_lo(b4.z); v[8 * q + 5] += bf16_hi(b4.z);
+      v[8 * q + 6] += bf16_lo(b4.w); v[8 * q + 7] += bf16_hi(b4.w);
+    }
   }
-  if (EPI == kEpiGelu) {
+  if constexpr (OP == kEpiGelu) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gemm::gelu_fast(v[i]);
   }
-  if (EPI == kEpiResidual) {
+  if constexpr (OP == kEpiResidual) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint4 r4 = rv[q];
@@ -114,37 +165,66 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, in
     }
   }
   uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
+  uint4 o[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    if (col0 + 8 * q < N) {
-      uint4 o;
-      o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-      o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-      o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-      o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-      yp[q] = o;
+    o[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    o[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    o[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    o[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    if (col0 + 8 * q < N) yp[q] = o[q];
+  }
+  if constexpr ((EPI & kEpiStats) != 0) {
+    // statistics of the values as stored: the next GEMM multiplies these
+    float w[32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      w[8 * q + 0] = bf16_lo(o[q].x); w[8 * q + 1] = bf16_hi(o[q].x);
+      w[8 * q + 2] = bf16_lo(o[q].y); w[8 * q + 3] = bf16_hi(o[q].y);
+      w[8 * q + 4] = bf16_lo(o[q].z); w[8 * q + 5] = bf16_hi(o[q].z);
+      w[8 * q + 6] = bf16_lo(o[q].w); w[8 * q + 7] = bf16_hi(o[q].w);
     }
+    const int nq = min(4, (N - col0) >> 3);  // valid 8-column groups (>= 1)
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < nq)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum += w[8 * q + e];
+    const float nb = float(8 * nq);
+    const float mb = sum / nb;
+    float m2 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < nq)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float d = w[8 * q + e] - mb;
+          m2 = fmaf(d, d, m2);
+        }
+    rs.merge(nb, mb, m2);
   }
 }
 
 // Epilogue of one accumulator (one output tile) by the 8 epilogue warps:
 // epilogue warp e (= warp - 2) drains TMEM lane quarter (warp & 3), i.e. one
 // row per thread, and column half (e >> 2) of the tile.  The warp's half of
-// the tile bias was staged in its shared-memory slot (bias_w).
+// the tile bias was staged in its shared-memory slot (bias_w).  mu / rstd:
+// the row's LayerNorm statistics (kEpiLn).
 template <int BN, int EPI, int TS = BN>
 __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int lane, int row,
                                               bool row_ok, int n0, int N, const RopeEpi &re,
-                                              const __nv_bfloat16 *bias_w,
-                                              const __nv_bfloat16 *__restrict__ bias,
-                                              const __nv_bfloat16 *__restrict__ res,
-                                              __nv_bfloat16 *__restrict__ y) {
+                                              const __nv_bfloat16 *bias_w, const EpiArgs &ea,
+                                              float mu, float rstd) {
   constexpr int kChunks = BN / 64;  // 32-column chunks per half
+  constexpr int OP = EPI & kEpiOpMask;
   const int quarter = warp & 3, half = (warp - 2) >> 2;
-  if constexpr (EPI == kEpiRope) {
+  __nv_bfloat16 *__restrict__ y = ea.y;
+  if constexpr (OP == kEpiRope) {
     // whole heads: the tile holds HPT heads of HD columns (TS = HPT * HD;
     // the MMA width BN may round TS up); warp `half` of a lane quarter takes
-    // heads half, half + 2, ...: bias, then the 2D rotation of Q/K pairs
-    // (j, j + HD/4) in each half of the head, in fp32
+    // heads half, half + 2, ...: bias (or the folded LayerNorm), then the 2D
+    // rotation of Q/K pairs (j, j + HD/4) in each half of the head, in fp32
     constexpr int HPT = TS == 216 ? 3 : 2, HD = TS / HPT, Q4 = HD / 4, NF = HD / 32;
     static_assert(HPT * HD == TS && TS <= BN, "RoPE tile of whole heads");
 #pragma unroll 1
@@ -165,8 +245,20 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
       const uint32_t bits = i < NF * 32 ? r[i / 32][i % 32] : r8[i - NF * 32];
       v[i] = __uint_as_float(bits);
     }
-    if (bias != nullptr) {  // the head's bias (the same for the whole warp: broadcast loads)
-      const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
+    if constexpr ((EPI & kEpiLn) != 0) {
+      // the head's s and c (the same for the whole warp: broadcast loads)
+      const float4 *sp = reinterpret_cast<const float4 *>(ea.ln_sc + col0);
+      const float4 *cp = reinterpret_cast<const float4 *>(ea.ln_sc + N + col0);
+#pragma unroll
+      for (int u = 0; u < HD / 4; ++u) {
+        const float4 s4 = __ldg(sp + u), c4 = __ldg(cp + u);
+        v[4 * u + 0] = fmaf(rstd, fmaf(-mu, s4.x, v[4 * u + 0]), c4.x);
+        v[4 * u + 1] = fmaf(rstd, fmaf(-mu, s4.y, v[4 * u + 1]), c4.y);
+        v[4 * u + 2] = fmaf(rstd, fmaf(-mu, s4.z, v[4 * u + 2]), c4.z);
+        v[4 * u + 3] = fmaf(rstd, fmaf(-mu, s4.w, v[4 * u + 3]), c4.w);
+      }
+    } else if (ea.bias != nullptr) {  // the head's bias (broadcast loads)
+      const uint4 *bp = reinterpret_cast<const uint4 *>(ea.bias + col0);
 #pragma unroll
       for (int u = 0; u < HD / 8; ++u) {
         const uint4 b4 = __ldg(bp + u);
@@ -205,6 +297,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
     }
     }
   } else {
+  RunStats rs;
 #pragma unroll 1
   for (int i = 0; i < kChunks; ++i) {
     const int c = half * kChunks + i;
@@ -213,14 +306,32 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
     uint32_t r[32];
     __syncwarp();
     tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c * 32), r);
+    // operands of the epilogue, in flight together with the TMEM load
     uint4 rv[4];
-    if (EPI == kEpiResidual && ok) {  // in flight together with the TMEM load
-      const uint4 *rp = reinterpret_cast<const uint4 *>(res + size_t(row) * N + col0);
+    if (OP == kEpiResidual && ok) {
+      const uint4 *rp = reinterpret_cast<const uint4 *>(ea.res + size_t(row) * N + col0);
 #pragma unroll
       for (int q = 0; q < 4; ++q) rv[q] = (col0 + 8 * q < N) ? __ldg(rp + q) : make_uint4(0, 0, 0, 0);
     }
+    float4 sv[8], cv[8];
+    if ((EPI & kEpiLn) && ok) {
+      const float4 *sp = reinterpret_cast<const float4 *>(ea.ln_sc + col0);
+      const float4 *cp = reinterpret_cast<const float4 *>(ea.ln_sc + N + col0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const bool in = col0 + 4 * q < N;
+        sv[q] = in ? __ldg(sp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cv[q] = in ? __ldg(cp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
     tmem_ld_wait();
-    if (ok) store_chunk<EPI>(r, row, col0, N, bias_w + i * 32, rv, y);
+    if (ok) store_chunk<EPI>(r, row, col0, N, bias_w + i * 32, rv, sv, cv, mu, rstd, y, rs);
+  }
+  if constexpr ((EPI & kEpiStats) != 0) {
+    // this warp's slice of the row: columns [n0 + half BN/2, + BN/2)
+    const int c0 = n0 + half * (BN / 2);
+    if (row_ok && c0 < N)
+      ea.stats_out.p[size_t(row) * ea.stats_out.parts + c0 / (BN / 2)] = make_float2(rs.mean, rs.m2);
   }
   }
 }
@@ -247,8 +358,7 @@ __device__ __forceinline__ void stage_bias_warp(__nv_bfloat16 *bias_w, const __n
 template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
-                   __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status,
+                   const __grid_constant__ EpiArgs ea, int M, int N, int K, int *status,
                    const __grid_constant__ RopeEpi re, uint32_t lost_tx) {
   using namespace gemm;
   using CF = Cfg<BN>;
@@ -367,12 +477,17 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      stage_bias_warp<BN>(bias_w, bias, nb * BN, N, warp, lane);
+      const int row = mb * BM + row_in_tile;
+      float mu = 0.f, rstd = 0.f;  // LayerNorm statistics of the row (kEpiLn)
+      if constexpr ((EPI & kEpiLn) != 0) {
+        if (row < M) ln_row_stats(ea, row, K, mu, rstd);
+      } else {
+        stage_bias_warp<BN>(bias_w, ea.bias, nb * BN, N, warp, lane);
+      }
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
-      const int row = mb * BM + row_in_tile;
       epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, re,
-                             bias_w, bias, res, y);
+                             bias_w, ea, mu, rstd);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
@@ -417,9 +532,8 @@ struct Cfg2 {
 template <int BN, int EPI, int TS = BN>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
-                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status,
-                   const __grid_constant__ RopeEpi re) {
+                    const __grid_constant__ EpiArgs ea, int M, int N, int K, int *status,
+                    const __grid_constant__ RopeEpi re) {
   using namespace gemm;
   using CF = Cfg2<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -545,12 +659,17 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (EPI != kEpiRope) stage_bias_warp<BN>(bias_w, bias, nb * TS, N, warp, lane);
+      const int row = mb * 2 * BM + row_in_tile;
+      float mu = 0.f, rstd = 0.f;  // LayerNorm statistics of the row (kEpiLn)
+      if constexpr ((EPI & kEpiLn) != 0) {
+        if (row < M) ln_row_stats(ea, row, K, mu, rstd);
+      } else if constexpr ((EPI & kEpiOpMask) != kEpiRope) {
+        stage_bias_warp<BN>(bias_w, ea.bias, nb * TS, N, warp, lane);
+      }
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
-      const int row = mb * 2 * BM + row_in_tile;
       epilogue_tile<BN, EPI, TS>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * TS, N, re,
-                                 bias_w, bias, res, y);
+                                 bias_w, ea, mu, rstd);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_cta(&bars->acc_empty[a], 0));
@@ -598,10 +717,9 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const vo
 }
 
 template <int BN, int EPI>
-static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
-                             const void *res, void *y, int M, int N, int K, int num_sms,
-                             int *status, cudaStream_t st, const RopeEpi &re,
-                             uint32_t lost_tx) {
+static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const EpiArgs &ea,
+                             int M, int N, int K, int num_sms, int *status, cudaStream_t st,
+                             const RopeEpi &re, uint32_t lost_tx) {
   using CF = gemm::Cfg<BN>;
   auto kern = gemm_tc_kernel<BN, EPI>;
   cudaError_t e =
@@ -609,32 +727,42 @@ static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const
   if (e != cudaSuccess) return e;
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + BN - 1) / BN);
   const int grid = std::max(1, std::min(tiles, num_sms));
-  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb,
-                    static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-                    static_cast<__nv_bfloat16 *>(y), M, N, K, status, re, lost_tx);
+  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb, ea, M,
+                    N, K, status, re, lost_tx);
 }
 
+// the epilogue combinations the library launches: plain bias, GELU and
+// residual; LayerNorm folded into bias or GELU; residual with row statistics
 template <int BN>
 static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
-                              const void *b, const void *res, void *y, int M, int N, int K,
-                              int num_sms, int *status, cudaStream_t st, uint32_t lost_tx) {
+                              const EpiArgs &ea, int M, int N, int K, int num_sms, int *status,
+                              cudaStream_t st, uint32_t lost_tx) {
+  const RopeEpi none{};
   switch (epi) {
+    case kEpiBias:
+      return launch_bn<BN, kEpiBias>(ta, tb, ea, M, N, K, num_sms, status, st, none, lost_tx);
     case kEpiGelu:
-      return launch_bn<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{},
-                                     lost_tx);
+      return launch_bn<BN, kEpiGelu>(ta, tb, ea, M, N, K, num_sms, status, st, none, lost_tx);
     case kEpiResidual:
-      return launch_bn<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st,
-                                         RopeEpi{}, lost_tx);
+      return launch_bn<BN, kEpiResidual>(ta, tb, ea, M, N, K, num_sms, status, st, none, lost_tx);
+    case kEpiBias | kEpiLn:
+      return launch_bn<BN, kEpiBias | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none,
+                                              lost_tx);
+    case kEpiGelu | kEpiLn:
+      return launch_bn<BN, kEpiGelu | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none,
+                                              lost_tx);
+    case kEpiResidual | kEpiStats:
+      return launch_bn<BN, kEpiResidual | kEpiStats>(ta, tb, ea, M, N, K, num_sms, status, st,
+                                                     none, lost_tx);
     default:
-      return launch_bn<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st, RopeEpi{},
-                                     lost_tx);
+      return cudaErrorInvalidValue;
   }
 }
 
 template <int BN, int EPI, int TS = BN>
-static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const void *b,
-                               const void *res, void *y, int M, int N, int K, int num_sms,
-                               int *status, cudaStream_t st, const RopeEpi &re) {
+static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const EpiArgs &ea,
+                               int M, int N, int K, int num_sms, int *status, cudaStream_t st,
+                               const RopeEpi &re) {
   using CF = gemm::Cfg2<BN>;
   auto kern = gemm_tc2_kernel<BN, EPI, TS>;
   cudaError_t e =
@@ -670,23 +798,30 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
   }
   const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + TS - 1) / TS);
   return launch_pdl(kern, dim3(2 * std::max(1, std::min(tiles, max_clusters))),
-                    dim3(gemm::kThreads), CF::kSmemBytes, st, 2, ta, tb,
-                    static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-                    static_cast<__nv_bfloat16 *>(y), M, N, K, status, re);
+                    dim3(gemm::kThreads), CF::kSmemBytes, st, 2, ta, tb, ea, M, N, K, status, re);
 }
 
 template <int BN>
 static cudaError_t launch_pair_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
-                                   const void *b, const void *res, void *y, int M, int N, int K,
-                                   int num_sms, int *status, cudaStream_t st) {
+                                   const EpiArgs &ea, int M, int N, int K, int num_sms,
+                                   int *status, cudaStream_t st) {
   const RopeEpi none{};
   switch (epi) {
+    case kEpiBias:
+      return launch_pair<BN, kEpiBias>(ta, tb, ea, M, N, K, num_sms, status, st, none);
     case kEpiGelu:
-      return launch_pair<BN, kEpiGelu>(ta, tb, b, res, y, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiGelu>(ta, tb, ea, M, N, K, num_sms, status, st, none);
     case kEpiResidual:
-      return launch_pair<BN, kEpiResidual>(ta, tb, b, res, y, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiResidual>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+    case kEpiBias | kEpiLn:
+      return launch_pair<BN, kEpiBias | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+    case kEpiGelu | kEpiLn:
+      return launch_pair<BN, kEpiGelu | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+    case kEpiResidual | kEpiStats:
+      return launch_pair<BN, kEpiResidual | kEpiStats>(ta, tb, ea, M, N, K, num_sms, status, st,
+                                                       none);
     default:
-      return launch_pair<BN, kEpiBias>(ta, tb, b, res, y, M, N, K, num_sms, status, st, none);
+      return cudaErrorInvalidValue;
   }
 }
 
@@ -726,15 +861,27 @@ static GemmVariant choose_variant(int M, int N, int K, int num_sms) {
   return pick;
 }
 
-cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
-                           int M, int N, int K, int epi, int num_sms, int *status,
-                           cudaStream_t st, const RopeEpi *rope, uint32_t lost_tx) {
+int gemm_stats_width(int M, int N, int K, int num_sms) {
+  return choose_variant(M, N, K, num_sms).bn / 2;
+}
+
+cudaError_t launch_gemm_tc(const void *x, const void *w, const EpiArgs &ea, int M, int N, int K,
+                           int epi, int num_sms, cudaStream_t st, int *status,
+                           const RopeEpi *rope, uint32_t lost_tx) {
   if (M == 0 || N == 0) return cudaSuccess;
   GemmVariant v = choose_variant(M, N, K, num_sms);
-  if (epi == kEpiRope) {  // tiles of whole heads on a CTA pair: 3 x 72 (MMA N = 224) or 2 x 128
-    if (rope == nullptr || (rope->head_dim != 72 && rope->head_dim != 128)) return cudaErrorInvalidValue;
+  const int op = epi & kEpiOpMask;
+  if (op == kEpiRope) {  // tiles of whole heads on a CTA pair: 3 x 72 (MMA N = 224) or 2 x 128
+    if (rope == nullptr || (rope->head_dim != 72 && rope->head_dim != 128) || (epi & kEpiStats))
+      return cudaErrorInvalidValue;
     v = {2, rope->head_dim == 72 ? 224 : 256};
   }
+  if ((epi & kEpiStats) && (ea.stats_out.p == nullptr || ea.stats_out.w != v.bn / 2 ||
+                            ea.stats_out.parts != (N + v.bn / 2 - 1) / (v.bn / 2)))
+    return cudaErrorInvalidValue;
+  if ((epi & kEpiLn) && (ea.ln_sc == nullptr || ea.stats_in.p == nullptr || ea.stats_in.w <= 0 ||
+                         ea.stats_in.parts != (K + ea.stats_in.w - 1) / ea.stats_in.w))
+    return cudaErrorInvalidValue;
   const int b_rows = v.pair == 2 ? v.bn / 2 : v.bn;
   CUtensorMap ta, tb;
   if (encode_tensor_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, uint64_t(K) * 2,
@@ -743,19 +890,24 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const vo
   if (encode_tensor_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, uint64_t(K) * 2,
                            gemm::BK, b_rows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  if (epi == kEpiRope) {
+  if (op == kEpiRope) {
+    const bool ln = (epi & kEpiLn) != 0;
     if (v.bn == 224)
-      return launch_pair<224, kEpiRope, 216>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
-    return launch_pair<256, kEpiRope, 256>(ta, tb, b, res, y, M, N, K, num_sms, status, st, *rope);
+      return ln ? launch_pair<224, kEpiRope | kEpiLn, 216>(ta, tb, ea, M, N, K, num_sms, status, st,
+                                                           *rope)
+                : launch_pair<224, kEpiRope, 216>(ta, tb, ea, M, N, K, num_sms, status, st, *rope);
+    return ln ? launch_pair<256, kEpiRope | kEpiLn, 256>(ta, tb, ea, M, N, K, num_sms, status, st,
+                                                         *rope)
+              : launch_pair<256, kEpiRope, 256>(ta, tb, ea, M, N, K, num_sms, status, st, *rope);
   }
   if (v.pair == 2) {
-    if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
-    if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
-    return launch_pair_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st);
+    if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, ea, M, N, K, num_sms, status, st);
+    if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, ea, M, N, K, num_sms, status, st);
+    return launch_pair_epi<128>(epi, ta, tb, ea, M, N, K, num_sms, status, st);
   }
   if (v.bn == 256)
-    return launch_epi<256>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st, lost_tx);
-  return launch_epi<128>(epi, ta, tb, b, res, y, M, N, K, num_sms, status, st, lost_tx);
+    return launch_epi<256>(epi, ta, tb, ea, M, N, K, num_sms, status, st, lost_tx);
+  return launch_epi<128>(epi, ta, tb, ea, M, N, K, num_sms, status, st, lost_tx);
 }
 
 // ---------------------------------------------------------------- MXFP8 GEMM
@@ -793,8 +945,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfb,
-                    const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ res,
-                    __nv_bfloat16 *__restrict__ y, int M, int N, int K, int *status) {
+                    const __grid_constant__ EpiArgs ea, int M, int N, int K, int *status) {
   using namespace gemm;
   using CF = CfgMx<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -922,12 +1073,12 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      stage_bias_warp<BN>(bias_w, bias, nb * BN, N, warp, lane);
+      stage_bias_warp<BN>(bias_w, ea.bias, nb * BN, N, warp, lane);
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * BM + row_in_tile;
       epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, none,
-                             bias_w, bias, res, y);
+                             bias_w, ea, 0.f, 0.f);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
@@ -945,8 +1096,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 
 template <int BN, int EPI>
 static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb, const uint8_t *sfa,
-                                 const uint8_t *sfb, const void *b, const void *res, void *y, int M,
-                                 int N, int K, int num_sms, int *status, cudaStream_t st) {
+                                 const uint8_t *sfb, const EpiArgs &ea, int M, int N, int K,
+                                 int num_sms, int *status, cudaStream_t st) {
   using CF = gemm::CfgMx<BN>;
   auto kern = gemm_mx8_kernel<BN, EPI>;
   cudaError_t e =
@@ -955,8 +1106,7 @@ static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb, c
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + BN - 1) / BN);
   const int grid = std::max(1, std::min(tiles, num_sms));
   return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb, sfa, sfb,
-                    static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(res),
-                    static_cast<__nv_bfloat16 *>(y), M, N, K, status);
+                    ea, M, N, K, status);
 }
 
 cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes,
@@ -971,16 +1121,20 @@ cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, con
   if (encode_tensor_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K, N, mx8_row_bytes(K),
                            gemm::kMxBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  EpiArgs ea{};
+  ea.bias = static_cast<const __nv_bfloat16 *>(b);
+  ea.res = static_cast<const __nv_bfloat16 *>(res);
+  ea.y = static_cast<__nv_bfloat16 *>(y);
   switch (epi) {
     case kEpiGelu:
-      return launch_mx8_bn<BN, kEpiGelu>(ta, tb, a_scales, w_scales, b, res, y, M, N, K, num_sms,
-                                         status, st);
+      return launch_mx8_bn<BN, kEpiGelu>(ta, tb, a_scales, w_scales, ea, M, N, K, num_sms, status,
+                                         st);
     case kEpiResidual:
-      return launch_mx8_bn<BN, kEpiResidual>(ta, tb, a_scales, w_scales, b, res, y, M, N, K,
-                                             num_sms, status, st);
+      return launch_mx8_bn<BN, kEpiResidual>(ta, tb, a_scales, w_scales, ea, M, N, K, num_sms,
+                                             status, st);
     default:
-      return launch_mx8_bn<BN, kEpiBias>(ta, tb, a_scales, w_scales, b, res, y, M, N, K, num_sms,
-                                         status, st);
+      return launch_mx8_bn<BN, kEpiBias>(ta, tb, a_scales, w_scales, ea, M, N, K, num_sms, status,
+                                         st);
   }
 }
 

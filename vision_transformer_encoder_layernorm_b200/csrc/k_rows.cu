@@ -106,10 +106,91 @@ __global__ void __launch_bounds__(256) layernorm_warp_kernel(
   }
 }
 
+// Rows wider than a warp holds (cols > 4096, e.g. the 4C = 4608 columns of
+// merged tokens): one block of 256 threads per row, thread t holding the
+// 4-element vectors t, t + 256, ... (MAXV at most); the mean, then the
+// centred variance, are reduced over the block (warp shuffles, then the 8
+// warp partials through shared memory, summed in a fixed order).
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(256) layernorm_block_kernel(
+    const T *__restrict__ x, T *__restrict__ y, const T *__restrict__ gamma,
+    const T *__restrict__ beta, int rows, int cols, float eps) {
+  using V = Vec4<T>;
+  using R = typename V::raw;
+  __shared__ float red[2][8];
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvec = cols >> 2;
+  const R *xr = reinterpret_cast<const R *>(x + size_t(row) * cols);
+  float v[MAXV][4];
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = threadIdx.x + 256 * i;
+    if (c < nvec) {
+      V::unpack(xr[c], v[i]);
+    } else {
+      v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.f;
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[0][warp] = s;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[0][w];
+  const float mean = tot / float(cols);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    if (threadIdx.x + 256 * i < nvec) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d = v[i][e] - mean;
+        q = fmaf(d, d, q);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  if (lane == 0) red[1][warp] = q;
+  __syncthreads();
+  float qt = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) qt += red[1][w];
+  const float rstd = 1.0f / sqrtf(qt / float(cols) + eps);
+  R *yr = reinterpret_cast<R *>(y + size_t(row) * cols);
+  const R *gr = reinterpret_cast<const R *>(gamma);
+  const R *br = reinterpret_cast<const R *>(beta);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = threadIdx.x + 256 * i;
+    if (c < nvec) {
+      float g[4], b[4], o[4];
+      V::unpack(__ldg(gr + c), g);
+      V::unpack(__ldg(br + c), b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = (v[i][e] - mean) * rstd * g[e] + b[e];
+      yr[c] = V::pack(o);
+    }
+  }
+}
+
 template <typename T>
 cudaError_t launch_layernorm_t(const void *x, void *y, const void *g, const void *b, int rows,
                                int cols, float eps, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (cols > 4096) {  // a block per row (cols <= 16384, checked by the caller)
+    auto k = layernorm_block_kernel<T, 16>;
+    return launch_pdl(k, dim3(rows), dim3(256), 0, st, 1, static_cast<const T *>(x),
+                      static_cast<T *>(y), static_cast<const T *>(g), static_cast<const T *>(b),
+                      rows, cols, eps);
+  }
   const int warps = 8;
   dim3 grid((rows + warps - 1) / warps), block(32 * warps);
   const int nvec = cols / 4;
@@ -137,57 +218,199 @@ cudaError_t launch_layernorm(int dtype, const void *x, void *y, const void *g, c
                        : launch_layernorm_t<__nv_bfloat16>(x, y, g, b, rows, cols, eps, st);
 }
 
+// ---------------------------------------------------------------- LayerNorm folded into a GEMM
+// With the LayerNorm folded into the projection that follows it, the
+// projection reads the raw row x and forms
+//   LN(x) w^T + b = rstd (x w'^T - mean s) + c,
+//   w' = w diag(gamma), s_n = sum_k w'_nk, c = b + w beta,
+// so only the row's mean and rstd are needed, as slice statistics: these
+// come from the epilogue of the GEMM that wrote x (kEpiStats), or, for a
+// stack's input, from this kernel.
+
+// Row statistics of x [rows, cols] (bf16) in slices of kRowStatsWidth = 64
+// columns: (mean, sum of squared deviations) per slice.  One warp per row;
+// lane l holds 4-element vectors l, l + 32, ... (vector c = columns
+// [4c, 4c + 4)), so for a fixed i lanes 0-15 hold slice 2i and lanes 16-31
+// slice 2i + 1; each half-warp reduces its slice with shuffles, two passes
+// over the registers.
+template <int MAXV>
+__global__ void __launch_bounds__(256) rowstats_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                       float2 *__restrict__ out, int rows,
+                                                       int cols) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;  // whole warps only
+  const int nvec = cols >> 2, parts = (cols + kRowStatsWidth - 1) / kRowStatsWidth;
+  const uint2 *xr = reinterpret_cast<const uint2 *>(x + size_t(row) * cols);
+  float v[MAXV][4];
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nvec) {
+      const uint2 r = xr[c];
+      v[i][0] = bf16_lo(r.x); v[i][1] = bf16_hi(r.x); v[i][2] = bf16_lo(r.y); v[i][3] = bf16_hi(r.y);
+    } else {
+      v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    const int j = 2 * i + (lane >> 4);  // this half-warp's slice
+    const int n = min(kRowStatsWidth, cols - j * kRowStatsWidth);  // <= 0: past the row
+    float s = (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
+#pragma unroll
+    for (int o = 8; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / float(max(n, 1));
+    float q = 0.f;
+    if (c < nvec) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d = v[i][e] - mean;
+        q = fmaf(d, d, q);
+      }
+    }
+#pragma unroll
+    for (int o = 8; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if ((lane & 15) == 0 && n > 0) out[size_t(row) * parts + j] = make_float2(mean, q);
+  }
+}
+
+cudaError_t launch_rowstats(const void *x, float2 *out, int rows, int cols, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  const int warps = 8;
+  dim3 grid((rows + warps - 1) / warps), block(32 * warps);
+  const int nvec = cols / 4;
+  auto xp = static_cast<const __nv_bfloat16 *>(x);
+  if (nvec <= 32 * 4) return launch_pdl(rowstats_kernel<4>, grid, block, 0, st, 1, xp, out, rows, cols);
+  if (nvec <= 32 * 9) return launch_pdl(rowstats_kernel<9>, grid, block, 0, st, 1, xp, out, rows, cols);
+  if (nvec <= 32 * 12) return launch_pdl(rowstats_kernel<12>, grid, block, 0, st, 1, xp, out, rows, cols);
+  if (nvec <= 32 * 24) return launch_pdl(rowstats_kernel<24>, grid, block, 0, st, 1, xp, out, rows, cols);
+  return launch_pdl(rowstats_kernel<32>, grid, block, 0, st, 1, xp, out, rows, cols);
+}
+
+// The folded weight and its vectors, one warp per output row n, 8 columns
+// per lane step: w_out = bf16(w * gamma) (a product of two bf16 values is
+// exact in fp32, so this is a single rounding), s = sum of w_out as stored,
+// c = b + sum_k w * beta, both accumulated in fp32 and reduced in a fixed
+// shuffle order.  w_out may be w itself: each element is read before the
+// same thread overwrites it.
+__global__ void __launch_bounds__(256) fold_ln_kernel(
+    const __nv_bfloat16 *w, const __nv_bfloat16 *__restrict__ gamma,
+    const __nv_bfloat16 *__restrict__ beta, const __nv_bfloat16 *__restrict__ b,
+    __nv_bfloat16 *w_out, float *__restrict__ sc, int n, int k) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= n) return;
+  const uint4 *wr = reinterpret_cast<const uint4 *>(w + size_t(row) * k);
+  uint4 *wo = reinterpret_cast<uint4 *>(w_out + size_t(row) * k);
+  const uint4 *gr = reinterpret_cast<const uint4 *>(gamma);
+  const uint4 *br = reinterpret_cast<const uint4 *>(beta);
+  float s = 0.f, c = 0.f;
+  for (int u = lane; u < k / 8; u += 32) {
+    const uint4 wv = wr[u], gv = __ldg(gr + u), bv = __ldg(br + u);
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+    const uint32_t gg[4] = {gv.x, gv.y, gv.z, gv.w};
+    const uint32_t bb[4] = {bv.x, bv.y, bv.z, bv.w};
+    uint32_t oo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float w0 = bf16_lo(ww[e]), w1 = bf16_hi(ww[e]);
+      oo[e] = pack_bf16x2(w0 * bf16_lo(gg[e]), w1 * bf16_hi(gg[e]));
+      s += bf16_lo(oo[e]) + bf16_hi(oo[e]);
+      c = fmaf(w0, bf16_lo(bb[e]), c);
+      c = fmaf(w1, bf16_hi(bb[e]), c);
+    }
+    wo[u] = make_uint4(oo[0], oo[1], oo[2], oo[3]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (lane == 0) {
+    sc[row] = s;
+    sc[n + row] = c + (b != nullptr ? __bfloat162float(b[row]) : 0.f);
+  }
+}
+
+cudaError_t launch_fold_ln(const void *w, const void *gamma, const void *beta, const void *b,
+                           void *w_out, float *sc, int n, int k, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int warps = 8;
+  return launch_pdl(fold_ln_kernel, dim3((n + warps - 1) / warps), dim3(32 * warps), 0, st, 1,
+                    static_cast<const __nv_bfloat16 *>(w), static_cast<const __nv_bfloat16 *>(gamma),
+                    static_cast<const __nv_bfloat16 *>(beta), static_cast<const __nv_bfloat16 *>(b),
+                    static_cast<__nv_bfloat16 *>(w_out), sc, n, k);
+}
+
 // ---------------------------------------------------------------- 2x2 merge
-// One thread copies one 16-byte unit (or one element-sized unit when the
-// token row is not a multiple of 16 bytes).  blockIdx.y = image.
+// One warp builds one merged token: the four source tokens' rows (each
+// `units_per_token` units of U: 16 bytes, or 4 / 2 bytes when the row is
+// not a multiple of 16 bytes) are concatenated in window order.  A lane
+// issues up to kMergeBatch loads before its stores, so each warp keeps
+// several kilobytes in flight; the index arithmetic is done once per token.
+// blockIdx.y = image, blockIdx.x * warps + warp = merged token of the image.
+constexpr int kMergeBatch = 16;
+
 template <typename U>
-__global__ void merge2x2_kernel(const __grid_constant__ ImageTable tab, const U *__restrict__ x,
-                                U *__restrict__ y, int units_per_token) {
+__global__ void __launch_bounds__(128) merge2x2_kernel(const __grid_constant__ ImageTable tab,
+                                                       const U *__restrict__ x,
+                                                       U *__restrict__ y, int units_per_token) {
   pdl_trigger();
   pdl_wait();
   const ImageEntry im = tab.img[blockIdx.y];
   const int half_w = im.cols >> 1;
-  const long long out_tokens = (long long)(im.rows >> 1) * half_w;
-  const long long total = out_tokens * 4 * units_per_token;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long o = i / (4 * units_per_token);
-    const int rem = int(i - o * 4 * units_per_token);
-    const int part = rem / units_per_token;  // 0 TL, 1 TR, 2 BL, 3 BR
-    const int u = rem - part * units_per_token;
-    const int R = int(o / half_w), Q = int(o - (long long)R * half_w);
-    const long long src_tok =
-        im.base + (long long)(2 * R + (part >> 1)) * im.cols + (2 * Q + (part & 1));
-    const long long dst_tok = im.base / 4 + o;
-    y[dst_tok * 4 * units_per_token + part * units_per_token + u] =
-        x[src_tok * units_per_token + u];
+  const int out_tokens = (im.rows >> 1) * half_w;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int o = blockIdx.x * (blockDim.x >> 5) + warp; o < out_tokens;
+       o += gridDim.x * (blockDim.x >> 5)) {
+    const int R = o / half_w, Q = o - R * half_w;
+    const long long top = im.base + (long long)(2 * R) * im.cols + 2 * Q;  // top-left source token
+    // source token of window part p: top + (p >> 1) * cols + (p & 1)
+    U *dst = y + ((long long)(im.base / 4) + o) * 4 * units_per_token;
+    const int n = 4 * units_per_token;
+    // flattened unit i = part * units_per_token + u, walked 32 at a time
+    int part = 0, u = lane;
+    while (part < 4 && u >= units_per_token) { u -= units_per_token; ++part; }
+    for (int i0 = lane; i0 < n; i0 += 32 * kMergeBatch) {
+      U v[kMergeBatch];
+      int pk[kMergeBatch], uk[kMergeBatch];
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k) {
+        pk[k] = part;
+        uk[k] = u;
+        if (part < 4)
+          v[k] = x[(top + (long long)(part >> 1) * im.cols + (part & 1)) * units_per_token + u];
+        u += 32;
+        while (part < 4 && u >= units_per_token) { u -= units_per_token; ++part; }
+      }
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k)
+        if (pk[k] < 4) dst[pk[k] * units_per_token + uk[k]] = v[k];
+    }
   }
 }
 
 cudaError_t launch_merge2x2(const ImageTable &tab, int n_images, const void *x, void *y,
                             size_t row_bytes, long long max_out_tokens, cudaStream_t st) {
   if (n_images == 0 || max_out_tokens == 0) return cudaSuccess;
-  const int threads = 256;
-  if (row_bytes % 16 == 0) {
-    const int upt = int(row_bytes / 16);
-    long long units = max_out_tokens * 4 * upt;
-    int bx = int(std::min<long long>((units + threads - 1) / threads, 4096));
+  const int threads = 128, warps = threads / 32;
+  const int bx = int(std::min<long long>((max_out_tokens + warps - 1) / warps, 65535));
+  if (row_bytes % 16 == 0)
     return launch_pdl(merge2x2_kernel<uint4>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
-                      static_cast<const uint4 *>(x), static_cast<uint4 *>(y), upt);
-  } else if (row_bytes % 4 == 0) {
-    const int upt = int(row_bytes / 4);
-    long long units = max_out_tokens * 4 * upt;
-    int bx = int(std::min<long long>((units + threads - 1) / threads, 4096));
+                      static_cast<const uint4 *>(x), static_cast<uint4 *>(y), int(row_bytes / 16));
+  if (row_bytes % 4 == 0)
     return launch_pdl(merge2x2_kernel<uint32_t>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
-                      static_cast<const uint32_t *>(x), static_cast<uint32_t *>(y), upt);
-  } else {
-    const int upt = int(row_bytes / 2);
-    long long units = max_out_tokens * 4 * upt;
-    int bx = int(std::min<long long>((units + threads - 1) / threads, 4096));
-    return launch_pdl(merge2x2_kernel<uint16_t>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
-                      static_cast<const uint16_t *>(x), static_cast<uint16_t *>(y), upt);
-  }
-  return cudaGetLastError();
+                      static_cast<const uint32_t *>(x), static_cast<uint32_t *>(y),
+                      int(row_bytes / 4));
+  return launch_pdl(merge2x2_kernel<uint16_t>, dim3(bx, n_images), dim3(threads), 0, st, 1, tab,
+                    static_cast<const uint16_t *>(x), static_cast<uint16_t *>(y),
+                    int(row_bytes / 2));
 }
 
 // ---------------------------------------------------------------- positions

@@ -62,11 +62,45 @@ cudaError_t launch_pad_cols(int dtype, const void *w, void *out, int n, int k, i
 cudaError_t launch_pos_interp(int dtype, const ImageTable &tab, int n_images, long long max_tokens,
                               const void *table, int gh, int gw, int C, void *y, cudaStream_t st);
 
-// Epilogue codes (match vit_epilogue)
+// Epilogue codes: an operation (the low two bits; 0-2 match vit_epilogue)
+// and two flags.
 constexpr int kEpiBias = 0;
 constexpr int kEpiGelu = 1;
 constexpr int kEpiResidual = 2;
 constexpr int kEpiRope = 3;  // bias, then 2D RoPE on columns < rot_cols (QKV projection)
+constexpr int kEpiOpMask = 3;
+// LayerNorm folded into this GEMM: A is the raw row x (length K), the weight
+// was folded to w' = w diag(gamma), and the epilogue forms
+// rstd (acc - mean s) + c in place of acc + bias (see EpiArgs).
+constexpr int kEpiLn = 4;
+// The output rows' statistics, per slice of the columns one epilogue warp
+// writes, go to EpiArgs::stats_out (for a later kEpiLn GEMM on this output).
+constexpr int kEpiStats = 8;
+
+// Per-row statistics of a row's column slices: slice j covers columns
+// [j w, min((j + 1) w, n)); entry (mean, M2) = mean of the slice and the sum
+// of squared deviations from it.  A row's slices merge (Chan's pairwise
+// update) into the row's mean and biased variance M2 / n.
+struct SliceStats {
+  float2 *p;   // [rows][parts]
+  int parts;   // ceil(n / w)
+  int w;       // slice width (columns)
+};
+
+// Epilogue operands of the tensor-core GEMMs (passed by value, __grid_constant__).
+struct EpiArgs {
+  const __nv_bfloat16 *bias;  // [N] or null; not read with kEpiLn
+  const __nv_bfloat16 *res;   // [M, N] residual (kEpiResidual)
+  __nv_bfloat16 *y;           // [M, N] output
+  // kEpiLn: fp32 [2][N]: s = row sums of the folded weight, c = b + w beta;
+  // stats_in: slice statistics of the rows of A (row length K)
+  const float *ln_sc;
+  SliceStats stats_in;
+  float ln_eps;
+  // kEpiStats: slice statistics of the (bf16-rounded) output rows, slice
+  // width = half the tile width (gemm_stats_width)
+  SliceStats stats_out;
+};
 
 // Arguments of the RoPE epilogue: the GEMM's tile width is 2 * head_dim so
 // each epilogue warp holds whole heads; output columns [0, rot_cols) (Q and
@@ -92,10 +126,21 @@ cudaError_t launch_attention_simt(int dtype, const void *qkv, void *o, const Seq
 struct GemmPlan;
 // lost_tx: fault injection for the watchdog tests (0 in normal use): the
 // one-CTA kernel's stage barriers expect this many bytes more than arrive.
-cudaError_t launch_gemm_tc(const void *x, const void *w, const void *b, const void *res, void *y,
-                           int M, int N, int K, int epi, int num_sms, int *status,
-                           cudaStream_t st, const RopeEpi *rope = nullptr,
-                           uint32_t lost_tx = 0);
+// With kEpiStats, ea.stats_out.w must equal gemm_stats_width(M, N, K).
+cudaError_t launch_gemm_tc(const void *x, const void *w, const EpiArgs &ea, int M, int N, int K,
+                           int epi, int num_sms, cudaStream_t st, int *status,
+                           const RopeEpi *rope = nullptr, uint32_t lost_tx = 0);
+// Slice width of the row statistics a kEpiStats GEMM of this shape writes.
+int gemm_stats_width(int M, int N, int K, int num_sms);
+
+// Row statistics of x [rows, cols] bf16 in slices of 64 columns.
+constexpr int kRowStatsWidth = 64;
+cudaError_t launch_rowstats(const void *x, float2 *out, int rows, int cols, cudaStream_t st);
+// LayerNorm folded into the following projection w [n, k] (bias b [n], LN
+// gamma/beta [k]): w_out = bf16(w diag(gamma)), sc = fp32 [2][n]:
+// s = row sums of w_out, c = b + w beta.
+cudaError_t launch_fold_ln(const void *w, const void *gamma, const void *beta, const void *b,
+                           void *w_out, float *sc, int n, int k, cudaStream_t st);
 
 // tcgen05 flash attention, bf16, head_dim 72 or 128.
 // Split (stream-K) attention schedule: most CTAs it uses, and the bytes of

@@ -149,12 +149,25 @@ SeqArgs to_seq_args(const vit_seqs *s, bool with_pos) {
   return a;
 }
 
-cudaError_t run_linear(vit_ctx *ctx, int kind, const void *x, const void *w, const void *b,
-                       const void *res, void *y, int M, int N, int K, int epi, cudaStream_t st,
+EpiArgs epi_args(const void *b, const void *res, void *y) {
+  EpiArgs ea{};
+  ea.bias = static_cast<const __nv_bfloat16 *>(b);
+  ea.res = static_cast<const __nv_bfloat16 *>(res);
+  ea.y = static_cast<__nv_bfloat16 *>(y);
+  return ea;
+}
+
+// y = epi(x w^T ...): the SIMT kernel for fp32 contexts (plain epilogues
+// only), the tcgen05 kernel for bf16.
+cudaError_t run_linear(vit_ctx *ctx, int kind, const void *x, const void *w, const EpiArgs &ea,
+                       int M, int N, int K, int epi, cudaStream_t st,
                        const RopeEpi *rope = nullptr) {
   return counted(ctx, kind, st, [&] {
-    if (ctx->cfg.dtype == VIT_F32) return launch_gemm_simt(kF32, x, w, b, res, y, M, N, K, epi, st);
-    return launch_gemm_tc(x, w, b, res, y, M, N, K, epi, ctx->num_sms, ctx->d_status, st, rope,
+    if (ctx->cfg.dtype == VIT_F32) {
+      if (epi & ~kEpiOpMask) return cudaErrorInvalidValue;
+      return launch_gemm_simt(kF32, x, w, ea.bias, ea.res, ea.y, M, N, K, epi, st);
+    }
+    return launch_gemm_tc(x, w, ea, M, N, K, epi, ctx->num_sms, st, ctx->d_status, rope,
                           ctx->debug_lost_tx);
   });
 }
@@ -174,6 +187,20 @@ cudaError_t run_attention(vit_ctx *ctx, const void *qkv, void *o, const SeqArgs 
 struct Workspace {
   void *h, *qkv, *attn, *x1, *g, *act[2];
   void *part, *cnt;  // split attention: partial rows and per-item counters (or null)
+  // slice statistics of the layer input x and of x1 (folded LayerNorms, bf16)
+  float2 *stats_x, *stats_x1;
+};
+
+// Most slices a row's statistics take: the narrowest slice written is 64
+// columns (the row-statistics kernel, and the half tile of the narrowest
+// GEMM tile, 128 columns)
+inline int max_stat_parts(int C) { return (C + 63) / 64; }
+
+// Whether slice statistics of the layer input are in ws.stats_x, and their
+// slice width.
+struct StatsState {
+  bool valid = false;
+  int w = 0;
 };
 
 // CTAs of the split attention schedule whose scratch the workspace holds
@@ -188,52 +215,68 @@ size_t workspace_layout(const vit_config &c, int T, Workspace *w, void *base, in
   const size_t es = esize(c);
   const size_t C = size_t(c.hidden);
   const size_t F = (c.flags & VIT_FLAG_NO_MLP) ? 0 : size_t(c.mlp);
-  const size_t sizes[9] = {T * C * es, T * 3 * C * es, T * C * es, T * C * es,
-                           T * F * es, T * C * es, T * C * es,
-                           size_t(sk_ctas) * attn_split_part_bytes(), size_t(sk_ctas) * 4};
+  const size_t st = c.dtype == VIT_BF16 ? size_t(T) * max_stat_parts(c.hidden) * sizeof(float2) : 0;
+  constexpr int kSlots = 11;
+  const size_t sizes[kSlots] = {T * C * es, T * 3 * C * es, T * C * es, T * C * es,
+                                T * F * es, T * C * es, T * C * es,
+                                size_t(sk_ctas) * attn_split_part_bytes(), size_t(sk_ctas) * 4,
+                                st, st};
   size_t off = 0;
-  void **slots[9] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-  if (w) {
-    slots[0] = &w->h; slots[1] = &w->qkv; slots[2] = &w->attn; slots[3] = &w->x1;
-    slots[4] = &w->g; slots[5] = &w->act[0]; slots[6] = &w->act[1];
-    slots[7] = &w->part; slots[8] = &w->cnt;
-  }
-  for (int i = 0; i < 9; ++i) {
-    if (w) *slots[i] = sizes[i] ? static_cast<char *>(base) + off : nullptr;
+  void *ptrs[kSlots];
+  for (int i = 0; i < kSlots; ++i) {
+    ptrs[i] = sizes[i] && base ? static_cast<char *>(base) + off : nullptr;
     off += align256(sizes[i]);
+  }
+  if (w) {
+    w->h = ptrs[0]; w->qkv = ptrs[1]; w->attn = ptrs[2]; w->x1 = ptrs[3]; w->g = ptrs[4];
+    w->act[0] = ptrs[5]; w->act[1] = ptrs[6]; w->part = ptrs[7]; w->cnt = ptrs[8];
+    w->stats_x = static_cast<float2 *>(ptrs[9]);
+    w->stats_x1 = static_cast<float2 *>(ptrs[10]);
   }
   return off;
 }
 
 vit_status check_layer_weights(const vit_config &c, const vit_layer_weights *w) {
   if (!w) return VIT_ERR_INVALID_ARG;
-  const void *need[6] = {w->ln1_g, w->ln1_b, w->w_qkv, w->b_qkv, w->w_o, w->b_o};
+  auto ok = [&](const void *p) { return p && (c.dtype != VIT_BF16 || aligned16(p)); };
+  const bool no_mlp = (c.flags & VIT_FLAG_NO_MLP) != 0;
+  if ((w->qkv_fold || (w->fc1_fold && !no_mlp)) && c.dtype != VIT_BF16) return VIT_ERR_UNSUPPORTED;
+  // a folded LayerNorm leaves its gamma, beta and the projection's bias unread
+  const void *need[4] = {w->w_qkv, w->w_o, w->b_o, w->qkv_fold ? w->qkv_fold : w->b_qkv};
   for (const void *p : need)
-    if (!p || (c.dtype == VIT_BF16 && !aligned16(p))) return VIT_ERR_INVALID_ARG;
-  if (!(c.flags & VIT_FLAG_NO_MLP)) {
-    const void *mlp[6] = {w->ln2_g, w->ln2_b, w->w_fc1, w->b_fc1, w->w_fc2, w->b_fc2};
+    if (!ok(p)) return VIT_ERR_INVALID_ARG;
+  if (!w->qkv_fold && !(ok(w->ln1_g) && ok(w->ln1_b))) return VIT_ERR_INVALID_ARG;
+  if (!no_mlp) {
+    const void *mlp[4] = {w->w_fc1, w->w_fc2, w->b_fc2, w->fc1_fold ? w->fc1_fold : w->b_fc1};
     for (const void *p : mlp)
-      if (!p || (c.dtype == VIT_BF16 && !aligned16(p))) return VIT_ERR_INVALID_ARG;
+      if (!ok(p)) return VIT_ERR_INVALID_ARG;
+    if (!w->fc1_fold && !(ok(w->ln2_g) && ok(w->ln2_b))) return VIT_ERR_INVALID_ARG;
   }
   return VIT_OK;
 }
 
-// One layer; all arguments already validated.
+// One layer; all arguments already validated.  xs: whether ws.stats_x holds
+// the slice statistics of x (updated to those of y when out_stats, i.e. the
+// next layer folds its first LayerNorm; else cleared).
 vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, void *y,
-                      const vit_seqs *seqs, const Workspace &ws, cudaStream_t st) {
+                      const vit_seqs *seqs, const Workspace &ws, cudaStream_t st, StatsState &xs,
+                      bool out_stats) {
   const vit_config &c = ctx->cfg;
   const int T = seqs->total_tokens, C = c.hidden, F = c.mlp;
   const int dt = c.dtype == VIT_F32 ? kF32 : kBF16;
   const bool rope = !(c.flags & VIT_FLAG_NO_ROPE) && seqs->pos_rc != nullptr;
+  const bool no_mlp = (c.flags & VIT_FLAG_NO_MLP) != 0;
   const float scale = 1.0f / sqrtf(float(c.head_dim));
   auto ln = [&](const void *in, const void *g, const void *b) {
     return counted(ctx, VIT_K_LAYERNORM, st, [&] {
       return launch_layernorm(dt, in, ws.h, g, b, T, C, c.ln_eps, st);
     });
   };
-  if (ln(x, w->ln1_g, w->ln1_b)) return VIT_ERR_CUDA;
-  // bf16: the QKV GEMM rotates Q and K in its epilogue (tiles of two whole
-  // heads); fp32: a separate RoPE pass over the projection output
+  auto slices = [&](float2 *p, int width) { return SliceStats{p, (C + width - 1) / width, width}; };
+  // ---- LN1 + QKV (+ RoPE).  bf16: the QKV GEMM rotates Q and K in its
+  // epilogue (tiles of whole heads); fp32: a separate RoPE pass.  With the
+  // first LayerNorm folded, the GEMM reads x itself and normalises in its
+  // epilogue from x's slice statistics.
   const bool fused_rope = rope && dt == kBF16 && (c.head_dim == 72 || c.head_dim == 128);
   RopeEpi re{};
   if (fused_rope) {
@@ -242,32 +285,84 @@ vit_status layer_impl(vit_ctx *ctx, const vit_layer_weights *w, const void *x, v
     re.head_dim = c.head_dim;
     re.fr = ctx->fr;
   }
-  if (run_linear(ctx, VIT_K_GEMM_QKV, ws.h, w->w_qkv, w->b_qkv, nullptr, ws.qkv, T, 3 * C, C,
-                 fused_rope ? kEpiRope : kEpiBias, st, fused_rope ? &re : nullptr))
+  int epi_q = fused_rope ? kEpiRope : kEpiBias;
+  EpiArgs eq = epi_args(w->b_qkv, nullptr, ws.qkv);
+  const void *a_qkv = ws.h;
+  if (w->qkv_fold) {
+    if (!xs.valid) {
+      if (counted(ctx, VIT_K_ROWSTATS, st,
+                  [&] { return launch_rowstats(x, ws.stats_x, T, C, st); }))
+        return VIT_ERR_CUDA;
+      xs.valid = true;
+      xs.w = kRowStatsWidth;
+    }
+    eq.bias = nullptr;
+    eq.ln_sc = static_cast<const float *>(w->qkv_fold);
+    eq.stats_in = slices(ws.stats_x, xs.w);
+    eq.ln_eps = c.ln_eps;
+    epi_q |= kEpiLn;
+    a_qkv = x;
+  } else if (ln(x, w->ln1_g, w->ln1_b)) {
+    return VIT_ERR_CUDA;
+  }
+  if (run_linear(ctx, VIT_K_GEMM_QKV, a_qkv, w->w_qkv, eq, T, 3 * C, C, epi_q, st,
+                 fused_rope ? &re : nullptr))
     return VIT_ERR_CUDA;
   if (rope && !fused_rope && counted(ctx, VIT_K_ROPE, st, [&] {
         return launch_rope2d(dt, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st);
       }))
     return VIT_ERR_CUDA;
+  // ---- attention
   const SeqArgs sa = to_seq_args(seqs, false);
   if (run_attention(ctx, ws.qkv, ws.attn, sa, scale, st, static_cast<float *>(ws.part),
                     static_cast<int *>(ws.cnt)))
     return VIT_ERR_CUDA;
-  if (c.flags & VIT_FLAG_NO_MLP) {
-    if (run_linear(ctx, VIT_K_GEMM_OUT, ws.attn, w->w_o, w->b_o, x, y, T, C, C, kEpiResidual, st))
-      return VIT_ERR_CUDA;
+  // ---- out-projection + residual; it writes the slice statistics of its
+  // output when a folded LayerNorm reads that output next
+  const bool fold2 = !no_mlp && w->fc1_fold != nullptr;
+  const bool stats_o = no_mlp ? out_stats : fold2;
+  EpiArgs eo = epi_args(w->b_o, x, no_mlp ? y : ws.x1);
+  int epi_o = kEpiResidual, w_o = 0;
+  if (stats_o) {
+    w_o = gemm_stats_width(T, C, C, ctx->num_sms);
+    eo.stats_out = slices(no_mlp ? ws.stats_x : ws.stats_x1, w_o);
+    epi_o |= kEpiStats;
+  }
+  if (run_linear(ctx, VIT_K_GEMM_OUT, ws.attn, w->w_o, eo, T, C, C, epi_o, st))
+    return VIT_ERR_CUDA;
+  if (no_mlp) {
+    xs.valid = out_stats;
+    xs.w = w_o;
     return VIT_OK;
   }
-  if (run_linear(ctx, VIT_K_GEMM_OUT, ws.attn, w->w_o, w->b_o, x, ws.x1, T, C, C, kEpiResidual,
-                 st))
+  // ---- LN2 + fc1 + GELU
+  EpiArgs e1 = epi_args(w->b_fc1, nullptr, ws.g);
+  int epi_1 = kEpiGelu;
+  const void *a_fc1 = ws.h;
+  if (fold2) {
+    e1.bias = nullptr;
+    e1.ln_sc = static_cast<const float *>(w->fc1_fold);
+    e1.stats_in = slices(ws.stats_x1, w_o);
+    e1.ln_eps = c.ln_eps;
+    epi_1 |= kEpiLn;
+    a_fc1 = ws.x1;
+  } else if (ln(ws.x1, w->ln2_g, w->ln2_b)) {
     return VIT_ERR_CUDA;
-  if (ln(ws.x1, w->ln2_g, w->ln2_b)) return VIT_ERR_CUDA;
-  if (run_linear(ctx, VIT_K_GEMM_FC1, ws.h, w->w_fc1, w->b_fc1, nullptr, ws.g, T, F, C, kEpiGelu,
-                 st))
+  }
+  if (run_linear(ctx, VIT_K_GEMM_FC1, a_fc1, w->w_fc1, e1, T, F, C, epi_1, st))
     return VIT_ERR_CUDA;
-  if (run_linear(ctx, VIT_K_GEMM_FC2, ws.g, w->w_fc2, w->b_fc2, ws.x1, y, T, C, F, kEpiResidual,
-                 st))
+  // ---- fc2 + residual (+ the next layer's input statistics)
+  EpiArgs e2 = epi_args(w->b_fc2, ws.x1, y);
+  int epi_2 = kEpiResidual, w_2 = 0;
+  if (out_stats) {
+    w_2 = gemm_stats_width(T, C, F, ctx->num_sms);
+    e2.stats_out = slices(ws.stats_x, w_2);
+    epi_2 |= kEpiStats;
+  }
+  if (run_linear(ctx, VIT_K_GEMM_FC2, ws.g, w->w_fc2, e2, T, C, F, epi_2, st))
     return VIT_ERR_CUDA;
+  xs.valid = out_stats;
+  xs.w = w_2;
   return VIT_OK;
 }
 
@@ -485,6 +580,38 @@ size_t vit_workspace_bytes(const vit_ctx *ctx, int total_tokens) {
   return workspace_layout(ctx->cfg, total_tokens, nullptr, nullptr, split_ctas(ctx, total_tokens));
 }
 
+vit_status vit_fold_layernorm(vit_ctx *ctx, const vit_layer_weights *in, void *w_qkv_out,
+                              void *qkv_fold, void *w_fc1_out, void *fc1_fold, void *stream) {
+  if (!ctx || !in) return VIT_ERR_INVALID_ARG;
+  const vit_config &c = ctx->cfg;
+  if (c.dtype != VIT_BF16) return VIT_ERR_UNSUPPORTED;
+  const bool do_qkv = w_qkv_out || qkv_fold, do_fc1 = w_fc1_out || fc1_fold;
+  if ((do_qkv && !(w_qkv_out && qkv_fold)) || (do_fc1 && !(w_fc1_out && fc1_fold)))
+    return VIT_ERR_INVALID_ARG;
+  if (do_fc1 && (c.flags & VIT_FLAG_NO_MLP)) return VIT_ERR_INVALID_ARG;
+  const void *qkv_in[6] = {in->ln1_g, in->ln1_b, in->w_qkv, in->b_qkv, w_qkv_out, qkv_fold};
+  const void *fc1_in[6] = {in->ln2_g, in->ln2_b, in->w_fc1, in->b_fc1, w_fc1_out, fc1_fold};
+  for (int i = 0; i < 6; ++i) {
+    if (do_qkv && (!qkv_in[i] || !aligned16(qkv_in[i]))) return VIT_ERR_INVALID_ARG;
+    if (do_fc1 && (!fc1_in[i] || !aligned16(fc1_in[i]))) return VIT_ERR_INVALID_ARG;
+  }
+  if (!do_qkv && !do_fc1) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int C = c.hidden;
+  if (do_qkv && counted(ctx, VIT_K_FOLD, st, [&] {
+        return launch_fold_ln(in->w_qkv, in->ln1_g, in->ln1_b, in->b_qkv, w_qkv_out,
+                              static_cast<float *>(qkv_fold), 3 * C, C, st);
+      }))
+    return VIT_ERR_CUDA;
+  if (do_fc1 && counted(ctx, VIT_K_FOLD, st, [&] {
+        return launch_fold_ln(in->w_fc1, in->ln2_g, in->ln2_b, in->b_fc1, w_fc1_out,
+                              static_cast<float *>(fc1_fold), c.mlp, C, st);
+      }))
+    return VIT_ERR_CUDA;
+  return VIT_OK;
+}
+
 vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const void *x, void *y,
                              const vit_seqs *seqs, void *workspace, size_t ws_bytes,
                              void *stream) {
@@ -500,7 +627,8 @@ vit_status vit_layer_forward(vit_ctx *ctx, const vit_layer_weights *w, const voi
   // the split attention's counters start at zero; each launch leaves them so
   if (ws.cnt && cudaMemsetAsync(ws.cnt, 0, size_t(split_ctas(ctx, seqs->total_tokens)) * 4, st) != cudaSuccess)
     return VIT_ERR_CUDA;
-  return layer_impl(ctx, w, x, y, seqs, ws, st);
+  StatsState xs;
+  return layer_impl(ctx, w, x, y, seqs, ws, st, xs, false);
 }
 
 vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, int n_layers,
@@ -520,10 +648,13 @@ vit_status vit_encoder_forward(vit_ctx *ctx, const vit_layer_weights *layers, in
   // the split attention's counters start at zero; each launch leaves them so
   if (ws.cnt && cudaMemsetAsync(ws.cnt, 0, size_t(split_ctas(ctx, seqs->total_tokens)) * 4, st) != cudaSuccess)
     return VIT_ERR_CUDA;
+  StatsState xs;  // slice statistics of each layer's input, when a folded LN reads them
   for (int i = 0; i < n_layers; ++i) {
     const void *in = i == 0 ? x : ws.act[(i - 1) & 1];
     void *out = i == n_layers - 1 ? y : ws.act[i & 1];
-    if ((s = layer_impl(ctx, &layers[i], in, out, seqs, ws, st)) != VIT_OK) return s;
+    const bool next_folds = i + 1 < n_layers && layers[i + 1].qkv_fold != nullptr;
+    if ((s = layer_impl(ctx, &layers[i], in, out, seqs, ws, st, xs, next_folds)) != VIT_OK)
+      return s;
   }
   return VIT_OK;
 }
@@ -546,7 +677,7 @@ vit_status vit_layernorm(vit_ctx *ctx, const void *x, void *y, const void *gamma
                          const void *beta, int rows, int cols, float eps, void *stream) {
   if (!ctx || !x || !y || !gamma || !beta || rows < 0 || cols <= 0 || !(eps >= 0.f))
     return VIT_ERR_INVALID_ARG;
-  if (cols % 4 || cols > 4096) return VIT_ERR_UNSUPPORTED;
+  if (cols % 4 || cols > 16384) return VIT_ERR_UNSUPPORTED;
   const size_t a = esize(ctx->cfg) * 4;
   const void *ps[4] = {x, y, gamma, beta};
   for (const void *p : ps)
@@ -575,9 +706,50 @@ vit_status vit_linear(vit_ctx *ctx, const void *x, const void *w, const void *bi
   }
   if (M == 0) return VIT_OK;
   DeviceGuard g(ctx->device);
-  return cuda_status(run_linear(ctx, VIT_K_GEMM, x, w, bias,
-                                epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr, y, M, N, K,
-                                int(epi), static_cast<cudaStream_t>(stream)));
+  return cuda_status(run_linear(ctx, VIT_K_GEMM, x, w,
+                                epi_args(bias, epi == VIT_EPI_BIAS_RESIDUAL ? residual : nullptr, y),
+                                M, N, K, int(epi), static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- projector
+size_t vit_projector_workspace_bytes(const vit_ctx *ctx, int M, int d_in, int d_hidden) {
+  if (!ctx || M < 0 || d_in <= 0 || d_hidden <= 0) return 0;
+  const size_t e = esize(ctx->cfg);
+  return align256(size_t(M) * d_in * e) + align256(size_t(M) * d_hidden * e);
+}
+
+vit_status vit_projector(vit_ctx *ctx, const vit_projector_weights *w, const void *x, void *y,
+                         int M, int d_in, int d_hidden, int d_out, void *workspace,
+                         size_t ws_bytes, void *stream) {
+  if (!ctx || !w || !x || !y || M < 0 || d_in <= 0 || d_hidden <= 0 || d_out <= 0)
+    return VIT_ERR_INVALID_ARG;
+  const void *need[6] = {w->ln_g, w->ln_b, w->w1, w->b1, w->w2, w->b2};
+  const bool bf16 = ctx->cfg.dtype == VIT_BF16;
+  const size_t al = bf16 ? 16 : esize(ctx->cfg) * 4;
+  for (const void *p : need)
+    if (!p || reinterpret_cast<uintptr_t>(p) % al) return VIT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) % al || reinterpret_cast<uintptr_t>(y) % al || x == y)
+    return VIT_ERR_INVALID_ARG;
+  if (d_in % 4 || d_in > 16384) return VIT_ERR_UNSUPPORTED;
+  if (bf16 && (d_in % 8 || d_hidden % 8 || d_out % 8)) return VIT_ERR_UNSUPPORTED;
+  if (M == 0) return VIT_OK;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      ws_bytes < vit_projector_workspace_bytes(ctx, M, d_in, d_hidden))
+    return VIT_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int dt = bf16 ? kBF16 : kF32;
+  char *h = static_cast<char *>(workspace);
+  char *hid = h + align256(size_t(M) * d_in * esize(ctx->cfg));
+  if (counted(ctx, VIT_K_LAYERNORM, st, [&] {
+        return launch_layernorm(dt, x, h, w->ln_g, w->ln_b, M, d_in, ctx->cfg.ln_eps, st);
+      }))
+    return VIT_ERR_CUDA;
+  if (run_linear(ctx, VIT_K_GEMM, h, w->w1, epi_args(w->b1, nullptr, hid), M, d_hidden, d_in,
+                 kEpiGelu, st))
+    return VIT_ERR_CUDA;
+  return cuda_status(run_linear(ctx, VIT_K_GEMM, hid, w->w2, epi_args(w->b2, nullptr, y), M,
+                                d_out, d_hidden, kEpiBias, st));
 }
 
 // ---------------------------------------------------------------- embedding
@@ -649,8 +821,8 @@ vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels, const int32_t *grid
   if (counted(ctx, VIT_K_EMBED, st, [&] { return launch_pad_cols(dt, w_pe, w_pad, C, k, kp, st); }))
     return VIT_ERR_CUDA;
   // tokens = patches . w_pad^T + b_pe + interpolated table (residual epilogue)
-  return cuda_status(run_linear(ctx, VIT_K_GEMM, patches, w_pad, b_pe, pos, y, int(T), C, kp,
-                                kEpiResidual, st));
+  return cuda_status(run_linear(ctx, VIT_K_GEMM, patches, w_pad, epi_args(b_pe, pos, y), int(T), C,
+                                kp, kEpiResidual, st));
 }
 
 // ---------------------------------------------------------------- MXFP8
@@ -889,7 +1061,8 @@ extern "C" vit_status vit_layer_forward_noalloc(vit_ctx *ctx, const vit_layer_we
   // launch counts only: no timing events are created during this call
   const bool prof_on = ctx->prof.on;
   ctx->prof.on = false;
-  s = layer_impl(ctx, w, x, y, seqs, ws, static_cast<cudaStream_t>(stream));
+  StatsState xs;
+  s = layer_impl(ctx, w, x, y, seqs, ws, static_cast<cudaStream_t>(stream), xs, false);
   ctx->prof.on = prof_on;
   return s;
 }
