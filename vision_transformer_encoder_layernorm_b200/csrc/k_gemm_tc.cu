@@ -38,15 +38,38 @@ constexpr int kThreads = 320;   // 2 role warps + 8 epilogue warps
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kATileBytes = BM * BK * 2;  // 16 KB
 
-template <int BN>
+constexpr size_t kSmemLimit = 232448;  // dynamic shared memory of one CTA (227 KB)
+
+// Shared memory after the operand ring, counted from the barrier block:
+// barriers and bias slots (3 KB), the folded LayerNorm's slots (kEpiLn),
+// then one output staging buffer per epilogue warp: a 32 x 32 chunk
+// (64-byte swizzled), or for a RoPE tile one head of 32 rows x HD columns.
+constexpr uint32_t kLnSlotBytes = 1280;
+constexpr uint32_t kLnSlotsOffset = 3072;
+template <int EPI, int TS>
+struct EpiSmem {
+  static constexpr bool kRope = (EPI & 3) == 3;
+  static constexpr int kHD = kRope ? (TS == 216 ? 72 : TS / 2) : 0;
+  static constexpr uint32_t kBufBytes = kRope ? uint32_t(32 * kHD * 2) : 2048u;
+  static constexpr uint32_t kLnBytes = (EPI & 4) ? kEpiWarps * kLnSlotBytes : 0u;
+  static constexpr uint32_t kBufOff = (kLnSlotsOffset + kLnBytes + 1023u) / 1024u * 1024u;
+  static constexpr uint32_t kAfterRing = kBufOff + kEpiWarps * kBufBytes;
+};
+
+// Operand ring of a GEMM variant: as many stages (at most 8) as fit next to
+// the epilogue's shared memory.  PAIR: a CTA holds half of the tile's W rows.
+template <int BN, int EPI, int TS, bool PAIR>
 struct Cfg {
-  static constexpr uint32_t kBTileBytes = BN * BK * 2;
-  static constexpr uint32_t kStageBytes = kATileBytes + kBTileBytes;
-  static constexpr int kStages = (BN >= 256) ? 4 : 6;
+  using ES = EpiSmem<EPI, TS>;
+  static constexpr uint32_t kBRows = PAIR ? BN / 2 : BN;
+  static constexpr uint32_t kStageBytes = kATileBytes + kBRows * BK * 2;
+  static constexpr int kFit = int((kSmemLimit - 1024 - ES::kAfterRing) / kStageBytes);
+  static constexpr int kStages = kFit > 8 ? 8 : kFit;
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
-  // ring + barriers/bookkeeping + bias slots (8 warps x 128 bf16) + 1 KB alignment slack
-  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 2048 + 1024;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
+  // ring + 1 KB alignment slack + barriers, slots and staging buffers
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + ES::kAfterRing;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(PAIR ? 256 : BM, BN);
+  static_assert(kStages >= 2 && kStageBytes % 1024 == 0, "operand ring");
 };
 
 struct __align__(16) Bars {
@@ -81,25 +104,53 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 }  // namespace gemm
 
 // Mean and 1/sqrt(var + eps) of row `row` of a LayerNorm input of K
-// columns, from its slice statistics (Chan's pairwise update, slice order).
+// columns, from its slice statistics (mean_j, M2_j) over slices of n_j
+// columns: mean = sum_j n_j mean_j / K, M2 = sum_j M2_j + sum_j n_j
+// (mean_j - mean)^2 (the two-pass form of Chan's merge); the second pass
+// reads the same bytes again from L1.
 __device__ __forceinline__ void ln_row_stats(const EpiArgs &ea, int row, int K, float &mu,
                                              float &rstd) {
   const SliceStats &st = ea.stats_in;
   const float2 *p = st.p + size_t(row) * st.parts;
-  float n_a = 0.f, mean = 0.f, m2 = 0.f;
-#pragma unroll 4
-  for (int j = 0; j < st.parts; ++j) {
+  const int last = st.parts - 1;
+  const float wf = float(st.w), nl = float(K - last * st.w);
+  float s = 0.f;
+#pragma unroll 6
+  for (int j = 0; j < last; ++j) s += __ldg(p + j).x;
+  const float mean = fmaf(wf, s, nl * __ldg(p + last).x) / float(K);
+  float m2 = 0.f, dev = 0.f;
+#pragma unroll 6
+  for (int j = 0; j < last; ++j) {
     const float2 e = __ldg(p + j);
-    const float nb = float(min(st.w, K - j * st.w));
-    const float n = n_a + nb;
-    const float f = nb / n;
     const float d = e.x - mean;
-    mean = fmaf(d, f, mean);
-    m2 += e.y + d * d * n_a * f;
-    n_a = n;
+    m2 += e.y;
+    dev = fmaf(d, d, dev);
   }
+  const float2 el = __ldg(p + last);
+  const float dl = el.x - mean;
+  m2 += el.y + fmaf(wf, dev, nl * dl * dl);
   mu = mean;
   rstd = 1.0f / sqrtf(m2 / float(K) + ea.ln_eps);
+}
+
+using gemm::kLnSlotBytes;
+using gemm::kLnSlotsOffset;
+
+// Stages s and c of `ncols` columns starting at col0 (fp32 [2][N] at
+// ea.ln_sc) into slot[0..ncols) and slot[ncols..2 ncols); columns past N
+// read as zero.  Warp-level only (the slot is private to the warp).
+__device__ __forceinline__ void stage_ln_cols(float *slot, const EpiArgs &ea, int col0,
+                                              int ncols, int N, int lane) {
+  for (int i = lane; i < ncols / 4; i += 32) {
+    const int c = col0 + 4 * i;
+    const bool in = c < N;
+    const float4 sv = in ? __ldg(reinterpret_cast<const float4 *>(ea.ln_sc + c))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 cv = in ? __ldg(reinterpret_cast<const float4 *>(ea.ln_sc + N + c))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4 *>(slot)[i] = sv;
+    reinterpret_cast<float4 *>(slot + ncols)[i] = cv;
+  }
 }
 
 // Running (count, mean, M2) of a row slice, merged chunk by chunk.
@@ -118,15 +169,14 @@ struct RunStats {
 // One 32-column slice of one output row: fp32 accumulators r, then either
 // + bias (from shared memory) or, with the LayerNorm folded in,
 // rstd (r - mu s) + c (s, c already loaded); then the epilogue op (GELU, or
-// + residual rv, already loaded) and bf16 stores (columns at or past N are
-// skipped; N % 8 == 0).  With kEpiStats, adds the stored (rounded) values'
-// mean and M2 to `rs`.
+// + residual rv, already loaded); the 32 results rounded to bf16 in o.
+// With kEpiStats and `valid` (the row and the chunk exist), adds the mean
+// and M2 of the stored values of the chunk's columns below N to `rs`.
 template <int EPI>
-__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, int col0, int N,
-                                            const __nv_bfloat16 *bias_s, const uint4 (&rv)[4],
-                                            const float4 (&sv)[8], const float4 (&cv)[8], float mu,
-                                            float rstd, __nv_bfloat16 *__restrict__ y,
-                                            RunStats &rs) {
+__device__ __forceinline__ void compute_chunk(const uint32_t (&r)[32], int col0, int N, bool valid,
+                                              const __nv_bfloat16 *bias_s, const uint4 (&rv)[4],
+                                              const float4 (&sv)[8], const float4 (&cv)[8],
+                                              float mu, float rstd, uint4 (&o)[4], RunStats &rs) {
   constexpr int OP = EPI & kEpiOpMask;
   float v[32];
 #pragma unroll
@@ -164,61 +214,87 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], int row, in
       v[8 * q + 6] += bf16_lo(r4.w); v[8 * q + 7] += bf16_hi(r4.w);
     }
   }
-  uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
-  uint4 o[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     o[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
     o[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
     o[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
     o[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    if (col0 + 8 * q < N) yp[q] = o[q];
   }
   if constexpr ((EPI & kEpiStats) != 0) {
-    // statistics of the values as stored: the next GEMM multiplies these
-    float w[32];
+    if (valid) {
+      // statistics of the values as stored: the next GEMM multiplies these
+      float w[32];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      w[8 * q + 0] = bf16_lo(o[q].x); w[8 * q + 1] = bf16_hi(o[q].x);
-      w[8 * q + 2] = bf16_lo(o[q].y); w[8 * q + 3] = bf16_hi(o[q].y);
-      w[8 * q + 4] = bf16_lo(o[q].z); w[8 * q + 5] = bf16_hi(o[q].z);
-      w[8 * q + 6] = bf16_lo(o[q].w); w[8 * q + 7] = bf16_hi(o[q].w);
+      for (int q = 0; q < 4; ++q) {
+        w[8 * q + 0] = bf16_lo(o[q].x); w[8 * q + 1] = bf16_hi(o[q].x);
+        w[8 * q + 2] = bf16_lo(o[q].y); w[8 * q + 3] = bf16_hi(o[q].y);
+        w[8 * q + 4] = bf16_lo(o[q].z); w[8 * q + 5] = bf16_hi(o[q].z);
+        w[8 * q + 6] = bf16_lo(o[q].w); w[8 * q + 7] = bf16_hi(o[q].w);
+      }
+      const int nq = min(4, (N - col0) >> 3);  // valid 8-column groups (>= 1)
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < nq)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sum += w[8 * q + e];
+      const float nb = float(8 * nq);
+      const float mb = sum / nb;
+      float m2 = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < nq)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float d = w[8 * q + e] - mb;
+            m2 = fmaf(d, d, m2);
+          }
+      rs.merge(nb, mb, m2);
     }
-    const int nq = min(4, (N - col0) >> 3);  // valid 8-column groups (>= 1)
-    float sum = 0.f;
+  }
+}
+
+// Stages one warp's 32 x 32 chunk (thread = row `lane`, 64 bytes each) in
+// its 64-byte-swizzled buffer and stores it with one TMA copy at (col0,
+// row0); rows past M and columns past N are not written.  The buffer is
+// reused only after the previous copy has read it.
+__device__ __forceinline__ void stage_store_chunk(uint8_t *buf, const CUtensorMap *tm_y,
+                                                  const uint4 (&o)[4], int lane, int col0,
+                                                  int row0, bool any) {
+  if (lane == 0) bulk_wait_group_read<0>();
+  __syncwarp();
+  uint8_t *rowp = buf + lane * 64;
+  const int sw = (lane >> 1) & 3;  // 64-byte swizzle: 16-byte unit u ^ ((row >> 1) & 3)
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < nq)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sum += w[8 * q + e];
-    const float nb = float(8 * nq);
-    const float mb = sum / nb;
-    float m2 = 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < nq)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float d = w[8 * q + e] - mb;
-          m2 = fmaf(d, d, m2);
-        }
-    rs.merge(nb, mb, m2);
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(rowp + ((q ^ sw) << 4)) = o[q];
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && any) {
+    tma_store_2d(tm_y, buf, col0, row0);
+    bulk_commit_group();
   }
 }
 
 // Epilogue of one accumulator (one output tile) by the 8 epilogue warps:
 // epilogue warp e (= warp - 2) drains TMEM lane quarter (warp & 3), i.e. one
-// row per thread, and column half (e >> 2) of the tile.  The warp's half of
-// the tile bias was staged in its shared-memory slot (bias_w).  mu / rstd:
-// the row's LayerNorm statistics (kEpiLn).
-template <int BN, int EPI, int TS = BN>
+// row per thread (rows row0 .. row0 + 31 of the warp), and column half
+// (e >> 2) of the tile.  The warp's half of the tile bias was staged in its
+// shared-memory slot (bias_w).  mu / rstd: the row's LayerNorm statistics
+// (kEpiLn), s and c in the warp's ln_slot.  STAGED: results go through the
+// warp's staging buffer `ebuf` and TMA stores (tensor map tm_y); otherwise
+// each thread stores its row directly.
+template <int BN, int EPI, int TS = BN, bool STAGED = true>
 __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int lane, int row,
-                                              bool row_ok, int n0, int N, const RopeEpi &re,
+                                              int M, int n0, int N, const RopeEpi &re,
                                               const __nv_bfloat16 *bias_w, const EpiArgs &ea,
-                                              float mu, float rstd) {
+                                              float mu, float rstd, const float *ln_slot,
+                                              uint8_t *ebuf, const CUtensorMap *tm_y) {
   constexpr int kChunks = BN / 64;  // 32-column chunks per half
   constexpr int OP = EPI & kEpiOpMask;
   const int quarter = warp & 3, half = (warp - 2) >> 2;
+  const bool row_ok = row < M;
+  const int row0 = row - lane;  // the warp's first row
   __nv_bfloat16 *__restrict__ y = ea.y;
   if constexpr (OP == kEpiRope) {
     // whole heads: the tile holds HPT heads of HD columns (TS = HPT * HD;
@@ -229,110 +305,136 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
     static_assert(HPT * HD == TS && TS <= BN, "RoPE tile of whole heads");
 #pragma unroll 1
     for (int hh = half; hh < HPT; hh += 2) {
-    const int col0 = n0 + hh * HD;
-    const uint32_t base = tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(hh * HD);
-    uint32_t r[NF][32];
-    uint32_t r8[8];
-    __syncwarp();
+      const int col0 = n0 + hh * HD;
+      const uint32_t base = tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(hh * HD);
+      uint32_t r[NF][32];
+      uint32_t r8[8];
+      __syncwarp();
 #pragma unroll
-    for (int c = 0; c < NF; ++c) tmem_ld32(base + c * 32, r[c]);
-    if (HD % 32) tmem_ld8(base + NF * 32, r8);
-    tmem_ld_wait();
-    if (!(row_ok && col0 < N)) continue;
-    float v[HD];
+      for (int c = 0; c < NF; ++c) tmem_ld32(base + c * 32, r[c]);
+      if (HD % 32) tmem_ld8(base + NF * 32, r8);
+      tmem_ld_wait();
+      const bool valid = row_ok && col0 < N;
+      float v[HD];
 #pragma unroll
-    for (int i = 0; i < HD; ++i) {
-      const uint32_t bits = i < NF * 32 ? r[i / 32][i % 32] : r8[i - NF * 32];
-      v[i] = __uint_as_float(bits);
-    }
-    if constexpr ((EPI & kEpiLn) != 0) {
-      // the head's s and c (the same for the whole warp: broadcast loads)
-      const float4 *sp = reinterpret_cast<const float4 *>(ea.ln_sc + col0);
-      const float4 *cp = reinterpret_cast<const float4 *>(ea.ln_sc + N + col0);
-#pragma unroll
-      for (int u = 0; u < HD / 4; ++u) {
-        const float4 s4 = __ldg(sp + u), c4 = __ldg(cp + u);
-        v[4 * u + 0] = fmaf(rstd, fmaf(-mu, s4.x, v[4 * u + 0]), c4.x);
-        v[4 * u + 1] = fmaf(rstd, fmaf(-mu, s4.y, v[4 * u + 1]), c4.y);
-        v[4 * u + 2] = fmaf(rstd, fmaf(-mu, s4.z, v[4 * u + 2]), c4.z);
-        v[4 * u + 3] = fmaf(rstd, fmaf(-mu, s4.w, v[4 * u + 3]), c4.w);
+      for (int i = 0; i < HD; ++i) {
+        const uint32_t bits = i < NF * 32 ? r[i / 32][i % 32] : r8[i - NF * 32];
+        v[i] = __uint_as_float(bits);
       }
-    } else if (ea.bias != nullptr) {  // the head's bias (broadcast loads)
-      const uint4 *bp = reinterpret_cast<const uint4 *>(ea.bias + col0);
+      if constexpr ((EPI & kEpiLn) != 0) {
+        // the head's s and c, staged in the warp's slot (the k-th head of the
+        // warp at k * 2 HD: s, then c)
+        const float4 *sp = reinterpret_cast<const float4 *>(ln_slot + (hh >> 1) * 2 * HD);
+        const float4 *cp = sp + HD / 4;
 #pragma unroll
-      for (int u = 0; u < HD / 8; ++u) {
-        const uint4 b4 = __ldg(bp + u);
-        const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
+        for (int u = 0; u < HD / 4; ++u) {
+          const float4 s4 = sp[u], c4 = cp[u];
+          v[4 * u + 0] = fmaf(rstd, fmaf(-mu, s4.x, v[4 * u + 0]), c4.x);
+          v[4 * u + 1] = fmaf(rstd, fmaf(-mu, s4.y, v[4 * u + 1]), c4.y);
+          v[4 * u + 2] = fmaf(rstd, fmaf(-mu, s4.z, v[4 * u + 2]), c4.z);
+          v[4 * u + 3] = fmaf(rstd, fmaf(-mu, s4.w, v[4 * u + 3]), c4.w);
+        }
+      } else if (ea.bias != nullptr && col0 < N) {  // the head's bias (broadcast loads)
+        const uint4 *bp = reinterpret_cast<const uint4 *>(ea.bias + col0);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[8 * u + 2 * e] += bf16_lo(bb[e]);
-          v[8 * u + 2 * e + 1] += bf16_hi(bb[e]);
+        for (int u = 0; u < HD / 8; ++u) {
+          const uint4 b4 = __ldg(bp + u);
+          const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[8 * u + 2 * e] += bf16_lo(bb[e]);
+            v[8 * u + 2 * e + 1] += bf16_hi(bb[e]);
+          }
         }
       }
-    }
-    if (col0 < re.rot_cols) {
-      const int2 pr = reinterpret_cast<const int2 *>(re.pos)[row];
+      if (valid && col0 < re.rot_cols) {
+        const int2 pr = reinterpret_cast<const int2 *>(re.pos)[row];
 #pragma unroll
-      for (int axis = 0; axis < 2; ++axis) {
-        const float p = float(axis == 0 ? pr.x : pr.y);
+        for (int axis = 0; axis < 2; ++axis) {
+          const float p = float(axis == 0 ? pr.x : pr.y);
 #pragma unroll
-        for (int j = 0; j < Q4; ++j) {
-          float sn, cs;
-          sincospif(p * re.fr.wpi[j], &sn, &cs);
-          const float a = v[axis * (HD / 2) + j], b = v[axis * (HD / 2) + Q4 + j];
-          v[axis * (HD / 2) + j] = a * cs - b * sn;
-          v[axis * (HD / 2) + Q4 + j] = b * cs + a * sn;
+          for (int j = 0; j < Q4; ++j) {
+            float sn, cs;
+            sincospif(p * re.fr.wpi[j], &sn, &cs);
+            const float a = v[axis * (HD / 2) + j], b = v[axis * (HD / 2) + Q4 + j];
+            v[axis * (HD / 2) + j] = a * cs - b * sn;
+            v[axis * (HD / 2) + Q4 + j] = b * cs + a * sn;
+          }
         }
       }
-    }
-    uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
+      if constexpr (STAGED) {
+        // one head of the warp's 32 rows through the staging buffer
+        // (unswizzled rows of HD columns), then one TMA copy
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        uint4 *rowp = reinterpret_cast<uint4 *>(ebuf + lane * (HD * 2));
 #pragma unroll
-    for (int u = 0; u < HD / 8; ++u) {
-      uint4 o;
-      o.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-      o.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-      o.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-      o.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-      yp[u] = o;
-    }
+        for (int u = 0; u < HD / 8; ++u)
+          rowp[u] = make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]),
+                               pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                               pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                               pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < M && col0 < N) {
+          tma_store_2d(tm_y, ebuf, col0, row0);
+          bulk_commit_group();
+        }
+      } else if (valid) {
+        uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
+#pragma unroll
+        for (int u = 0; u < HD / 8; ++u)
+          yp[u] = make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]),
+                             pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                             pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                             pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+      }
     }
   } else {
-  RunStats rs;
+    RunStats rs;
 #pragma unroll 1
-  for (int i = 0; i < kChunks; ++i) {
-    const int c = half * kChunks + i;
-    const int col0 = n0 + c * 32;
-    const bool ok = row_ok && col0 < N;
-    uint32_t r[32];
-    __syncwarp();
-    tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c * 32), r);
-    // operands of the epilogue, in flight together with the TMEM load
-    uint4 rv[4];
-    if (OP == kEpiResidual && ok) {
-      const uint4 *rp = reinterpret_cast<const uint4 *>(ea.res + size_t(row) * N + col0);
+    for (int i = 0; i < kChunks; ++i) {
+      const int c = half * kChunks + i;
+      const int col0 = n0 + c * 32;
+      const bool ok = row_ok && col0 < N;
+      uint32_t r[32];
+      __syncwarp();
+      tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c * 32), r);
+      // operands of the epilogue, in flight together with the TMEM load
+      uint4 rv[4] = {};
+      if (OP == kEpiResidual && ok) {
+        const uint4 *rp = reinterpret_cast<const uint4 *>(ea.res + size_t(row) * N + col0);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) rv[q] = (col0 + 8 * q < N) ? __ldg(rp + q) : make_uint4(0, 0, 0, 0);
-    }
-    float4 sv[8], cv[8];
-    if ((EPI & kEpiLn) && ok) {
-      const float4 *sp = reinterpret_cast<const float4 *>(ea.ln_sc + col0);
-      const float4 *cp = reinterpret_cast<const float4 *>(ea.ln_sc + N + col0);
+        for (int q = 0; q < 4; ++q) rv[q] = (col0 + 8 * q < N) ? __ldg(rp + q) : make_uint4(0, 0, 0, 0);
+      }
+      float4 sv[8], cv[8];
+      if constexpr ((EPI & kEpiLn) != 0) {  // this chunk's s and c from the warp's slot
+        const float4 *sp = reinterpret_cast<const float4 *>(ln_slot + i * 32);
+        const float4 *cp = reinterpret_cast<const float4 *>(ln_slot + BN / 2 + i * 32);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const bool in = col0 + 4 * q < N;
-        sv[q] = in ? __ldg(sp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-        cv[q] = in ? __ldg(cp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < 8; ++q) {
+          sv[q] = sp[q];
+          cv[q] = cp[q];
+        }
+      }
+      tmem_ld_wait();
+      uint4 o[4];
+      compute_chunk<EPI>(r, col0, N, ok, bias_w + i * 32, rv, sv, cv, mu, rstd, o, rs);
+      if constexpr (STAGED) {
+        stage_store_chunk(ebuf, tm_y, o, lane, col0, row0, row0 < M && col0 < N);
+      } else if (ok) {
+        uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (col0 + 8 * q < N) yp[q] = o[q];
       }
     }
-    tmem_ld_wait();
-    if (ok) store_chunk<EPI>(r, row, col0, N, bias_w + i * 32, rv, sv, cv, mu, rstd, y, rs);
-  }
-  if constexpr ((EPI & kEpiStats) != 0) {
-    // this warp's slice of the row: columns [n0 + half BN/2, + BN/2)
-    const int c0 = n0 + half * (BN / 2);
-    if (row_ok && c0 < N)
-      ea.stats_out.p[size_t(row) * ea.stats_out.parts + c0 / (BN / 2)] = make_float2(rs.mean, rs.m2);
-  }
+    if constexpr ((EPI & kEpiStats) != 0) {
+      // this warp's slice of the row: columns [n0 + half BN/2, + BN/2)
+      const int c0 = n0 + half * (BN / 2);
+      if (row_ok && c0 < N)
+        ea.stats_out.p[size_t(row) * ea.stats_out.parts + c0 / (BN / 2)] = make_float2(rs.mean, rs.m2);
+    }
   }
 }
 
@@ -358,10 +460,11 @@ __device__ __forceinline__ void stage_bias_warp(__nv_bfloat16 *bias_w, const __n
 template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ EpiArgs ea, int M, int N, int K, int *status,
-                   const __grid_constant__ RopeEpi re, uint32_t lost_tx) {
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ EpiArgs ea,
+                   int M, int N, int K, int *status, const __grid_constant__ RopeEpi re,
+                   uint32_t lost_tx) {
   using namespace gemm;
-  using CF = Cfg<BN>;
+  using CF = Cfg<BN, EPI, BN, false>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -390,6 +493,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, CF::kTmemCols);
@@ -473,6 +577,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     const int row_in_tile = (warp & 3) * 32 + lane;
     __nv_bfloat16 *bias_w = reinterpret_cast<__nv_bfloat16 *>(bars + 1) + (warp - 2) * 128;
     int it = 0;
+    float *ln_slot = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + kLnSlotsOffset +
+                                               (warp - 2) * kLnSlotBytes);
+    uint8_t *ebuf = reinterpret_cast<uint8_t *>(bars) + CF::ES::kBufOff + (warp - 2) * CF::ES::kBufBytes;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
@@ -480,18 +587,25 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int row = mb * BM + row_in_tile;
       float mu = 0.f, rstd = 0.f;  // LayerNorm statistics of the row (kEpiLn)
       if constexpr ((EPI & kEpiLn) != 0) {
+        __syncwarp();  // the previous tile's reads of the slot are done
+        stage_ln_cols(ln_slot, ea, nb * BN + ((warp - 2) >> 2) * (BN / 2), BN / 2, N, lane);
         if (row < M) ln_row_stats(ea, row, K, mu, rstd);
+        __syncwarp();
       } else {
         stage_bias_warp<BN>(bias_w, ea.bias, nb * BN, N, warp, lane);
       }
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, re,
-                             bias_w, ea, mu, rstd);
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, M, nb * BN, N, re,
+                             bias_w, ea, mu, rstd, ln_slot, ebuf, &tmY);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
+      // the accumulator's TMEM reads are complete (tcgen05.wait::ld): a
+      // relaxed arrival, which does not wait for the tile's stores
+      if (lane == 0) mbar_arrive_relaxed(&bars->acc_empty[a]);
     }
+    if (lane == 0) bulk_wait_group<0>();  // the TMA stores have completed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -516,26 +630,13 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 //   - acc_empty[a] lives in the leader and collects the 8 epilogue warps of
 //     both CTAs (remote arrivals from the peer).
 // No load uses cluster multicast.
-namespace gemm {
-template <int BN>
-struct Cfg2 {
-  static constexpr uint32_t kBHalfBytes = (BN / 2) * BK * 2;
-  static constexpr uint32_t kStageBytes = kATileBytes + kBHalfBytes;  // per CTA
-  static constexpr int kStages = int((196u * 1024u) / kStageBytes) > 8 ? 8
-                                                                         : int((196u * 1024u) / kStageBytes);
-  static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
-  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 2048 + 1024;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(256, BN);
-};
-}  // namespace gemm
-
 template <int BN, int EPI, int TS = BN>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ EpiArgs ea, int M, int N, int K, int *status,
-                    const __grid_constant__ RopeEpi re) {
+                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ EpiArgs ea,
+                    int M, int N, int K, int *status, const __grid_constant__ RopeEpi re) {
   using namespace gemm;
-  using CF = Cfg2<BN>;
+  using CF = Cfg<BN, EPI, TS, true>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -569,6 +670,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc_pair(&bars->tmem_base, CF::kTmemCols);
@@ -655,6 +757,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     const int row_in_tile = int(rank) * BM + (warp & 3) * 32 + lane;
     __nv_bfloat16 *bias_w = reinterpret_cast<__nv_bfloat16 *>(bars + 1) + (warp - 2) * 128;
     int it = 0;
+    float *ln_slot = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + kLnSlotsOffset +
+                                               (warp - 2) * kLnSlotBytes);
+    uint8_t *ebuf = reinterpret_cast<uint8_t *>(bars) + CF::ES::kBufOff + (warp - 2) * CF::ES::kBufBytes;
     for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
       const int mb = tile % num_m, nb = tile / num_m;
       const int a = it & 1;
@@ -662,18 +767,33 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int row = mb * 2 * BM + row_in_tile;
       float mu = 0.f, rstd = 0.f;  // LayerNorm statistics of the row (kEpiLn)
       if constexpr ((EPI & kEpiLn) != 0) {
+        __syncwarp();  // the previous tile's reads of the slot are done
+        const int half = (warp - 2) >> 2;
+        if constexpr ((EPI & kEpiOpMask) == kEpiRope) {
+          // the warp's heads half, half + 2, ... of the tile, each [s HD | c HD]
+          constexpr int HPT = TS == 216 ? 3 : 2, HD = TS / HPT;
+          for (int hh = half, k = 0; hh < HPT; hh += 2, ++k)
+            stage_ln_cols(ln_slot + k * 2 * HD, ea, nb * TS + hh * HD, HD, N, lane);
+        } else {
+          stage_ln_cols(ln_slot, ea, nb * TS + half * (BN / 2), BN / 2, N, lane);
+        }
         if (row < M) ln_row_stats(ea, row, K, mu, rstd);
+        __syncwarp();
       } else if constexpr ((EPI & kEpiOpMask) != kEpiRope) {
         stage_bias_warp<BN>(bias_w, ea.bias, nb * TS, N, warp, lane);
       }
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile<BN, EPI, TS>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * TS, N, re,
-                                 bias_w, ea, mu, rstd);
+      epilogue_tile<BN, EPI, TS>(tmem + uint32_t(a * BN), warp, lane, row, M, nb * TS, N, re,
+                                 bias_w, ea, mu, rstd, ln_slot, ebuf, &tmY);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_cta(&bars->acc_empty[a], 0));
+      // the accumulator's TMEM reads are complete (tcgen05.wait::ld): a
+      // relaxed arrival, which does not wait for the tile's stores
+      if (lane == 0) mbar_arrive_cluster_relaxed(map_to_cta(&bars->acc_empty[a], 0));
     }
+    if (lane == 0) bulk_wait_group<0>();  // the TMA stores have completed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -717,42 +837,44 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const vo
 }
 
 template <int BN, int EPI>
-static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const EpiArgs &ea,
+static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb,
+                             const CUtensorMap &ty, const EpiArgs &ea,
                              int M, int N, int K, int num_sms, int *status, cudaStream_t st,
                              const RopeEpi &re, uint32_t lost_tx) {
-  using CF = gemm::Cfg<BN>;
+  using CF = gemm::Cfg<BN, EPI, BN, false>;
   auto kern = gemm_tc_kernel<BN, EPI>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmemBytes));
+  const size_t smem = CF::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + BN - 1) / BN);
   const int grid = std::max(1, std::min(tiles, num_sms));
-  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb, ea, M,
-                    N, K, status, re, lost_tx);
+  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), smem, st, 1, ta, tb, ty, ea, M, N, K,
+                    status, re, lost_tx);
 }
 
 // the epilogue combinations the library launches: plain bias, GELU and
 // residual; LayerNorm folded into bias or GELU; residual with row statistics
 template <int BN>
 static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
+                             const CUtensorMap &ty,
                               const EpiArgs &ea, int M, int N, int K, int num_sms, int *status,
                               cudaStream_t st, uint32_t lost_tx) {
   const RopeEpi none{};
   switch (epi) {
     case kEpiBias:
-      return launch_bn<BN, kEpiBias>(ta, tb, ea, M, N, K, num_sms, status, st, none, lost_tx);
+      return launch_bn<BN, kEpiBias>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none, lost_tx);
     case kEpiGelu:
-      return launch_bn<BN, kEpiGelu>(ta, tb, ea, M, N, K, num_sms, status, st, none, lost_tx);
+      return launch_bn<BN, kEpiGelu>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none, lost_tx);
     case kEpiResidual:
-      return launch_bn<BN, kEpiResidual>(ta, tb, ea, M, N, K, num_sms, status, st, none, lost_tx);
+      return launch_bn<BN, kEpiResidual>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none, lost_tx);
     case kEpiBias | kEpiLn:
-      return launch_bn<BN, kEpiBias | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none,
+      return launch_bn<BN, kEpiBias | kEpiLn>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none,
                                               lost_tx);
     case kEpiGelu | kEpiLn:
-      return launch_bn<BN, kEpiGelu | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none,
+      return launch_bn<BN, kEpiGelu | kEpiLn>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none,
                                               lost_tx);
     case kEpiResidual | kEpiStats:
-      return launch_bn<BN, kEpiResidual | kEpiStats>(ta, tb, ea, M, N, K, num_sms, status, st,
+      return launch_bn<BN, kEpiResidual | kEpiStats>(ta, tb, ty, ea, M, N, K, num_sms, status, st,
                                                      none, lost_tx);
     default:
       return cudaErrorInvalidValue;
@@ -760,13 +882,14 @@ static cudaError_t launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap 
 }
 
 template <int BN, int EPI, int TS = BN>
-static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const EpiArgs &ea,
+static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb,
+                             const CUtensorMap &ty, const EpiArgs &ea,
                                int M, int N, int K, int num_sms, int *status, cudaStream_t st,
                                const RopeEpi &re) {
-  using CF = gemm::Cfg2<BN>;
+  using CF = gemm::Cfg<BN, EPI, TS, true>;
   auto kern = gemm_tc2_kernel<BN, EPI, TS>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CF::kSmemBytes));
+  const size_t smem = CF::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -775,7 +898,7 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(gemm::kThreads);
-  cfg.dynamicSmemBytes = CF::kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -798,27 +921,28 @@ static cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
   }
   const int tiles = ((M + 2 * gemm::BM - 1) / (2 * gemm::BM)) * ((N + TS - 1) / TS);
   return launch_pdl(kern, dim3(2 * std::max(1, std::min(tiles, max_clusters))),
-                    dim3(gemm::kThreads), CF::kSmemBytes, st, 2, ta, tb, ea, M, N, K, status, re);
+                    dim3(gemm::kThreads), smem, st, 2, ta, tb, ty, ea, M, N, K, status, re);
 }
 
 template <int BN>
 static cudaError_t launch_pair_epi(int epi, const CUtensorMap &ta, const CUtensorMap &tb,
+                             const CUtensorMap &ty,
                                    const EpiArgs &ea, int M, int N, int K, int num_sms,
                                    int *status, cudaStream_t st) {
   const RopeEpi none{};
   switch (epi) {
     case kEpiBias:
-      return launch_pair<BN, kEpiBias>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiBias>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none);
     case kEpiGelu:
-      return launch_pair<BN, kEpiGelu>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiGelu>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none);
     case kEpiResidual:
-      return launch_pair<BN, kEpiResidual>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiResidual>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none);
     case kEpiBias | kEpiLn:
-      return launch_pair<BN, kEpiBias | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiBias | kEpiLn>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none);
     case kEpiGelu | kEpiLn:
-      return launch_pair<BN, kEpiGelu | kEpiLn>(ta, tb, ea, M, N, K, num_sms, status, st, none);
+      return launch_pair<BN, kEpiGelu | kEpiLn>(ta, tb, ty, ea, M, N, K, num_sms, status, st, none);
     case kEpiResidual | kEpiStats:
-      return launch_pair<BN, kEpiResidual | kEpiStats>(ta, tb, ea, M, N, K, num_sms, status, st,
+      return launch_pair<BN, kEpiResidual | kEpiStats>(ta, tb, ty, ea, M, N, K, num_sms, status, st,
                                                        none);
     default:
       return cudaErrorInvalidValue;
@@ -883,7 +1007,18 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const EpiArgs &ea, int 
                          ea.stats_in.parts != (K + ea.stats_in.w - 1) / ea.stats_in.w))
     return cudaErrorInvalidValue;
   const int b_rows = v.pair == 2 ? v.bn / 2 : v.bn;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
+  // output stores: 32-row boxes of 32 columns (64-byte swizzled staging) or,
+  // for RoPE tiles, of one head
+  if (op == kEpiRope) {
+    if (encode_tensor_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ea.y, N, M, uint64_t(N) * 2,
+                             rope->head_dim, 32, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else if (encode_tensor_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ea.y, N, M,
+                                  uint64_t(N) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) !=
+             CUDA_SUCCESS) {
+    return cudaErrorInvalidValue;
+  }
   if (encode_tensor_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, uint64_t(K) * 2,
                            gemm::BK, gemm::BM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -893,21 +1028,21 @@ cudaError_t launch_gemm_tc(const void *x, const void *w, const EpiArgs &ea, int 
   if (op == kEpiRope) {
     const bool ln = (epi & kEpiLn) != 0;
     if (v.bn == 224)
-      return ln ? launch_pair<224, kEpiRope | kEpiLn, 216>(ta, tb, ea, M, N, K, num_sms, status, st,
+      return ln ? launch_pair<224, kEpiRope | kEpiLn, 216>(ta, tb, ty, ea, M, N, K, num_sms, status, st,
                                                            *rope)
-                : launch_pair<224, kEpiRope, 216>(ta, tb, ea, M, N, K, num_sms, status, st, *rope);
-    return ln ? launch_pair<256, kEpiRope | kEpiLn, 256>(ta, tb, ea, M, N, K, num_sms, status, st,
+                : launch_pair<224, kEpiRope, 216>(ta, tb, ty, ea, M, N, K, num_sms, status, st, *rope);
+    return ln ? launch_pair<256, kEpiRope | kEpiLn, 256>(ta, tb, ty, ea, M, N, K, num_sms, status, st,
                                                          *rope)
-              : launch_pair<256, kEpiRope, 256>(ta, tb, ea, M, N, K, num_sms, status, st, *rope);
+              : launch_pair<256, kEpiRope, 256>(ta, tb, ty, ea, M, N, K, num_sms, status, st, *rope);
   }
   if (v.pair == 2) {
-    if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, ea, M, N, K, num_sms, status, st);
-    if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, ea, M, N, K, num_sms, status, st);
-    return launch_pair_epi<128>(epi, ta, tb, ea, M, N, K, num_sms, status, st);
+    if (v.bn == 256) return launch_pair_epi<256>(epi, ta, tb, ty, ea, M, N, K, num_sms, status, st);
+    if (v.bn == 192) return launch_pair_epi<192>(epi, ta, tb, ty, ea, M, N, K, num_sms, status, st);
+    return launch_pair_epi<128>(epi, ta, tb, ty, ea, M, N, K, num_sms, status, st);
   }
   if (v.bn == 256)
-    return launch_epi<256>(epi, ta, tb, ea, M, N, K, num_sms, status, st, lost_tx);
-  return launch_epi<128>(epi, ta, tb, ea, M, N, K, num_sms, status, st, lost_tx);
+    return launch_epi<256>(epi, ta, tb, ty, ea, M, N, K, num_sms, status, st, lost_tx);
+  return launch_epi<128>(epi, ta, tb, ty, ea, M, N, K, num_sms, status, st, lost_tx);
 }
 
 // ---------------------------------------------------------------- MXFP8 GEMM
@@ -1077,8 +1212,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * BM + row_in_tile;
-      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, row < M, nb * BN, N, none,
-                             bias_w, ea, 0.f, 0.f);
+      epilogue_tile<BN, EPI, BN, false>(tmem + uint32_t(a * BN), warp, lane, row, M, nb * BN, N,
+                                        none, bias_w, ea, 0.f, 0.f, nullptr, nullptr, nullptr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
