@@ -378,6 +378,31 @@ VIT_API vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void 
                                   const void *residual, void *y, int M, int N, int K,
                                   vit_epilogue epi, void *stream);
 
+/* ---- FP8 encoder layers ------------------------------------------------
+ * The encoder layer with its four projections (QKV, output, fc1, fc2) in
+ * MXFP8 (reading: the pages list fp8 variants of dense checkpoints and put
+ * FP16 / INT8 on the KLiteInfer road map, without a format; OCP MX v1.0
+ * MXFP8 E4M3 is taken).  Per projection the input activation is quantised
+ * along K (vit_mx8_quantize's rule) and multiplied with the weight's codes
+ * by the block-scaled tensor-core GEMM (vit_linear_mx8); LayerNorm, RoPE
+ * (a pass over the projection output), attention, GELU and the residual
+ * adds are those of the bf16 layer.  Weights are quantised once by the
+ * caller with vit_mx8_quantize (w_* [out, in] along in); the LayerNorm
+ * vectors and biases stay bf16.  bf16 contexts only.
+ * Workspace: vit_workspace_bytes_mx8 (the bf16 layer's buffers plus the
+ * quantised activations).  Errors as vit_encoder_forward; the folded
+ * LayerNorm and prefix K/V are not supported here (VIT_ERR_UNSUPPORTED). */
+typedef struct {
+  const void *ln1_g, *ln1_b, *b_qkv, *b_o, *ln2_g, *ln2_b, *b_fc1, *b_fc2;  /* bf16 */
+  const void *w_qkv_codes, *w_qkv_scales, *w_o_codes, *w_o_scales;
+  const void *w_fc1_codes, *w_fc1_scales, *w_fc2_codes, *w_fc2_scales;
+} vit_layer_weights_mx8;
+VIT_API size_t vit_workspace_bytes_mx8(const vit_ctx *ctx, int total_tokens);
+VIT_API vit_status vit_encoder_forward_mx8(vit_ctx *ctx, const vit_layer_weights_mx8 *layers,
+                                           int n_layers, const void *x, void *y,
+                                           const vit_seqs *seqs, void *workspace,
+                                           size_t ws_bytes, void *stream);
+
 /* ---- launch accounting and per-kernel timing ---- */
 
 /* Kernel kinds counted by the context (one count per kernel launch). */

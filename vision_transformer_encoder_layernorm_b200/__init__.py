@@ -59,6 +59,15 @@ class VitProjectorWeights(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in ("ln_g", "ln_b", "w1", "b1", "w2", "b2")]
 
 
+_MX8KEYS = ("ln1_g", "ln1_b", "b_qkv", "b_o", "ln2_g", "ln2_b", "b_fc1", "b_fc2",
+            "w_qkv_codes", "w_qkv_scales", "w_o_codes", "w_o_scales",
+            "w_fc1_codes", "w_fc1_scales", "w_fc2_codes", "w_fc2_scales")
+
+
+class VitLayerWeightsMx8(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in _MX8KEYS]
+
+
 class VitSeqs(ctypes.Structure):
     _fields_ = [("total_tokens", ctypes.c_int), ("n_seqs", ctypes.c_int),
                 ("max_seqlen", ctypes.c_int), ("cu_seqlens", ctypes.c_void_p),
@@ -91,6 +100,9 @@ ABI_FUNCTIONS = {
                               ctypes.POINTER(ctypes.c_double), _I]),
     "vit_embed_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I]),
     "vit_projector_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I, _I]),
+    "vit_workspace_bytes_mx8": (ctypes.c_size_t, [_P, _I]),
+    "vit_encoder_forward_mx8": (_I, [_P, ctypes.POINTER(VitLayerWeightsMx8), _I, _P, _P,
+                                     ctypes.POINTER(VitSeqs), _P, ctypes.c_size_t, _P]),
     "vit_projector": (_I, [_P, ctypes.POINTER(VitProjectorWeights), _P, _P, _I, _I, _I, _I, _P,
                            ctypes.c_size_t, _P]),
     "vit_patch_embed": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32), _I, _I, _P, _P, _P, _I, _I,
@@ -262,6 +274,36 @@ class Context:
         for k in ("ln1_g", "ln1_b", "b_qkv") + (("ln2_g", "ln2_b", "b_fc1") if mlp else ()):
             out[k] = None  # not read by a folded layer
         return out
+
+    def quantize_layer_mx8(self, weights, stream=None):
+        """The layer's four projection weights quantised once to MXFP8 (new
+        tensors); returns the mapping vit_encoder_forward_mx8 takes (the
+        LayerNorm vectors and biases are passed through)."""
+        import torch
+        out = {k: weights.get(k) for k in ("ln1_g", "ln1_b", "b_qkv", "b_o", "ln2_g", "ln2_b",
+                                           "b_fc1", "b_fc2")}
+        for name in ("w_qkv", "w_o", "w_fc1", "w_fc2"):
+            w = weights.get(name)
+            if w is None:
+                continue
+            n, k = w.shape
+            codes = torch.empty((n, mx8_row_bytes(k)), dtype=torch.uint8, device=w.device)
+            scales = torch.empty(mx8_scale_bytes(n, k), dtype=torch.uint8, device=w.device)
+            self.mx8_quantize(w, codes, scales, stream)
+            out[name + "_codes"], out[name + "_scales"] = codes, scales
+        return out
+
+    def workspace_bytes_mx8(self, total_tokens: int) -> int:
+        return int(lib.vit_workspace_bytes_mx8(self._h, total_tokens))
+
+    def encoder_forward_mx8(self, layers, x, y, sq: VitSeqs, workspace, stream=None):
+        """vit_encoder_forward_mx8; ``layers`` are mappings from
+        quantize_layer_mx8."""
+        arr = (VitLayerWeightsMx8 * len(layers))(
+            *[VitLayerWeightsMx8(*[_ptr(l.get(k)) for k in _MX8KEYS]) for l in layers])
+        _check("vit_encoder_forward_mx8", lib.vit_encoder_forward_mx8(
+            self._h, arr, len(layers), _ptr(x), _ptr(y), ctypes.byref(sq), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream)))
 
     def layer_forward(self, weights, x, y, sq: VitSeqs, workspace, stream=None):
         lw = layer_weights(weights) if not isinstance(weights, VitLayerWeights) else weights

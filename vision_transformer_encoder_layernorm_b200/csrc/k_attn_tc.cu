@@ -495,7 +495,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (gu == 0) break;
         if (gu == 2) continue;
         const Item &it = u.it;
-        for (int t = 0; t < it.n_tiles_q; ++t) {
+        // Q tiles: loaded here only when warp 3 has no touch-ups to do; else
+        // warp 3 loads them, so this thread never waits for an item's Q
+        // buffer to be free and keeps the K/V ring full across items
+        for (int t = 0; !kPrep && t < it.n_tiles_q; ++t) {
           // the previous unit's S MMAs of this tile have finished reading Q_t
           if (act[t] > 0 && !mbar_wait(&bars->q_empty[t], (act[t] - 1) & 1, abort_flag)) {
             ok = false;
@@ -649,10 +652,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
     }
   } else if (warp == 3 && kPrep) {
-    // ------------------------------------------------------------ Q, K, V touch-ups
-    // thread handles rows lane, lane + 32, ... of each tile
+    // ------------------------------------------------------------ Q loads, Q, K, V touch-ups
+    // lane 0 loads each item's Q tiles as soon as the previous item's last S
+    // has read the buffer; the warp then prepares them.  Thread handles rows
+    // lane, lane + 32, ... of each tile
     uint32_t J = 0;
     uint32_t act[2] = {0, 0};
+    uint32_t q_issued = 0;  // lane 0: per tile, a load in flight and its parity
     bool ok = true;
     for (int k = 0; ok; ++k) {
       Unit u;
@@ -661,7 +667,22 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       if (gu == 2) continue;
       const Item &it = u.it;
       for (int t = 0; t < it.n_tiles_q; ++t) {
+        int okq = 1;
+        if (lane == 0) {
+          // the previous unit's S MMAs of this tile have finished reading Q_t
+          if (act[t] > 0) okq = mbar_wait(&bars->q_empty[t], (act[t] - 1) & 1, abort_flag);
+          if (okq) {
+            uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
+            const int row = it.seg0 + it.q0 + t * kBlockQ;
+            mbar_arrive_expect_tx(&bars->q_full[t], CF::kQTile);
+            tma_load_2d(qt, &tm_q0, &bars->q_full[t], it.h * HD, row);
+            tma_load_2d(qt + CF::kQChunk0, &tm_q1, &bars->q_full[t], it.h * HD + 64, row);
+            q_issued = (q_issued & ~(3u << (2 * t))) | ((1u | ((act[t] & 1) << 1)) << (2 * t));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, okq, 0)) { ok = false; break; }
         if (!mbar_wait(&bars->q_full[t], act[t] & 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) q_issued &= ~(1u << (2 * t));  // landed
         uint8_t *qt = smem + CF::kQOff + t * CF::kQTile;
 #pragma unroll 1
         for (int r = lane; r < kBlockQ; r += 32) {
@@ -706,6 +727,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           mbar_arrive(&bars->v_ready[st]);
         }
       }
+    }
+    if (!ok && lane == 0) {  // Q copies still in flight land before the CTA exits
+      for (int t = 0; t < 2; ++t)
+        if (q_issued & (1u << (2 * t))) drain_wait(&bars->q_full[t], (q_issued >> (2 * t + 1)) & 1);
     }
   }
   } else {  // warps 4-19
@@ -771,7 +796,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tmem_ld_cols<HC>(s_addr, s);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&bars->s_free[t]);  // S_t may now be overwritten by the next key tile
+        // S_t may now be overwritten by the next key tile: the loads are
+        // complete (tcgen05.wait::ld), so the arrival is relaxed and does not
+        // wait for this thread's output stores of the previous item
+        mbar_arrive_relaxed(&bars->s_free[t]);
         if (nvalid < HC) {  // keys past the sequence end: -inf, so p = 0
 #pragma unroll
           for (int i = 0; i < HC; ++i)

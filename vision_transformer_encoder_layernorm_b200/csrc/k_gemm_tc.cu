@@ -41,18 +41,22 @@ constexpr uint32_t kATileBytes = BM * BK * 2;  // 16 KB
 constexpr size_t kSmemLimit = 232448;  // dynamic shared memory of one CTA (227 KB)
 
 // Shared memory after the operand ring, counted from the barrier block:
-// barriers and bias slots (3 KB), the folded LayerNorm's slots (kEpiLn),
-// then one output staging buffer per epilogue warp: a 32 x 32 chunk
-// (64-byte swizzled), or for a RoPE tile one head of 32 rows x HD columns.
-constexpr uint32_t kLnSlotBytes = 1280;
-constexpr uint32_t kLnSlotsOffset = 3072;
+// barriers and bias slots (3 KB) -- with a folded LayerNorm (no bias) the
+// LayerNorm's slots take the place of the bias slots, right after the
+// barriers -- then one output staging buffer per epilogue warp: a 32 x 32
+// chunk (64-byte swizzled), or for a RoPE tile one head of 32 rows x HD
+// columns.  A LayerNorm slot holds s and c of the warp's columns: half a
+// non-RoPE tile (<= 128 columns) or two heads of 72 / one of 128.
+constexpr uint32_t kLnSlotBytes = 1152;
+constexpr uint32_t kLnSlotsOffset = 256;
 template <int EPI, int TS>
 struct EpiSmem {
   static constexpr bool kRope = (EPI & 3) == 3;
   static constexpr int kHD = kRope ? (TS == 216 ? 72 : TS / 2) : 0;
   static constexpr uint32_t kBufBytes = kRope ? uint32_t(32 * kHD * 2) : 2048u;
   static constexpr uint32_t kLnBytes = (EPI & 4) ? kEpiWarps * kLnSlotBytes : 0u;
-  static constexpr uint32_t kBufOff = (kLnSlotsOffset + kLnBytes + 1023u) / 1024u * 1024u;
+  static constexpr uint32_t kBufOff =
+      (EPI & 4) ? (kLnSlotsOffset + kLnBytes + 1023u) / 1024u * 1024u : 3072u;
   static constexpr uint32_t kAfterRing = kBufOff + kEpiWarps * kBufBytes;
 };
 
@@ -81,6 +85,7 @@ struct __align__(16) Bars {
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(Bars) <= kLnSlotsOffset, "barrier block overlaps the LayerNorm slots");
 
 __device__ __forceinline__ float tanh_fast(float x) {
   float y;
@@ -106,29 +111,56 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 // Mean and 1/sqrt(var + eps) of row `row` of a LayerNorm input of K
 // columns, from its slice statistics (mean_j, M2_j) over slices of n_j
 // columns: mean = sum_j n_j mean_j / K, M2 = sum_j M2_j + sum_j n_j
-// (mean_j - mean)^2 (the two-pass form of Chan's merge); the second pass
-// reads the same bytes again from L1.
+// (mean_j - mean)^2 (the two-pass form of Chan's merge).  Rows of up to
+// kStatRegs slices are loaded at once into registers (all loads in flight
+// together); longer rows take a loop over L1.
+constexpr int kStatRegs = 20;
 __device__ __forceinline__ void ln_row_stats(const EpiArgs &ea, int row, int K, float &mu,
                                              float &rstd) {
   const SliceStats &st = ea.stats_in;
   const float2 *p = st.p + size_t(row) * st.parts;
   const int last = st.parts - 1;
   const float wf = float(st.w), nl = float(K - last * st.w);
-  float s = 0.f;
+  float mean, m2 = 0.f, dev = 0.f;
+  if (st.parts <= kStatRegs) {
+    float2 e[kStatRegs];
+#pragma unroll
+    for (int j = 0; j < kStatRegs; ++j) e[j] = j < st.parts ? __ldg(p + j) : make_float2(0.f, 0.f);
+    float s = 0.f, ml = 0.f, m2l = 0.f;
+#pragma unroll
+    for (int j = 0; j < kStatRegs; ++j) {
+      if (j < last) s += e[j].x;
+      if (j == last) {
+        ml = e[j].x;
+        m2l = e[j].y;
+      }
+    }
+    mean = fmaf(wf, s, nl * ml) / float(K);
+#pragma unroll
+    for (int j = 0; j < kStatRegs; ++j)
+      if (j < last) {
+        const float d = e[j].x - mean;
+        m2 += e[j].y;
+        dev = fmaf(d, d, dev);
+      }
+    const float dl = ml - mean;
+    m2 += m2l + fmaf(wf, dev, nl * dl * dl);
+  } else {
+    float s = 0.f;
 #pragma unroll 6
-  for (int j = 0; j < last; ++j) s += __ldg(p + j).x;
-  const float mean = fmaf(wf, s, nl * __ldg(p + last).x) / float(K);
-  float m2 = 0.f, dev = 0.f;
+    for (int j = 0; j < last; ++j) s += __ldg(p + j).x;
+    mean = fmaf(wf, s, nl * __ldg(p + last).x) / float(K);
 #pragma unroll 6
-  for (int j = 0; j < last; ++j) {
-    const float2 e = __ldg(p + j);
-    const float d = e.x - mean;
-    m2 += e.y;
-    dev = fmaf(d, d, dev);
+    for (int j = 0; j < last; ++j) {
+      const float2 e = __ldg(p + j);
+      const float d = e.x - mean;
+      m2 += e.y;
+      dev = fmaf(d, d, dev);
+    }
+    const float2 el = __ldg(p + last);
+    const float dl = el.x - mean;
+    m2 += el.y + fmaf(wf, dev, nl * dl * dl);
   }
-  const float2 el = __ldg(p + last);
-  const float dl = el.x - mean;
-  m2 += el.y + fmaf(wf, dev, nl * dl * dl);
   mu = mean;
   rstd = 1.0f / sqrtf(m2 / float(K) + ea.ln_eps);
 }
@@ -136,21 +168,37 @@ __device__ __forceinline__ void ln_row_stats(const EpiArgs &ea, int row, int K, 
 using gemm::kLnSlotBytes;
 using gemm::kLnSlotsOffset;
 
-// Stages s and c of `ncols` columns starting at col0 (fp32 [2][N] at
-// ea.ln_sc) into slot[0..ncols) and slot[ncols..2 ncols); columns past N
-// read as zero.  Warp-level only (the slot is private to the warp).
-__device__ __forceinline__ void stage_ln_cols(float *slot, const EpiArgs &ea, int col0,
-                                              int ncols, int N, int lane) {
-  for (int i = lane; i < ncols / 4; i += 32) {
-    const int c = col0 + 4 * i;
-    const bool in = c < N;
-    const float4 sv = in ? __ldg(reinterpret_cast<const float4 *>(ea.ln_sc + c))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 cv = in ? __ldg(reinterpret_cast<const float4 *>(ea.ln_sc + N + c))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-    reinterpret_cast<float4 *>(slot)[i] = sv;
-    reinterpret_cast<float4 *>(slot + ncols)[i] = cv;
-  }
+// Stages s and c of NSEG column segments of `ncols` columns each, starting
+// at col0[k] (fp32 [2][N] at ea.ln_sc), into slot + k * 2 ncols: s, then c;
+// columns past N read as zero.  Every load is issued before the first
+// shared-memory store.  Warp-level only (the slot is private to the warp).
+template <int NSEG, int MAXV>
+__device__ __forceinline__ void stage_ln_cols(float *slot, const EpiArgs &ea,
+                                              const int (&col0)[NSEG], int nseg, int ncols, int N,
+                                              int lane) {
+  float4 sv[NSEG][MAXV], cv[NSEG][MAXV];
+#pragma unroll
+  for (int k = 0; k < NSEG; ++k)
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int i = lane + 32 * m;
+      const int c = col0[k] + 4 * i;
+      const bool in = k < nseg && i < ncols / 4 && c < N;
+      sv[k][m] = in ? __ldg(reinterpret_cast<const float4 *>(ea.ln_sc + c))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      cv[k][m] = in ? __ldg(reinterpret_cast<const float4 *>(ea.ln_sc + N + c))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+  for (int k = 0; k < NSEG; ++k)
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int i = lane + 32 * m;
+      if (k < nseg && i < ncols / 4) {
+        reinterpret_cast<float4 *>(slot + k * 2 * ncols)[i] = sv[k][m];
+        reinterpret_cast<float4 *>(slot + k * 2 * ncols + ncols)[i] = cv[k][m];
+      }
+    }
 }
 
 // Running (count, mean, M2) of a row slice, merged chunk by chunk.
@@ -588,7 +636,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       float mu = 0.f, rstd = 0.f;  // LayerNorm statistics of the row (kEpiLn)
       if constexpr ((EPI & kEpiLn) != 0) {
         __syncwarp();  // the previous tile's reads of the slot are done
-        stage_ln_cols(ln_slot, ea, nb * BN + ((warp - 2) >> 2) * (BN / 2), BN / 2, N, lane);
+        const int c0[1] = {nb * BN + ((warp - 2) >> 2) * (BN / 2)};
+        stage_ln_cols<1, (BN / 2 / 4 + 31) / 32>(ln_slot, ea, c0, 1, BN / 2, N, lane);
         if (row < M) ln_row_stats(ea, row, K, mu, rstd);
         __syncwarp();
       } else {
@@ -772,10 +821,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         if constexpr ((EPI & kEpiOpMask) == kEpiRope) {
           // the warp's heads half, half + 2, ... of the tile, each [s HD | c HD]
           constexpr int HPT = TS == 216 ? 3 : 2, HD = TS / HPT;
-          for (int hh = half, k = 0; hh < HPT; hh += 2, ++k)
-            stage_ln_cols(ln_slot + k * 2 * HD, ea, nb * TS + hh * HD, HD, N, lane);
+          constexpr int NSEG = (HPT + 1) / 2;
+          int c0[NSEG];
+#pragma unroll
+          for (int k = 0; k < NSEG; ++k) c0[k] = nb * TS + (half + 2 * k) * HD;
+          stage_ln_cols<NSEG, (HD / 4 + 31) / 32>(ln_slot, ea, c0, (HPT - half + 1) / 2, HD, N,
+                                                  lane);
         } else {
-          stage_ln_cols(ln_slot, ea, nb * TS + half * (BN / 2), BN / 2, N, lane);
+          const int c0[1] = {nb * TS + half * (BN / 2)};
+          stage_ln_cols<1, (BN / 2 / 4 + 31) / 32>(ln_slot, ea, c0, 1, BN / 2, N, lane);
         }
         if (row < M) ln_row_stats(ea, row, K, mu, rstd);
         __syncwarp();

@@ -872,6 +872,119 @@ vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void *a_scale
   }));
 }
 
+// ---------------------------------------------------------------- FP8 layers
+namespace {
+
+// the bf16 layer's workspace, then the quantised activation (codes and
+// scales sized for the widest K, the MLP width)
+size_t mx8_extra(const vit_config &c, int T) {
+  const int kmax = (c.flags & VIT_FLAG_NO_MLP) ? c.hidden : std::max(c.hidden, c.mlp);
+  return align256(size_t(T) * mx8_row_bytes(kmax)) + align256(mx8_scale_bytes(T, kmax));
+}
+
+vit_status check_layer_weights_mx8(const vit_config &c, const vit_layer_weights_mx8 *w) {
+  if (!w) return VIT_ERR_INVALID_ARG;
+  const void *need[8] = {w->ln1_g, w->ln1_b, w->b_qkv, w->b_o,
+                         w->w_qkv_codes, w->w_qkv_scales, w->w_o_codes, w->w_o_scales};
+  for (const void *p : need)
+    if (!p || !aligned16(p)) return VIT_ERR_INVALID_ARG;
+  if (!(c.flags & VIT_FLAG_NO_MLP)) {
+    const void *mlp[8] = {w->ln2_g, w->ln2_b, w->b_fc1, w->b_fc2,
+                          w->w_fc1_codes, w->w_fc1_scales, w->w_fc2_codes, w->w_fc2_scales};
+    for (const void *p : mlp)
+      if (!p || !aligned16(p)) return VIT_ERR_INVALID_ARG;
+  }
+  return VIT_OK;
+}
+
+// One FP8 layer (all arguments validated).  aq / asc: quantised activation.
+vit_status layer_mx8_impl(vit_ctx *ctx, const vit_layer_weights_mx8 *w, const void *x, void *y,
+                          const vit_seqs *seqs, const Workspace &ws, uint8_t *aq, uint8_t *asc,
+                          cudaStream_t st) {
+  const vit_config &c = ctx->cfg;
+  const int T = seqs->total_tokens, C = c.hidden, F = c.mlp;
+  const bool rope = !(c.flags & VIT_FLAG_NO_ROPE) && seqs->pos_rc != nullptr;
+  const bool no_mlp = (c.flags & VIT_FLAG_NO_MLP) != 0;
+  const float scale = 1.0f / sqrtf(float(c.head_dim));
+  auto ln = [&](const void *in, const void *g, const void *b) {
+    return counted(ctx, VIT_K_LAYERNORM, st, [&] {
+      return launch_layernorm(kBF16, in, ws.h, g, b, T, C, c.ln_eps, st);
+    });
+  };
+  auto quant = [&](const void *a, int K) {
+    return counted(ctx, VIT_K_MX8_QUANTIZE, st,
+                   [&] { return launch_mx8_quantize(a, T, K, aq, asc, st); });
+  };
+  auto gemm = [&](int kind, const void *wc, const void *wsc, const void *b, const void *res,
+                  void *out, int N, int K, int epi) {
+    return counted(ctx, kind, st, [&] {
+      return launch_gemm_mx8(aq, asc, static_cast<const uint8_t *>(wc),
+                             static_cast<const uint8_t *>(wsc), b, res, out, T, N, K, epi,
+                             ctx->num_sms, ctx->d_status, st);
+    });
+  };
+  if (ln(x, w->ln1_g, w->ln1_b) || quant(ws.h, C) ||
+      gemm(VIT_K_GEMM_QKV, w->w_qkv_codes, w->w_qkv_scales, w->b_qkv, nullptr, ws.qkv, 3 * C, C,
+           kEpiBias))
+    return VIT_ERR_CUDA;
+  if (rope && counted(ctx, VIT_K_ROPE, st, [&] {
+        return launch_rope2d(kBF16, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st);
+      }))
+    return VIT_ERR_CUDA;
+  const SeqArgs sa = to_seq_args(seqs, false);
+  if (run_attention(ctx, ws.qkv, ws.attn, sa, scale, st)) return VIT_ERR_CUDA;
+  if (quant(ws.attn, C) || gemm(VIT_K_GEMM_OUT, w->w_o_codes, w->w_o_scales, w->b_o, x,
+                                no_mlp ? y : ws.x1, C, C, kEpiResidual))
+    return VIT_ERR_CUDA;
+  if (no_mlp) return VIT_OK;
+  if (ln(ws.x1, w->ln2_g, w->ln2_b) || quant(ws.h, C) ||
+      gemm(VIT_K_GEMM_FC1, w->w_fc1_codes, w->w_fc1_scales, w->b_fc1, nullptr, ws.g, F, C,
+           kEpiGelu) ||
+      quant(ws.g, F) ||
+      gemm(VIT_K_GEMM_FC2, w->w_fc2_codes, w->w_fc2_scales, w->b_fc2, ws.x1, y, C, F,
+           kEpiResidual))
+    return VIT_ERR_CUDA;
+  return VIT_OK;
+}
+
+}  // namespace
+
+size_t vit_workspace_bytes_mx8(const vit_ctx *ctx, int total_tokens) {
+  if (!ctx || total_tokens < 0 || ctx->cfg.dtype != VIT_BF16) return 0;
+  return workspace_layout(ctx->cfg, total_tokens, nullptr, nullptr, 0) +
+         mx8_extra(ctx->cfg, total_tokens);
+}
+
+vit_status vit_encoder_forward_mx8(vit_ctx *ctx, const vit_layer_weights_mx8 *layers,
+                                   int n_layers, const void *x, void *y, const vit_seqs *seqs,
+                                   void *workspace, size_t ws_bytes, void *stream) {
+  if (!ctx) return VIT_ERR_INVALID_ARG;
+  if (ctx->cfg.dtype != VIT_BF16) return VIT_ERR_UNSUPPORTED;
+  vit_status s = check_layer_call(ctx, x, y, seqs, workspace, ws_bytes, 0);
+  if (s != VIT_OK) return s;
+  if (seqs->prefix_kv) return VIT_ERR_UNSUPPORTED;
+  if (!layers || n_layers < 1) return VIT_ERR_INVALID_ARG;
+  for (int i = 0; i < n_layers; ++i)
+    if ((s = check_layer_weights_mx8(ctx->cfg, &layers[i])) != VIT_OK) return s;
+  const int T = seqs->total_tokens;
+  if (T == 0) return VIT_OK;
+  if (ws_bytes < vit_workspace_bytes_mx8(ctx, T)) return VIT_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  Workspace ws;
+  const size_t base = workspace_layout(ctx->cfg, T, &ws, workspace, 0);
+  const int kmax = (ctx->cfg.flags & VIT_FLAG_NO_MLP) ? ctx->cfg.hidden
+                                                      : std::max(ctx->cfg.hidden, ctx->cfg.mlp);
+  uint8_t *aq = static_cast<uint8_t *>(workspace) + base;
+  uint8_t *asc = aq + align256(size_t(T) * mx8_row_bytes(kmax));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < n_layers; ++i) {
+    const void *in = i == 0 ? x : ws.act[(i - 1) & 1];
+    void *out = i == n_layers - 1 ? y : ws.act[i & 1];
+    if ((s = layer_mx8_impl(ctx, &layers[i], in, out, seqs, ws, aq, asc, st)) != VIT_OK) return s;
+  }
+  return VIT_OK;
+}
+
 vit_status vit_rope2d(vit_ctx *ctx, void *qkv, const int32_t *pos_rc, int total_tokens,
                       void *stream) {
   if (!ctx || !qkv || !pos_rc || total_tokens < 0) return VIT_ERR_INVALID_ARG;
