@@ -1123,7 +1123,12 @@ struct CfgMx {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSfaCol = 2 * BN;      // 4 columns
   static constexpr uint32_t kSfbCol = 2 * BN + 4;  // 4 columns per 128 rows of W
-  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 2048 + 1024;
+  // ring + 1 KB alignment slack + barriers and bias slots (3 KB) + the
+  // epilogue warps' 2 KB output staging buffers
+  static constexpr uint32_t kBufOff = 3072;
+  static constexpr size_t kSmemBytes =
+      size_t(kStages) * kStageBytes + 1024 + kBufOff + kEpiWarps * 2048;
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory");
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KB alignment of the swizzled tiles");
   static_assert(kSfbCol + 4 * kSfbBlocks <= kTmemCols, "TMEM columns");
   static_assert(kStages <= 8, "barrier slots");
@@ -1133,8 +1138,9 @@ struct CfgMx {
 template <int BN, int EPI>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfb,
-                    const __grid_constant__ EpiArgs ea, int M, int N, int K, int *status) {
+                    const __grid_constant__ CUtensorMap tmY, const uint8_t *__restrict__ sfa,
+                    const uint8_t *__restrict__ sfb, const __grid_constant__ EpiArgs ea, int M,
+                    int N, int K, int *status) {
   using namespace gemm;
   using CF = CfgMx<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -1165,6 +1171,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, CF::kTmemCols);
@@ -1256,6 +1263,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int row_in_tile = (warp & 3) * 32 + lane;
     __nv_bfloat16 *bias_w = reinterpret_cast<__nv_bfloat16 *>(bars + 1) + (warp - 2) * 128;
+    uint8_t *ebuf = reinterpret_cast<uint8_t *>(bars) + CF::kBufOff + (warp - 2) * 2048;
     const RopeEpi none{};
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -1266,12 +1274,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (!mbar_wait(&bars->acc_full[a], aphase, abort_flag)) break;
       tc_fence_after();
       const int row = mb * BM + row_in_tile;
-      epilogue_tile<BN, EPI, BN, false>(tmem + uint32_t(a * BN), warp, lane, row, M, nb * BN, N,
-                                        none, bias_w, ea, 0.f, 0.f, nullptr, nullptr, nullptr);
+      epilogue_tile<BN, EPI>(tmem + uint32_t(a * BN), warp, lane, row, M, nb * BN, N, none,
+                             bias_w, ea, 0.f, 0.f, nullptr, ebuf, &tmY);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
+      if (lane == 0) mbar_arrive_relaxed(&bars->acc_empty[a]);  // TMEM reads complete
     }
+    if (lane == 0) bulk_wait_group<0>();  // the TMA stores have completed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -1284,7 +1294,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 }
 
 template <int BN, int EPI>
-static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb, const uint8_t *sfa,
+static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb,
+                                 const CUtensorMap &ty, const uint8_t *sfa,
                                  const uint8_t *sfb, const EpiArgs &ea, int M, int N, int K,
                                  int num_sms, int *status, cudaStream_t st) {
   using CF = gemm::CfgMx<BN>;
@@ -1294,8 +1305,8 @@ static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb, c
   if (e != cudaSuccess) return e;
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + BN - 1) / BN);
   const int grid = std::max(1, std::min(tiles, num_sms));
-  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb, sfa, sfb,
-                    ea, M, N, K, status);
+  return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), CF::kSmemBytes, st, 1, ta, tb, ty,
+                    sfa, sfb, ea, M, N, K, status);
 }
 
 cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes,
@@ -1310,19 +1321,23 @@ cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, con
   if (encode_tensor_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K, N, mx8_row_bytes(K),
                            gemm::kMxBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  CUtensorMap ty;  // output stores: 32 x 32 boxes, 64-byte swizzled staging
+  if (encode_tensor_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, uint64_t(N) * 2, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   EpiArgs ea{};
   ea.bias = static_cast<const __nv_bfloat16 *>(b);
   ea.res = static_cast<const __nv_bfloat16 *>(res);
   ea.y = static_cast<__nv_bfloat16 *>(y);
   switch (epi) {
     case kEpiGelu:
-      return launch_mx8_bn<BN, kEpiGelu>(ta, tb, a_scales, w_scales, ea, M, N, K, num_sms, status,
+      return launch_mx8_bn<BN, kEpiGelu>(ta, tb, ty, a_scales, w_scales, ea, M, N, K, num_sms, status,
                                          st);
     case kEpiResidual:
-      return launch_mx8_bn<BN, kEpiResidual>(ta, tb, a_scales, w_scales, ea, M, N, K, num_sms,
+      return launch_mx8_bn<BN, kEpiResidual>(ta, tb, ty, a_scales, w_scales, ea, M, N, K, num_sms,
                                              status, st);
     default:
-      return launch_mx8_bn<BN, kEpiBias>(ta, tb, a_scales, w_scales, ea, M, N, K, num_sms, status,
+      return launch_mx8_bn<BN, kEpiBias>(ta, tb, ty, a_scales, w_scales, ea, M, N, K, num_sms, status,
                                          st);
   }
 }
