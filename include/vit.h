@@ -271,13 +271,33 @@ VIT_API vit_status vit_positions_from_grids(vit_ctx *ctx, const int32_t *grids_h
  * centres, as PyTorch's align_corners = false) to (rows, cols) at (r, c).
  * 1 <= patch <= 32, n_images <= 1024, C % 8 == 0; b_pe, pos_table, y and the
  * workspace 16-byte aligned.  Workspace:
- * vit_embed_workspace_bytes (patches, padded weight, interpolated table). */
+ * vit_embed_workspace_bytes (patches, padded weight, interpolated table).
+ * Launches: one for the GEMM's operands (patch rows and resized position
+ * rows), one that pads w_pe to the GEMM's layout (see
+ * vit_patch_embed_padded, which skips it), and the GEMM, whose epilogue adds
+ * b_pe and the position rows. */
 VIT_API size_t vit_embed_workspace_bytes(const vit_ctx *ctx, int total_tokens, int patch);
 VIT_API vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels,
                                    const int32_t *grids_hw_host, int n_images, int patch,
                                    const void *w_pe, const void *b_pe, const void *pos_table,
                                    int table_h, int table_w, void *y, void *workspace,
                                    size_t ws_bytes, void *stream);
+/* The GEMM's weight layout: w_pad [C, Kp], Kp = vit_patch_kp(patch) = 3 p^2
+ * rounded up to a multiple of 8 (a TMA row must be a multiple of 16 bytes),
+ * columns 3p^2 .. Kp-1 zero.  vit_pad_patch_weight writes it from w_pe
+ * [C, 3 p^2] once (a model constant, as a loader would prepare it);
+ * vit_patch_embed_padded is vit_patch_embed with that weight, one launch
+ * fewer per call.  vit_patch_kp returns 0 for a patch outside 1..32;
+ * w_pad 16-byte aligned; same workspace as vit_patch_embed. */
+VIT_API int vit_patch_kp(int patch);
+VIT_API vit_status vit_pad_patch_weight(vit_ctx *ctx, const void *w_pe, int patch, void *w_pad,
+                                        void *stream);
+VIT_API vit_status vit_patch_embed_padded(vit_ctx *ctx, const void *pixels,
+                                          const int32_t *grids_hw_host, int n_images, int patch,
+                                          const void *w_pad, const void *b_pe,
+                                          const void *pos_table, int table_h, int table_w,
+                                          void *y, void *workspace, size_t ws_bytes,
+                                          void *stream);
 /* The interpolation alone: y [T, C] = resized pos_table per image (as above). */
 VIT_API vit_status vit_pos_interp(vit_ctx *ctx, const void *pos_table, int table_h, int table_w,
                                   const int32_t *grids_hw_host, int n_images, void *y,

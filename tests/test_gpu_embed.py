@@ -81,3 +81,39 @@ def test_patch_embed_errors_leave_output_untouched():
     torch.cuda.synchronize()
     assert bool((y == 3.0).all())
     ctx.close()
+
+
+@pytest.mark.parametrize("name,grids,patch,px_offset", [
+    ("c1", [(50, 78)], 14, 0), ("c1", [(4, 6), (6, 4), (2, 2)], 14, 1), ("c1", [(3, 5)], 16, 0),
+    ("c0", [(5, 3)], 7, 0), ("c0", [(4, 4), (2, 6)], 4, 0)])
+def test_patch_embed_padded_weight(name, grids, patch, px_offset):
+    """The weight padded once (vit_pad_patch_weight) and the padded entry give
+    the same tokens as vit_patch_embed, bit for bit, and match the oracle;
+    px_offset = 1 starts the pixels off a four-byte boundary (element path)."""
+    wl = synth.get(name).with_(grids=grids)
+    inp = synth.make_embed_inputs(wl, patch=patch)
+    ctx = context_for(wl)
+    T = sum(r * c for r, c in grids)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    flat = _pixels(inp, wl.dtype)
+    px = torch.empty(flat.numel() + px_offset, dtype=flat.dtype, device="cuda")[px_offset:]
+    px.copy_(flat)
+    w = to_dev(inp.w_pe, wl.dtype)
+    b, t = to_dev(inp.b_pe, wl.dtype), to_dev(inp.table, wl.dtype)
+    w_pad = ctx.pad_patch_weight(w, patch)
+    kp = vit.lib.vit_patch_kp(patch)
+    assert w_pad.shape == (wl.hidden, kp) and kp % 8 == 0 and kp >= 3 * patch * patch
+    assert torch.equal(w_pad[:, :3 * patch * patch], w) and not w_pad[:, 3 * patch * patch:].any()
+    ws = torch.empty(ctx.embed_workspace_bytes(T, patch), dtype=torch.uint8, device="cuda")
+    y0 = torch.empty((T, wl.hidden), dtype=dt, device="cuda")
+    y1 = torch.empty_like(y0)
+    ctx.patch_embed(px, grids, patch, w, b, t, y0, ws)
+    ctx.patch_embed_padded(px, grids, patch, w_pad, b, t, y1, ws)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    assert torch.equal(y0, y1)
+    f = lambda a: synth.to_f64(a, wl.dtype)
+    ref = E.embed_images([f(im) for im in inp.images], grids, patch, f(inp.w_pe), f(inp.b_pe),
+                         f(inp.table))
+    assert_close(from_dev(y1), ref, *TOL[wl.dtype], f"embed padded {name} {grids} p{patch}")
+    ctx.close()

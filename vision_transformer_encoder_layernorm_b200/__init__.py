@@ -107,6 +107,10 @@ ABI_FUNCTIONS = {
                            ctypes.c_size_t, _P]),
     "vit_patch_embed": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32), _I, _I, _P, _P, _P, _I, _I,
                              _P, _P, ctypes.c_size_t, _P]),
+    "vit_patch_embed_padded": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32), _I, _I, _P, _P, _P, _I,
+                                    _I, _P, _P, ctypes.c_size_t, _P]),
+    "vit_patch_kp": (_I, [_I]),
+    "vit_pad_patch_weight": (_I, [_P, _P, _I, _P, _P]),
     "vit_pos_interp": (_I, [_P, _P, _I, _I, ctypes.POINTER(ctypes.c_int32), _I, _P, _P]),
     "vit_graph_begin": (_I, [_P, ctypes.POINTER(_P)]),
     "vit_graph_end": (_I, [_P, ctypes.POINTER(_P)]),
@@ -404,6 +408,28 @@ class Context:
         th, tw = int(pos_table.shape[0]), int(pos_table.shape[1])
         _check("vit_patch_embed", lib.vit_patch_embed(
             self._h, _ptr(pixels), arr, n, patch, _ptr(w_pe), _ptr(b_pe), _ptr(pos_table), th, tw,
+            _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream)))
+
+    def pad_patch_weight(self, w_pe, patch: int, stream=None):
+        """vit_pad_patch_weight: w_pe [C, 3*patch*patch] (or [C, 3, patch,
+        patch]) -> a new [C, vit_patch_kp(patch)] tensor in the GEMM's layout."""
+        import torch
+        kp = int(lib.vit_patch_kp(patch))
+        if kp <= 0:
+            raise VitError(STATUS["VIT_ERR_INVALID_ARG"], "vit_patch_kp")
+        w_pad = torch.empty((w_pe.shape[0], kp), dtype=w_pe.dtype, device=w_pe.device)
+        _check("vit_pad_patch_weight", lib.vit_pad_patch_weight(self._h, _ptr(w_pe), patch,
+                                                                _ptr(w_pad), _stream(stream)))
+        return w_pad
+
+    def patch_embed_padded(self, pixels, grids, patch: int, w_pad, b_pe, pos_table, y, workspace,
+                           stream=None):
+        """patch_embed with the weight from pad_patch_weight (one launch fewer)."""
+        arr, n = _grids_arr(grids)
+        th, tw = int(pos_table.shape[0]), int(pos_table.shape[1])
+        _check("vit_patch_embed_padded", lib.vit_patch_embed_padded(
+            self._h, _ptr(pixels), arr, n, patch, _ptr(w_pad), _ptr(b_pe), _ptr(pos_table), th, tw,
             _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
             _stream(stream)))
 

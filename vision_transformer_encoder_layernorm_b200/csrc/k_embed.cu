@@ -14,39 +14,8 @@
 
 namespace vit {
 
-// ---------------------------------------------------------------- patches
-// patches [T, Kp] (Kp = 3*p*p rounded up to a multiple of 8, zero padded).
-// Block (x, image): kTokPerBlock tokens of the image, the threads across
-// each token's Kp entries.  Image i's pixels start at base(i) * 3 * p * p.
+// Tokens per block of the operand kernel below.
 constexpr int kTokPerBlock = 4;
-
-template <typename T>
-__global__ void __launch_bounds__(256) patchify_kernel(const __grid_constant__ ImageTable tab,
-                                                        const T *__restrict__ px,
-                                                        T *__restrict__ out, int p, int kp) {
-  pdl_trigger();
-  pdl_wait();
-  const ImageEntry im = tab.img[blockIdx.y];
-  const int n_tok = im.rows * im.cols;
-  const int pp = p * p, k3 = 3 * pp;
-  const int W = im.cols * p, Hh = im.rows * p;
-  const T *img = px + (long long)im.base * k3;
-  for (int tt = 0; tt < kTokPerBlock; ++tt) {
-    const int tok = blockIdx.x * kTokPerBlock + tt;
-    if (tok >= n_tok) break;
-    const int r = tok / im.cols, c = tok - r * im.cols;
-    const T *src = img + (long long)(r * p) * W + c * p;
-    T *dst = out + (long long)(im.base + tok) * kp;
-    for (int k = threadIdx.x; k < kp; k += blockDim.x) {
-      T v = from_f32<T>(0.0f);
-      if (k < k3) {
-        const int ch = k / pp, rem = k - ch * pp, y = rem / p, x = rem - y * p;
-        v = src[((long long)ch * Hh + y) * W + x];
-      }
-      dst[k] = v;
-    }
-  }
-}
 
 // w [N, K] -> w_pad [N, Kp], zero columns K..Kp-1; block per row
 template <typename T>
@@ -141,16 +110,95 @@ __global__ void __launch_bounds__(128) pos_interp_kernel(const __grid_constant__
   }
 }
 
-cudaError_t launch_patchify(int dtype, const ImageTable &tab, int n_images, long long max_tokens,
-                            const void *px, void *out, int p, int kp, cudaStream_t st) {
+// ---------------------------------------------------------------- both inputs of the GEMM
+// One launch for the embedding GEMM's operands: block (x, image) covers
+// kTokPerBlock tokens of the image and writes their patch rows (patches
+// [T, Kp], zero padded) and their resized position rows (pos [T, C]).  A
+// patch row is 3p runs of p pixels (one per channel and pixel row); with
+// bf16 pixels and an even p a run moves as p/2 four-byte words (a run starts
+// at an even element of an image row, and at an even element of the patch
+// row, and the pixels start at a four-byte boundary: `words`), otherwise
+// element by element.  Position rows as pos_interp_kernel:
+// 16-byte table loads, fp32 blend.
+template <typename T>
+__global__ void __launch_bounds__(256) embed_inputs_kernel(const __grid_constant__ ImageTable tab,
+                                                            const T *__restrict__ px,
+                                                            T *__restrict__ patches, int p, int kp,
+                                                            int words, const T *__restrict__ table,
+                                                            int gh, int gw, int C,
+                                                            T *__restrict__ pos) {
+  pdl_trigger();
+  pdl_wait();
+  const ImageEntry im = tab.img[blockIdx.y];
+  const int n_tok = im.rows * im.cols;
+  const int tok0 = blockIdx.x * kTokPerBlock;
+  if (tok0 >= n_tok) return;
+  const int nt = min(kTokPerBlock, n_tok - tok0);
+  const int pp = p * p, k3 = 3 * pp;
+  const int W = im.cols * p, Hh = im.rows * p;
+  const T *img = px + (long long)im.base * k3;
+  // patch rows: work unit = (token, run); then the padding columns
+  const int runs = 3 * p;
+  for (int u = threadIdx.x; u < nt * runs; u += blockDim.x) {
+    const int tt = u / runs, run = u - tt * runs;
+    const int tok = tok0 + tt;
+    const int r = tok / im.cols, c = tok - r * im.cols;
+    const int ch = run / p, y = run - ch * p;
+    const T *src = img + ((long long)ch * Hh + (long long)r * p + y) * W + (long long)c * p;
+    T *dst = patches + (long long)(im.base + tok) * kp + ch * pp + y * p;
+    if (words) {
+      const uint32_t *s4 = reinterpret_cast<const uint32_t *>(src);
+      uint32_t *d4 = reinterpret_cast<uint32_t *>(dst);
+      for (int i = 0; i < p / 2; ++i) d4[i] = __ldg(s4 + i);
+    } else {
+      for (int i = 0; i < p; ++i) dst[i] = src[i];
+    }
+  }
+  const int pad = kp - k3;
+  for (int u = threadIdx.x; u < nt * pad; u += blockDim.x) {
+    const int tt = u / pad;
+    patches[(long long)(im.base + tok0 + tt) * kp + k3 + (u - tt * pad)] = from_f32<T>(0.0f);
+  }
+  // position rows: work unit = (token, 8 channels)
+  const int c8 = C / 8;
+  for (int u = threadIdx.x; u < nt * c8; u += blockDim.x) {
+    const int tt = u / c8, ch = (u - tt * c8) * 8;
+    const int tok = tok0 + tt;
+    const int r = tok / im.cols, c = tok - r * im.cols;
+    int y0, y1, x0, x1;
+    float wy, wx;
+    bilinear_axis(r, im.rows, gh, y0, y1, wy);
+    bilinear_axis(c, im.cols, gw, x0, x1, wx);
+    float a[8], b[8], d[8], f[8], o[8];
+    Vec8<T>::load(table + ((long long)y0 * gw + x0) * C + ch, a);
+    Vec8<T>::load(table + ((long long)y0 * gw + x1) * C + ch, b);
+    Vec8<T>::load(table + ((long long)y1 * gw + x0) * C + ch, d);
+    Vec8<T>::load(table + ((long long)y1 * gw + x1) * C + ch, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float top = (1.0f - wx) * a[e] + wx * b[e];
+      const float bot = (1.0f - wx) * d[e] + wx * f[e];
+      o[e] = (1.0f - wy) * top + wy * bot;
+    }
+    Vec8<T>::store(pos + (long long)(im.base + tok) * C + ch, o);
+  }
+}
+
+cudaError_t launch_embed_inputs(int dtype, const ImageTable &tab, int n_images,
+                                long long max_tokens, const void *px, void *patches, int p, int kp,
+                                const void *table, int gh, int gw, int C, void *pos,
+                                cudaStream_t st) {
   if (n_images == 0 || max_tokens == 0) return cudaSuccess;
   const dim3 grid(unsigned((max_tokens + kTokPerBlock - 1) / kTokPerBlock), n_images);
   if (dtype == kF32)
-    return launch_pdl(patchify_kernel<float>, grid, dim3(256), 0, st, 1, tab,
-                      static_cast<const float *>(px), static_cast<float *>(out), p, kp);
-  return launch_pdl(patchify_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, 1, tab,
-                    static_cast<const __nv_bfloat16 *>(px), static_cast<__nv_bfloat16 *>(out), p,
-                    kp);
+    return launch_pdl(embed_inputs_kernel<float>, grid, dim3(256), 0, st, 1, tab,
+                      static_cast<const float *>(px), static_cast<float *>(patches), p, kp, 0,
+                      static_cast<const float *>(table), gh, gw, C, static_cast<float *>(pos));
+  const int words = (p % 2 == 0 && (reinterpret_cast<uintptr_t>(px) & 3) == 0) ? 1 : 0;
+  return launch_pdl(embed_inputs_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, 1, tab,
+                    static_cast<const __nv_bfloat16 *>(px), static_cast<__nv_bfloat16 *>(patches),
+                    p, kp, words, static_cast<const __nv_bfloat16 *>(table), gh, gw, C,
+                    static_cast<__nv_bfloat16 *>(pos));
 }
 
 cudaError_t launch_pad_cols(int dtype, const void *w, void *out, int n, int k, int kp,

@@ -55,8 +55,10 @@ cudaError_t launch_rope2d(int dtype, void *qkv, const int32_t *pos, int T, int H
                           const RopeFreqs &fr, cudaStream_t st);
 
 // patch embedding inputs (k_embed.cu)
-cudaError_t launch_patchify(int dtype, const ImageTable &tab, int n_images, long long max_tokens,
-                            const void *px, void *out, int p, int kp, cudaStream_t st);
+cudaError_t launch_embed_inputs(int dtype, const ImageTable &tab, int n_images,
+                                long long max_tokens, const void *px, void *patches, int p, int kp,
+                                const void *table, int gh, int gw, int C, void *pos,
+                                cudaStream_t st);
 cudaError_t launch_pad_cols(int dtype, const void *w, void *out, int n, int k, int kp,
                             cudaStream_t st);
 cudaError_t launch_pos_interp(int dtype, const ImageTable &tab, int n_images, long long max_tokens,

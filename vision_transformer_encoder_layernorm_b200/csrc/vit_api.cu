@@ -780,10 +780,14 @@ vit_status vit_pos_interp(vit_ctx *ctx, const void *pos_table, int table_h, int 
   }));
 }
 
-vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels, const int32_t *grids_hw_host,
-                           int n_images, int patch, const void *w_pe, const void *b_pe,
-                           const void *pos_table, int table_h, int table_w, void *y,
-                           void *workspace, size_t ws_bytes, void *stream) {
+// The embedding with a weight already in the GEMM's [C, Kp] layout: one
+// launch for both GEMM operands (patch rows and resized position rows), then
+// the GEMM, whose residual epilogue adds the bias and the position rows.
+static vit_status patch_embed_impl(vit_ctx *ctx, const void *pixels, const int32_t *grids_hw_host,
+                                   int n_images, int patch, const void *w_pad, const void *b_pe,
+                                   const void *pos_table, int table_h, int table_w, void *y,
+                                   void *workspace, size_t ws_bytes, bool pad_from,
+                                   const void *w_pe, void *stream) {
   if (!ctx || !pixels || !w_pe || !b_pe || !pos_table || !y || !workspace || table_h < 1 ||
       table_w < 1 || patch < 1 || patch > 32)
     return VIT_ERR_INVALID_ARG;
@@ -797,32 +801,63 @@ vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels, const int32_t *grid
     const void *ps[4] = {b_pe, pos_table, y, workspace};
     for (const void *q : ps)
       if (!aligned16(q)) return VIT_ERR_INVALID_ARG;
+    if (!pad_from && !aligned16(w_pad)) return VIT_ERR_INVALID_ARG;
   }
   const size_t e = esize(ctx->cfg);
   const int k = 3 * patch * patch, kp = embed_kp(patch);
   uint8_t *wsb = static_cast<uint8_t *>(workspace);
   void *patches = wsb;
-  void *w_pad = wsb + align256(size_t(T) * kp * e);
-  void *pos = static_cast<uint8_t *>(w_pad) + align256(size_t(C) * kp * e);
+  void *w_ws = wsb + align256(size_t(T) * kp * e);
+  void *pos = static_cast<uint8_t *>(w_ws) + align256(size_t(C) * kp * e);
   DeviceGuard g(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int dt = ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16;
   cudaError_t err = for_image_tables(grids_hw_host, n_images, [&](const ImageTable &tab, int n,
                                                                  long long max_t) {
-    cudaError_t r = counted(ctx, VIT_K_EMBED, st, [&] {
-      return launch_patchify(dt, tab, n, max_t, pixels, patches, patch, kp, st);
-    });
-    if (r != cudaSuccess) return r;
     return counted(ctx, VIT_K_EMBED, st, [&] {
-      return launch_pos_interp(dt, tab, n, max_t, pos_table, table_h, table_w, C, pos, st);
+      return launch_embed_inputs(dt, tab, n, max_t, pixels, patches, patch, kp, pos_table, table_h,
+                                 table_w, C, pos, st);
     });
   });
   if (err != cudaSuccess) return VIT_ERR_CUDA;
-  if (counted(ctx, VIT_K_EMBED, st, [&] { return launch_pad_cols(dt, w_pe, w_pad, C, k, kp, st); }))
-    return VIT_ERR_CUDA;
+  if (pad_from) {
+    if (counted(ctx, VIT_K_EMBED, st, [&] { return launch_pad_cols(dt, w_pe, w_ws, C, k, kp, st); }))
+      return VIT_ERR_CUDA;
+    w_pad = w_ws;
+  }
   // tokens = patches . w_pad^T + b_pe + interpolated table (residual epilogue)
   return cuda_status(run_linear(ctx, VIT_K_GEMM, patches, w_pad, epi_args(b_pe, pos, y), int(T), C,
                                 kp, kEpiResidual, st));
+}
+
+vit_status vit_patch_embed(vit_ctx *ctx, const void *pixels, const int32_t *grids_hw_host,
+                           int n_images, int patch, const void *w_pe, const void *b_pe,
+                           const void *pos_table, int table_h, int table_w, void *y,
+                           void *workspace, size_t ws_bytes, void *stream) {
+  return patch_embed_impl(ctx, pixels, grids_hw_host, n_images, patch, nullptr, b_pe, pos_table,
+                          table_h, table_w, y, workspace, ws_bytes, true, w_pe, stream);
+}
+
+vit_status vit_patch_embed_padded(vit_ctx *ctx, const void *pixels, const int32_t *grids_hw_host,
+                                  int n_images, int patch, const void *w_pad, const void *b_pe,
+                                  const void *pos_table, int table_h, int table_w, void *y,
+                                  void *workspace, size_t ws_bytes, void *stream) {
+  return patch_embed_impl(ctx, pixels, grids_hw_host, n_images, patch, w_pad, b_pe, pos_table,
+                          table_h, table_w, y, workspace, ws_bytes, false, w_pad, stream);
+}
+
+int vit_patch_kp(int patch) { return patch < 1 || patch > 32 ? 0 : embed_kp(patch); }
+
+vit_status vit_pad_patch_weight(vit_ctx *ctx, const void *w_pe, int patch, void *w_pad,
+                                void *stream) {
+  if (!ctx || !w_pe || !w_pad || patch < 1 || patch > 32) return VIT_ERR_INVALID_ARG;
+  if (!aligned16(w_pad)) return VIT_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int dt = ctx->cfg.dtype == VIT_F32 ? kF32 : kBF16;
+  return cuda_status(counted(ctx, VIT_K_EMBED, st, [&] {
+    return launch_pad_cols(dt, w_pe, w_pad, ctx->cfg.hidden, 3 * patch * patch, embed_kp(patch), st);
+  }));
 }
 
 // ---------------------------------------------------------------- MXFP8
