@@ -301,32 +301,27 @@ __device__ __forceinline__ void store_o_half(uint32_t o_addr, float l_sum, __nv_
 }
 
 // Maximum of the first `nvalid` of N consecutive TMEM columns of this
-// thread's lane (N % 8 == 0), read in pieces of at most 32 columns.
+// thread's lane (N % 4 == 0): all N columns in one load round trip (one
+// tcgen05.wait::ld), then two independent chains of 3-input maxima.
 template <int N>
 __device__ __forceinline__ float tmem_rowmax(uint32_t addr, int nvalid) {
-  float mx = -INFINITY;
-  int base = 0;
-  auto piece = [&](auto wc) {
-    constexpr int W = decltype(wc)::value;
-    uint32_t q[W];
-    __syncwarp();
-    tmem_ld_cols<W>(addr + base, q);
-    tmem_ld_wait();
-    if (nvalid - base < W) {
+  static_assert(N <= 56 && N % 8 == 0, "row width");
+  uint32_t q[N];
+  __syncwarp();
+  tmem_ld_cols<N>(addr, q);
+  tmem_ld_wait();
+  if (nvalid < N) {
 #pragma unroll
-      for (int i = 0; i < W; ++i)
-        if (base + i >= nvalid) q[i] = 0xFF800000u;
-    }
+    for (int i = 0; i < N; ++i)
+      if (i >= nvalid) q[i] = 0xFF800000u;
+  }
+  float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-    for (int i = 0; i + 1 < W; i += 2)
-      mx = fmax3(mx, __uint_as_float(q[i]), __uint_as_float(q[i + 1]));
-    base += W;
-  };
-  if constexpr (N >= 32) piece(std::integral_constant<int, 32>{});
-  if constexpr (N % 32 >= 16) piece(std::integral_constant<int, 16>{});
-  if constexpr (N % 16 >= 8) piece(std::integral_constant<int, 8>{});
-  static_assert(N <= 56 && N % 8 == 0, "row pieces");
-  return mx;
+  for (int i = 0; i + 3 < N; i += 4) {
+    a0 = fmax3(a0, __uint_as_float(q[i]), __uint_as_float(q[i + 1]));
+    a1 = fmax3(a1, __uint_as_float(q[i + 2]), __uint_as_float(q[i + 3]));
+  }
+  return fmaxf(a0, a1);
 }
 
 // Partial rows of a split item: this half's O columns (fp32, unnormalised;
@@ -788,8 +783,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const int nv_tile = ja < n_pre ? min(BK, prm.P - ja * BK) : min(BK, len - (ja - n_pre) * BK);
         const int nvalid = nv_tile - half * HC;  // valid keys among this thread's columns
         // the row max needs the other half's scores too: read them from TMEM
-        // in pieces and keep only their maximum (cheaper than a hand-off
-        // between the two threads of the row)
+        // and keep only their maximum (cheaper than a hand-off between the
+        // two threads of the row)
         const float m_other = tmem_rowmax<HC>(s_other, nv_tile - (half ^ 1) * HC);
         uint32_t s[HC];
         __syncwarp();
