@@ -801,9 +801,10 @@ def main():
         nxt["fp8_encoder"] = {"workload": "c2 stack (27 layers, 3900 patches) with the four "
                                           "projections in MXFP8, no merge",
                               "ms_per_step": t8, "patches_per_s": T / (t8 / 1e3),
-                              "launches_per_layer": 12,
-                              "note": "quantisation of every projection input is a separate "
-                                      "pass; graph replays, L2 flushed before each"}
+                              "launches_per_layer": 9,
+                              "note": "LayerNorms and fc1's epilogue write MXFP8 directly; the "
+                                      "attention output is quantised in its own pass; graph "
+                                      "replays, L2 flushed before each"}
         del mx_layers, mx_ws
         # MXFP8 block-scaled GEMM on fc1's shape (3900 x 4304 x 1152, bias +
         # GELU) with layer 0's fc1 weights quantised once outside the timed

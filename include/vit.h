@@ -388,6 +388,15 @@ VIT_API size_t vit_mx8_scale_bytes(int rows, int K);
 VIT_API vit_status vit_mx8_quantize(vit_ctx *ctx, const void *x, int rows, int K,
                                     void *codes, void *scales, void *stream);
 
+/* LayerNorm straight to MXFP8: codes, scales = vit_mx8_quantize(bf16 of
+ * vit_layernorm(x, gamma, beta)), bit for bit, in one launch (the FP8
+ * layer's LayerNorms).  x bf16 [rows, cols], gamma / beta [cols], eps as
+ * vit_layernorm.  cols a multiple of 4, at most 1536 (VIT_ERR_UNSUPPORTED
+ * beyond, or in an fp32 context); errors otherwise as vit_mx8_quantize. */
+VIT_API vit_status vit_layernorm_mx8(vit_ctx *ctx, const void *x, const void *gamma,
+                                     const void *beta, int rows, int cols, float eps, void *codes,
+                                     void *scales, void *stream);
+
 /* y bf16 [M, N] = epi(deq(A) deq(W)^T + bias) with A = (a_codes, a_scales)
  * [M, K] and W = (w_codes, w_scales) [N, K] (a PyTorch Linear weight,
  * quantised along K); bias bf16 [N] or NULL; residual bf16 [M, N] for
@@ -403,14 +412,19 @@ VIT_API vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void 
  * MXFP8 (reading: the pages list fp8 variants of dense checkpoints and put
  * FP16 / INT8 on the KLiteInfer road map, without a format; OCP MX v1.0
  * MXFP8 E4M3 is taken).  Per projection the input activation is quantised
- * along K (vit_mx8_quantize's rule) and multiplied with the weight's codes
- * by the block-scaled tensor-core GEMM (vit_linear_mx8); LayerNorm, RoPE
- * (a pass over the projection output), attention, GELU and the residual
- * adds are those of the bf16 layer.  Weights are quantised once by the
- * caller with vit_mx8_quantize (w_* [out, in] along in); the LayerNorm
- * vectors and biases stay bf16.  bf16 contexts only.
- * Workspace: vit_workspace_bytes_mx8 (the bf16 layer's buffers plus the
- * quantised activations).  Errors as vit_encoder_forward; the folded
+ * along K (vit_mx8_quantize's rule: the bf16 activation, quantised) and
+ * multiplied with the weight's codes by the block-scaled tensor-core GEMM
+ * (vit_linear_mx8); LayerNorm, RoPE (a pass over the projection output),
+ * attention, GELU and the residual adds are those of the bf16 layer.  The
+ * quantisation is fused where the producer holds whole 32-element groups:
+ * the two LayerNorms write MXFP8 directly (hidden <= 1536), and fc1's
+ * epilogue writes GELU's output as MXFP8 for fc2; the attention output has
+ * its own pass (its 72-wide heads split the groups).  Nine launches per
+ * layer.  Weights are quantised once by the caller with vit_mx8_quantize
+ * (w_* [out, in] along in); the LayerNorm vectors and biases stay bf16.
+ * bf16 contexts only.
+ * Workspace: vit_workspace_bytes_mx8 (the bf16 layer's buffers plus two
+ * quantised activations, K = hidden and K = MLP width).  Errors as vit_encoder_forward; the folded
  * LayerNorm and prefix K/V are not supported here (VIT_ERR_UNSUPPORTED). */
 typedef struct {
   const void *ln1_g, *ln1_b, *b_qkv, *b_o, *ln2_g, *ln2_b, *b_fc1, *b_fc2;  /* bf16 */

@@ -77,6 +77,48 @@ def test_mx8_quantize_bit_exact(ctx, rows, K):
     assert ctx.device_status() == 0
 
 
+LN_MX_CASES = [(3900, 1152), (257, 200), (130, 36), (7, 4), (129, 1536)]
+
+
+@pytest.mark.parametrize("rows,cols", LN_MX_CASES)
+def test_layernorm_mx8_equals_layernorm_then_quantise(ctx, rows, cols):
+    """vit_layernorm_mx8 gives the codes and scales of vit_mx8_quantize applied
+    to vit_layernorm's bf16 output, bit for bit (padding scales included),
+    across ragged row blocks, a partial last group and widths of 1 to 48
+    groups; and the codes match the oracle's quantiser on that output."""
+    x, _ = _t((rows, cols), 90 + cols, 3.0)
+    g, _ = _t((cols,), 91 + cols)
+    b, _ = _t((cols,), 92 + cols, 0.5)
+    y = torch.empty_like(x)
+    ctx.layernorm(x, y, g, b, eps=1e-6)
+    c0, s0 = _quantize(ctx, y, rows, cols)
+    c1 = torch.empty_like(c0)
+    s1 = torch.full_like(s0, 0xFF)  # every byte must be written (no 0xFF is a valid scale here)
+    ctx.layernorm_mx8(x, g, b, c1, s1, eps=1e-6)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    assert torch.equal(c0[:, :cols], c1[:, :cols])
+    assert torch.equal(s0, s1)
+    q_ref, s_ref = MX.mx_quantize(from_dev(y))
+    assert np.array_equal(c1.cpu().numpy()[:, :cols], q_ref)
+    assert np.array_equal(s1.cpu().numpy()[_scale_index(rows, cols)], s_ref)
+
+
+def test_layernorm_mx8_errors(ctx):
+    x, _ = _t((4, 1540), 95)
+    g, _ = _t((1540,), 96)
+    c = torch.empty((4, vit.mx8_row_bytes(1540)), dtype=torch.uint8, device="cuda")
+    sc = torch.empty(vit.mx8_scale_bytes(4, 1540), dtype=torch.uint8, device="cuda")
+    with pytest.raises(vit.VitError) as ei:
+        ctx.layernorm_mx8(x, g, g, c, sc)
+    assert ei.value.code == 3  # wider than 1536 columns: unsupported
+    x2, _ = _t((4, 6), 97)
+    g2, _ = _t((6,), 98)
+    with pytest.raises(vit.VitError) as ei:
+        ctx.layernorm_mx8(x2, g2, g2, c, sc)
+    assert ei.value.code == 3  # cols % 4 != 0
+
+
 GEMM_CASES = [
     # (M, N, K, epilogue): ragged M, several N tiles, K with a partial
     # 128-column block and a partial 32-element group; then fc1 of the

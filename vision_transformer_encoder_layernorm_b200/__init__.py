@@ -120,6 +120,7 @@ ABI_FUNCTIONS = {
     "vit_mx8_row_bytes": (ctypes.c_size_t, [_I]),
     "vit_mx8_scale_bytes": (ctypes.c_size_t, [_I, _I]),
     "vit_mx8_quantize": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "vit_layernorm_mx8": (_I, [_P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P, _P]),
     "vit_linear_mx8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "vit_get_last_device_status": (_I, [_P]),
     "vit_debug_lost_tx": (_I, [_P, ctypes.c_uint]),
@@ -360,6 +361,15 @@ class Context:
         rows, K = x.shape
         _check("vit_mx8_quantize", lib.vit_mx8_quantize(self._h, _ptr(x), rows, K, _ptr(codes),
                                                         _ptr(scales), _stream(stream)))
+
+    def layernorm_mx8(self, x, gamma, beta, codes, scales, eps=None, stream=None):
+        """vit_layernorm_mx8: LayerNorm of bf16 x [rows, cols] straight to MXFP8
+        codes / scales (the layout of mx8_quantize)."""
+        rows, cols = x.shape
+        e = self.cfg.ln_eps if eps is None else eps
+        _check("vit_layernorm_mx8", lib.vit_layernorm_mx8(self._h, _ptr(x), _ptr(gamma), _ptr(beta),
+                                                          rows, cols, e, _ptr(codes), _ptr(scales),
+                                                          _stream(stream)))
 
     def linear_mx8(self, a, w, bias, y, K, epi=EPI_BIAS, residual=None, stream=None):
         """y = epi(deq(A) deq(W)^T + bias) with a = (codes, scales) [M, K] and

@@ -146,10 +146,17 @@ __global__ void __launch_bounds__(256) embed_inputs_kernel(const __grid_constant
     const int ch = run / p, y = run - ch * p;
     const T *src = img + ((long long)ch * Hh + (long long)r * p + y) * W + (long long)c * p;
     T *dst = patches + (long long)(im.base + tok) * kp + ch * pp + y * p;
-    if (words) {
+    if (words) {  // all of the run's loads in flight before its stores (p <= 32)
       const uint32_t *s4 = reinterpret_cast<const uint32_t *>(src);
       uint32_t *d4 = reinterpret_cast<uint32_t *>(dst);
-      for (int i = 0; i < p / 2; ++i) d4[i] = __ldg(s4 + i);
+      const int nw = p / 2;
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < nw) w[i] = __ldg(s4 + i);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < nw) d4[i] = w[i];
     } else {
       for (int i = 0; i < p; ++i) dst[i] = src[i];
     }

@@ -24,6 +24,8 @@
 
 #include <atomic>
 
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 #include "mx8.h"
 #include "sm100.cuh"
@@ -324,6 +326,58 @@ __device__ __forceinline__ void stage_store_chunk(uint8_t *buf, const CUtensorMa
   }
 }
 
+// kEpiQuant: one thread's 32-column chunk of row `row` (bf16 values o) as
+// one MXFP8 group -- X = floor(log2 amax) - 8 clamped to [-127, 127], E4M3
+// codes of x 2^-X (nearest even, saturating) -- codes to ea.y viewed as
+// bytes, the scale byte into ea.q_scales' 512-byte blocks.  Threads of the
+// blocks' padding (rows past M, groups past N inside the last 128-column
+// block) write the padding scale 127.
+__device__ __forceinline__ void quant_store_chunk(const uint4 (&o)[4], const EpiArgs &ea, int row,
+                                                  int M, int col0, int N) {
+  if (row >= (M + 127) / 128 * 128 || col0 >= (N + 127) / 128 * 128) return;
+  const int g = col0 >> 5, rr = row & 127;
+  uint8_t &sc = ea.q_scales[(size_t(row >> 7) * ea.q_kblocks + (g >> 2)) * 512 + (rr & 31) * 16 +
+                            (rr >> 5) * 4 + (g & 3)];
+  if (row >= M || col0 >= N) {
+    sc = 127;
+    return;
+  }
+  const int n = min(32, N - col0);
+  float v[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w[4] = {o[q].x, o[q].y, o[q].z, o[q].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e] = bf16_lo(w[e]);
+      v[8 * q + 2 * e + 1] = bf16_hi(w[e]);
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, i < n ? fabsf(v[i]) : 0.f);
+  const int ef = int(__float_as_uint(amax) >> 23) & 0xFF;
+  const int X = ef == 0 ? -127 : min(max(ef - 127 - 8, -127), 127);
+  const float inv = __uint_as_float(uint32_t(127 - X) << 23);
+  uint32_t packed[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+    packed[q] = (lo & 0xFFFFu) | ((hi & 0xFFFFu) << 16);
+  }
+  uint8_t *cr = reinterpret_cast<uint8_t *>(ea.y) + size_t(row) * ea.q_row_bytes + col0;
+  if (n == 32) {  // q_row_bytes % 16 == 0 and col0 % 32 == 0: 16-byte aligned
+    reinterpret_cast<uint4 *>(cr)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    reinterpret_cast<uint4 *>(cr)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  } else {
+    for (int i = 0; i < n; ++i) cr[i] = uint8_t(packed[i >> 2] >> (8 * (i & 3)));
+  }
+  sc = uint8_t(X + 127);
+}
+
 // Epilogue of one accumulator (one output tile) by the 8 epilogue warps:
 // epilogue warp e (= warp - 2) drains TMEM lane quarter (warp & 3), i.e. one
 // row per thread (rows row0 .. row0 + 31 of the warp), and column half
@@ -468,7 +522,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem_acc, int warp, int l
       tmem_ld_wait();
       uint4 o[4];
       compute_chunk<EPI>(r, col0, N, ok, bias_w + i * 32, rv, sv, cv, mu, rstd, o, rs);
-      if constexpr (STAGED) {
+      if constexpr ((EPI & kEpiQuant) != 0) {
+        quant_store_chunk(o, ea, row, M, col0, N);
+      } else if constexpr (STAGED) {
         stage_store_chunk(ebuf, tm_y, o, lane, col0, row0, row0 < M && col0 < N);
       } else if (ok) {
         uint4 *yp = reinterpret_cast<uint4 *>(y + size_t(row) * N + col0);
@@ -1311,9 +1367,12 @@ static cudaError_t launch_mx8_bn(const CUtensorMap &ta, const CUtensorMap &tb,
 
 cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes,
                             const uint8_t *w_scales, const void *b, const void *res, void *y, int M,
-                            int N, int K, int epi, int num_sms, int *status, cudaStream_t st) {
+                            int N, int K, int epi, int num_sms, int *status, cudaStream_t st,
+                            uint8_t *y_scales) {
   if (M == 0 || N == 0) return cudaSuccess;
   constexpr int BN = 128;
+  if ((epi & kEpiQuant) && (epi != (kEpiGelu | kEpiQuant) || y_scales == nullptr))
+    return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
   if (encode_tensor_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K, M, mx8_row_bytes(K),
                            gemm::kMxBK, gemm::BM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
@@ -1329,10 +1388,16 @@ cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, con
   ea.bias = static_cast<const __nv_bfloat16 *>(b);
   ea.res = static_cast<const __nv_bfloat16 *>(res);
   ea.y = static_cast<__nv_bfloat16 *>(y);
+  ea.q_scales = y_scales;
+  ea.q_row_bytes = mx8_row_bytes(N);
+  ea.q_kblocks = (N + 127) / 128;
   switch (epi) {
     case kEpiGelu:
       return launch_mx8_bn<BN, kEpiGelu>(ta, tb, ty, a_scales, w_scales, ea, M, N, K, num_sms, status,
                                          st);
+    case kEpiGelu | kEpiQuant:
+      return launch_mx8_bn<BN, kEpiGelu | kEpiQuant>(ta, tb, ty, a_scales, w_scales, ea, M, N, K,
+                                                     num_sms, status, st);
     case kEpiResidual:
       return launch_mx8_bn<BN, kEpiResidual>(ta, tb, ty, a_scales, w_scales, ea, M, N, K, num_sms,
                                              status, st);

@@ -11,7 +11,9 @@
 // x * 2^-X is exact in fp32 (a power-of-two rescale that stays in range for
 // every bf16 input), so the conversion decides exactly as an fp64 reference.
 // The scale byte X + 127 is written straight into the 512-byte blocks the
-// GEMM copies into tensor memory (layout in mx8.h).
+// GEMM copies into tensor memory (layout in mx8.h); the threads run over the
+// blocks' whole padded shape, and those past the rows or groups write the
+// padding byte 127 (2^0), so no separate fill is needed.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -26,10 +28,15 @@ __global__ void __launch_bounds__(256) mx8_quantize_kernel(const __nv_bfloat16 *
                                                            uint8_t *__restrict__ scales) {
   pdl_trigger();
   pdl_wait();
-  const int groups = (K + 31) / 32;
+  const int groups = (K + 31) / 32, pgroups = 4 * k_blocks, prows = (rows + 127) / 128 * 128;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= (long long)rows * groups) return;
-  const int r = int(gid / groups), j = int(gid - (long long)r * groups);
+  if (gid >= (long long)prows * pgroups) return;
+  const int r = int(gid / pgroups), j = int(gid - (long long)r * pgroups);
+  if (r >= rows || j >= groups) {  // a padding entry of the scale blocks
+    const int rb = r >> 7, rr = r & 127, kb = j >> 2, jj = j & 3;
+    scales[(size_t(rb) * k_blocks + kb) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + jj] = 127;
+    return;
+  }
   const int k0 = j * 32, n = min(32, K - k0);
   const __nv_bfloat16 *xr = x + size_t(r) * K + k0;
   float v[32];
@@ -84,10 +91,7 @@ __global__ void __launch_bounds__(256) mx8_quantize_kernel(const __nv_bfloat16 *
 cudaError_t launch_mx8_quantize(const void *x, int rows, int K, uint8_t *codes, uint8_t *scales,
                                 cudaStream_t st) {
   if (rows == 0 || K == 0) return cudaSuccess;
-  // padding entries of the scale blocks (rows past `rows`, groups past K) = 2^0
-  cudaError_t e = cudaMemsetAsync(scales, 127, mx8_scale_bytes(rows, K), st);
-  if (e != cudaSuccess) return e;
-  const long long threads = (long long)rows * ((K + 31) / 32);
+  const long long threads = (long long)((rows + 127) / 128 * 128) * (4 * ((K + 127) / 128));
   const int block = 256;
   const long long grid = (threads + block - 1) / block;
   if (grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;

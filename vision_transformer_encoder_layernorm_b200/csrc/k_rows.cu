@@ -5,6 +5,8 @@
 // row-major batched tokens, 2D RoPE, 2x2 spatial merge.  The pages' LayerNorm
 // is one block per row with a two-pass reduction; here one warp owns a row,
 // holds it in registers (one HBM read, one write) and reduces with shuffles.
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 
 namespace vit {
@@ -179,6 +181,137 @@ __global__ void __launch_bounds__(256) layernorm_block_kernel(
       yr[c] = V::pack(o);
     }
   }
+}
+
+// LayerNorm whose output goes straight to MXFP8 (bf16 only): the row is
+// normalised exactly as layernorm_warp_kernel does, each result rounded to
+// bf16 -- the value the plain kernel would store -- and then quantised as
+// mx8_quantize_kernel does (X = floor(log2 amax) - 8 per 32-element group,
+// clamped to [-127, 127]; E4M3 codes of x 2^-X, nearest even, saturating).
+// Lane l holds 4-element vectors l, l + 32, ..., so a group is 8 lanes'
+// vectors of one iteration and its amax takes three shuffles.  The grid
+// covers the scale blocks' padded rows: a warp past the last row writes its
+// padding scale bytes (127) and stops; every row writes the padding bytes
+// of groups past the last column.
+template <int MAXV>
+__global__ void __launch_bounds__(256) layernorm_mx8_kernel(
+    const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ gamma,
+    const __nv_bfloat16 *__restrict__ beta, int rows, int cols, float eps,
+    uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, size_t row_bytes, int k_blocks) {
+  using V = Vec4<__nv_bfloat16>;
+  using R = V::raw;
+  extern __shared__ __align__(16) unsigned char ln_smem[];
+  pdl_trigger();
+  pdl_wait();
+  const int nvec = cols >> 2;
+  const int groups = (cols + 31) / 32, pgroups = 4 * k_blocks;
+  R *sg = reinterpret_cast<R *>(ln_smem);
+  R *sb = sg + nvec;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  const bool active = row < rows;
+  auto scale_at = [&](int g) -> uint8_t & {
+    const int rb = row >> 7, rr = row & 127, kb = g >> 2, jj = g & 3;
+    return scales[(size_t(rb) * k_blocks + kb) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + jj];
+  };
+  const R *xr = reinterpret_cast<const R *>(x + size_t(active ? row : 0) * cols);
+  float v[MAXV][4];
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (active && c < nvec) {
+      V::unpack(xr[c], v[i]);
+    } else {
+      v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.f;
+    }
+  }
+  const R *gr = reinterpret_cast<const R *>(gamma);
+  const R *br = reinterpret_cast<const R *>(beta);
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    sg[i] = __ldg(gr + i);
+    sb[i] = __ldg(br + i);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s / float(cols);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nvec) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d = v[i][e] - mean;
+        q += d * d;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  const float rstd = 1.0f / sqrtf(q / float(cols) + eps);
+  __syncthreads();
+  if (row >= (rows + 127) / 128 * 128) return;
+  if (!active) {  // a padding row of the last row block
+    for (int g = lane; g < pgroups; g += 32) scale_at(g) = 127;
+    return;
+  }
+  for (int g = groups + lane; g < pgroups; g += 32) scale_at(g) = 127;
+  uint32_t *cr = reinterpret_cast<uint32_t *>(codes + size_t(row) * row_bytes);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    if (32 * i >= nvec) break;  // the same for the whole warp
+    const int c = lane + 32 * i;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    if (c < nvec) {
+      float g[4], b[4];
+      V::unpack(sg[c], g);
+      V::unpack(sb[c], b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = (v[i][e] - mean) * rstd * g[e] + b[e];
+      V::unpack(V::pack(o), o);  // the bf16 value the plain kernel stores
+    }
+    float amax = fmaxf(fmaxf(fabsf(o[0]), fabsf(o[1])), fmaxf(fabsf(o[2]), fabsf(o[3])));
+#pragma unroll
+    for (int m = 1; m < 8; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    const int ef = int(__float_as_uint(amax) >> 23) & 0xFF;
+    const int X = ef == 0 ? -127 : min(max(ef - 127 - 8, -127), 127);
+    const float inv = __uint_as_float(uint32_t(127 - X) << 23);
+    if (c < nvec) {
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(o[0] * inv, o[1] * inv),
+                                                   __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(o[2] * inv, o[3] * inv),
+                                                   __NV_SATFINITE, __NV_E4M3);
+      cr[c] = (lo & 0xFFFFu) | ((hi & 0xFFFFu) << 16);
+      if ((lane & 7) == 0) scale_at(c >> 3) = uint8_t(X + 127);
+    }
+  }
+}
+
+cudaError_t launch_layernorm_mx8(const void *x, const void *g, const void *b, int rows, int cols,
+                                 float eps, uint8_t *codes, uint8_t *scales, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  const int nvec = cols / 4;
+  if (cols % 4 || nvec > 32 * 12) return cudaErrorInvalidValue;
+  const int warps = 8;
+  const int prows = (rows + 127) / 128 * 128;
+  dim3 grid((prows + warps - 1) / warps), block(32 * warps);
+  const size_t smem = 2 * size_t(nvec) * sizeof(uint2);
+  auto xp = static_cast<const __nv_bfloat16 *>(x);
+  auto gp = static_cast<const __nv_bfloat16 *>(g);
+  auto bp = static_cast<const __nv_bfloat16 *>(b);
+  const size_t rb = (size_t(cols) + 15) / 16 * 16;
+  const int kb = (cols + 127) / 128;
+  if (nvec <= 32 * 4)
+    return launch_pdl(layernorm_mx8_kernel<4>, grid, block, smem, st, 1, xp, gp, bp, rows, cols,
+                      eps, codes, scales, rb, kb);
+  if (nvec <= 32 * 9)
+    return launch_pdl(layernorm_mx8_kernel<9>, grid, block, smem, st, 1, xp, gp, bp, rows, cols,
+                      eps, codes, scales, rb, kb);
+  return launch_pdl(layernorm_mx8_kernel<12>, grid, block, smem, st, 1, xp, gp, bp, rows, cols,
+                    eps, codes, scales, rb, kb);
 }
 
 template <typename T>

@@ -47,6 +47,11 @@ struct SeqArgs {
 
 cudaError_t launch_layernorm(int dtype, const void *x, void *y, const void *g, const void *b,
                              int rows, int cols, float eps, cudaStream_t st);
+// LayerNorm of bf16 rows straight to MXFP8 codes and scales (layout as
+// launch_mx8_quantize; the bf16-rounded LayerNorm quantised); cols % 4 == 0,
+// cols <= 1536.
+cudaError_t launch_layernorm_mx8(const void *x, const void *g, const void *b, int rows, int cols,
+                                 float eps, uint8_t *codes, uint8_t *scales, cudaStream_t st);
 cudaError_t launch_merge2x2(const ImageTable &tab, int n_images, const void *x, void *y,
                             size_t row_bytes, long long max_out_tokens, cudaStream_t st);
 cudaError_t launch_positions(const ImageTable &tab, int n_images, int cu_offset_index,
@@ -78,6 +83,11 @@ constexpr int kEpiLn = 4;
 // The output rows' statistics, per slice of the columns one epilogue warp
 // writes, go to EpiArgs::stats_out (for a later kEpiLn GEMM on this output).
 constexpr int kEpiStats = 8;
+// MXFP8 output (MXFP8 GEMM only): each 32-column chunk of a row, rounded to
+// bf16, is quantised as launch_mx8_quantize does; codes go to y viewed as
+// bytes with row stride q_row_bytes, scales to q_scales (its 512-byte blocks,
+// padding entries 127)
+constexpr int kEpiQuant = 16;
 
 // Per-row statistics of a row's column slices: slice j covers columns
 // [j w, min((j + 1) w, n)); entry (mean, M2) = mean of the slice and the sum
@@ -102,6 +112,11 @@ struct EpiArgs {
   // kEpiStats: slice statistics of the (bf16-rounded) output rows, slice
   // width = half the tile width (gemm_stats_width)
   SliceStats stats_out;
+  // kEpiQuant: scales of the MXFP8 output, row stride of its codes, and its
+  // 128-column blocks
+  uint8_t *q_scales;
+  size_t q_row_bytes;
+  int q_kblocks;
 };
 
 // Arguments of the RoPE epilogue: the GEMM's tile width is 2 * head_dim so

@@ -27,9 +27,12 @@ cudaError_t launch_mx8_quantize(const void *x, int rows, int K, uint8_t *codes, 
                                 cudaStream_t st);
 
 // y[M, N] (bf16) = epi(deq(A) . deq(W)^T + b): A codes/scales [M, K], W
-// codes/scales [N, K]; epi as launch_gemm_tc (bias, GELU, residual).
+// codes/scales [N, K]; epi as launch_gemm_tc (bias, GELU, residual).  With
+// kEpiGelu | kEpiQuant the output is MXFP8 instead: codes to y [M,
+// mx8_row_bytes(N)] and scales to y_scales [mx8_scale_bytes(M, N)].
 cudaError_t launch_gemm_mx8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes,
                             const uint8_t *w_scales, const void *b, const void *res, void *y, int M,
-                            int N, int K, int epi, int num_sms, int *status, cudaStream_t st);
+                            int N, int K, int epi, int num_sms, int *status, cudaStream_t st,
+                            uint8_t *y_scales = nullptr);
 
 }  // namespace vit

@@ -880,6 +880,24 @@ vit_status vit_mx8_quantize(vit_ctx *ctx, const void *x, int rows, int K, void *
   }));
 }
 
+vit_status vit_layernorm_mx8(vit_ctx *ctx, const void *x, const void *gamma, const void *beta,
+                             int rows, int cols, float eps, void *codes, void *scales,
+                             void *stream) {
+  if (!ctx || !x || !gamma || !beta || !codes || !scales || rows < 0 || cols < 0)
+    return VIT_ERR_INVALID_ARG;
+  if (ctx->cfg.dtype != VIT_BF16 || cols % 4 || cols > 1536) return VIT_ERR_UNSUPPORTED;
+  const void *ps[5] = {x, gamma, beta, codes, scales};
+  for (const void *q : ps)
+    if (!aligned16(q)) return VIT_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return VIT_OK;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(counted(ctx, VIT_K_LAYERNORM, st, [&] {
+    return launch_layernorm_mx8(x, gamma, beta, rows, cols, eps, static_cast<uint8_t *>(codes),
+                                static_cast<uint8_t *>(scales), st);
+  }));
+}
+
 vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void *a_scales,
                           const void *w_codes, const void *w_scales, const void *bias,
                           const void *residual, void *y, int M, int N, int K, vit_epilogue epi,
@@ -910,11 +928,15 @@ vit_status vit_linear_mx8(vit_ctx *ctx, const void *a_codes, const void *a_scale
 // ---------------------------------------------------------------- FP8 layers
 namespace {
 
-// the bf16 layer's workspace, then the quantised activation (codes and
-// scales sized for the widest K, the MLP width)
+// the bf16 layer's workspace, then two quantised activations: the inputs of
+// the QKV, out and fc1 projections (K = hidden), and fc1's output, written
+// quantised by its epilogue as fc2's input (K = MLP width)
+size_t mx8_act_bytes(int T, int K) {
+  return align256(size_t(T) * mx8_row_bytes(K)) + align256(mx8_scale_bytes(T, K));
+}
 size_t mx8_extra(const vit_config &c, int T) {
-  const int kmax = (c.flags & VIT_FLAG_NO_MLP) ? c.hidden : std::max(c.hidden, c.mlp);
-  return align256(size_t(T) * mx8_row_bytes(kmax)) + align256(mx8_scale_bytes(T, kmax));
+  return mx8_act_bytes(T, c.hidden) +
+         ((c.flags & VIT_FLAG_NO_MLP) ? size_t(0) : mx8_act_bytes(T, c.mlp));
 }
 
 vit_status check_layer_weights_mx8(const vit_config &c, const vit_layer_weights_mx8 *w) {
@@ -935,32 +957,40 @@ vit_status check_layer_weights_mx8(const vit_config &c, const vit_layer_weights_
 // One FP8 layer (all arguments validated).  aq / asc: quantised activation.
 vit_status layer_mx8_impl(vit_ctx *ctx, const vit_layer_weights_mx8 *w, const void *x, void *y,
                           const vit_seqs *seqs, const Workspace &ws, uint8_t *aq, uint8_t *asc,
-                          cudaStream_t st) {
+                          uint8_t *gq, uint8_t *gsc, cudaStream_t st) {
   const vit_config &c = ctx->cfg;
   const int T = seqs->total_tokens, C = c.hidden, F = c.mlp;
   const bool rope = !(c.flags & VIT_FLAG_NO_ROPE) && seqs->pos_rc != nullptr;
   const bool no_mlp = (c.flags & VIT_FLAG_NO_MLP) != 0;
   const float scale = 1.0f / sqrtf(float(c.head_dim));
-  auto ln = [&](const void *in, const void *g, const void *b) {
-    return counted(ctx, VIT_K_LAYERNORM, st, [&] {
-      return launch_layernorm(kBF16, in, ws.h, g, b, T, C, c.ln_eps, st);
-    });
-  };
   auto quant = [&](const void *a, int K) {
     return counted(ctx, VIT_K_MX8_QUANTIZE, st,
                    [&] { return launch_mx8_quantize(a, T, K, aq, asc, st); });
   };
-  auto gemm = [&](int kind, const void *wc, const void *wsc, const void *b, const void *res,
-                  void *out, int N, int K, int epi) {
+  // LayerNorm straight to MXFP8 (one launch) where the row fits a warp's
+  // registers, else LayerNorm then the quantiser
+  auto ln_q = [&](const void *in, const void *g, const void *b) {
+    if (C <= 1536)
+      return counted(ctx, VIT_K_LAYERNORM, st, [&] {
+        return launch_layernorm_mx8(in, g, b, T, C, c.ln_eps, aq, asc, st);
+      });
+    cudaError_t e = counted(ctx, VIT_K_LAYERNORM, st, [&] {
+      return launch_layernorm(kBF16, in, ws.h, g, b, T, C, c.ln_eps, st);
+    });
+    return e != cudaSuccess ? e : quant(ws.h, C);
+  };
+  auto gemm = [&](int kind, const uint8_t *a, const uint8_t *asf, const void *wc, const void *wsc,
+                  const void *b, const void *res, void *out, int N, int K, int epi,
+                  uint8_t *out_sc = nullptr) {
     return counted(ctx, kind, st, [&] {
-      return launch_gemm_mx8(aq, asc, static_cast<const uint8_t *>(wc),
+      return launch_gemm_mx8(a, asf, static_cast<const uint8_t *>(wc),
                              static_cast<const uint8_t *>(wsc), b, res, out, T, N, K, epi,
-                             ctx->num_sms, ctx->d_status, st);
+                             ctx->num_sms, ctx->d_status, st, out_sc);
     });
   };
-  if (ln(x, w->ln1_g, w->ln1_b) || quant(ws.h, C) ||
-      gemm(VIT_K_GEMM_QKV, w->w_qkv_codes, w->w_qkv_scales, w->b_qkv, nullptr, ws.qkv, 3 * C, C,
-           kEpiBias))
+  if (ln_q(x, w->ln1_g, w->ln1_b) ||
+      gemm(VIT_K_GEMM_QKV, aq, asc, w->w_qkv_codes, w->w_qkv_scales, w->b_qkv, nullptr, ws.qkv,
+           3 * C, C, kEpiBias))
     return VIT_ERR_CUDA;
   if (rope && counted(ctx, VIT_K_ROPE, st, [&] {
         return launch_rope2d(kBF16, ws.qkv, seqs->pos_rc, T, c.heads, c.head_dim, ctx->fr, st);
@@ -968,15 +998,15 @@ vit_status layer_mx8_impl(vit_ctx *ctx, const vit_layer_weights_mx8 *w, const vo
     return VIT_ERR_CUDA;
   const SeqArgs sa = to_seq_args(seqs, false);
   if (run_attention(ctx, ws.qkv, ws.attn, sa, scale, st)) return VIT_ERR_CUDA;
-  if (quant(ws.attn, C) || gemm(VIT_K_GEMM_OUT, w->w_o_codes, w->w_o_scales, w->b_o, x,
+  if (quant(ws.attn, C) || gemm(VIT_K_GEMM_OUT, aq, asc, w->w_o_codes, w->w_o_scales, w->b_o, x,
                                 no_mlp ? y : ws.x1, C, C, kEpiResidual))
     return VIT_ERR_CUDA;
   if (no_mlp) return VIT_OK;
-  if (ln(ws.x1, w->ln2_g, w->ln2_b) || quant(ws.h, C) ||
-      gemm(VIT_K_GEMM_FC1, w->w_fc1_codes, w->w_fc1_scales, w->b_fc1, nullptr, ws.g, F, C,
-           kEpiGelu) ||
-      quant(ws.g, F) ||
-      gemm(VIT_K_GEMM_FC2, w->w_fc2_codes, w->w_fc2_scales, w->b_fc2, ws.x1, y, C, F,
+  // fc1's epilogue writes GELU(.) as MXFP8 codes and scales: fc2's input
+  if (ln_q(ws.x1, w->ln2_g, w->ln2_b) ||
+      gemm(VIT_K_GEMM_FC1, aq, asc, w->w_fc1_codes, w->w_fc1_scales, w->b_fc1, nullptr, gq, F, C,
+           kEpiGelu | kEpiQuant, gsc) ||
+      gemm(VIT_K_GEMM_FC2, gq, gsc, w->w_fc2_codes, w->w_fc2_scales, w->b_fc2, ws.x1, y, C, F,
            kEpiResidual))
     return VIT_ERR_CUDA;
   return VIT_OK;
@@ -1007,15 +1037,17 @@ vit_status vit_encoder_forward_mx8(vit_ctx *ctx, const vit_layer_weights_mx8 *la
   DeviceGuard g(ctx->device);
   Workspace ws;
   const size_t base = workspace_layout(ctx->cfg, T, &ws, workspace, 0);
-  const int kmax = (ctx->cfg.flags & VIT_FLAG_NO_MLP) ? ctx->cfg.hidden
-                                                      : std::max(ctx->cfg.hidden, ctx->cfg.mlp);
+  const int C = ctx->cfg.hidden, F = ctx->cfg.mlp;
   uint8_t *aq = static_cast<uint8_t *>(workspace) + base;
-  uint8_t *asc = aq + align256(size_t(T) * mx8_row_bytes(kmax));
+  uint8_t *asc = aq + align256(size_t(T) * mx8_row_bytes(C));
+  uint8_t *gq = aq + mx8_act_bytes(T, C);  // used only with the MLP
+  uint8_t *gsc = gq + align256(size_t(T) * mx8_row_bytes(F));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int i = 0; i < n_layers; ++i) {
     const void *in = i == 0 ? x : ws.act[(i - 1) & 1];
     void *out = i == n_layers - 1 ? y : ws.act[i & 1];
-    if ((s = layer_mx8_impl(ctx, &layers[i], in, out, seqs, ws, aq, asc, st)) != VIT_OK) return s;
+    if ((s = layer_mx8_impl(ctx, &layers[i], in, out, seqs, ws, aq, asc, gq, gsc, st)) != VIT_OK)
+      return s;
   }
   return VIT_OK;
 }
