@@ -386,7 +386,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // unit).  x = j + f with j = round(x) (the 1.5 * 2^23 shift trick) and
 // f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted in this project
 // (iteratively reweighted least squares on Chebyshev nodes, max relative
-// error 7.5e-5 on [-1/2, 1/2]); 2^j inserted into the exponent field.
+// error 7.5e-5 on [-1/2, 1/2]; fit_exp2_poly.py beside this file reproduces
+// the coefficients); 2^j inserted into the exponent field.
 // x is clamped at -125 so the exponent never leaves the normal range.
 __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float &y0, float &y1) {
   float a, b;
