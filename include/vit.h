@@ -234,8 +234,11 @@ VIT_API void vit_graph_destroy(vit_graph *g);
 /* Bidirectional multi-head attention over packed sequences ("视觉算子":
  * softmax(Q K^T * scale) V per head and sequence).  qkv [T, 3, H, d]
  * (the QKV projection's output layout), o [T, H, d].  With seqs->pos_rc the
- * kernel rotates Q and K by 2D RoPE as it loads them.  scale <= 0 selects
- * 1/sqrt(d). */
+ * kernel rotates Q and K by 2D RoPE as it loads them, every key tile once
+ * per query-tile pair that reads it: a convenience for unrotated inputs,
+ * about six times slower at head_dim 72 (3900 tokens: 733 against 121 us)
+ * than rotating once (vit_rope2d, or the layer's QKV epilogue) and calling
+ * without positions.  scale <= 0 selects 1/sqrt(d). */
 VIT_API vit_status vit_attention(vit_ctx *ctx, const void *qkv, void *o,
                          const vit_seqs *seqs, float scale, void *stream);
 
