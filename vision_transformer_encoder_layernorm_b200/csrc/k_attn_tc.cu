@@ -111,6 +111,7 @@ static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
 struct Params {
   int H, C, Hkv, P, n_pairs, n_seqs;
+  int tpi;               // query tiles per item: 2, or 1 when the items would not fill the SMs
   float scale_log2;      // softmax scale * log2(e)
   const int32_t *cu;
   const int32_t *pos;
@@ -135,7 +136,7 @@ struct SkTable {
   int bw[kMaxSkCtas + 1], bj[kMaxSkCtas + 1];
 };
 
-// One work item: query tiles [q0, q0 + 256) of head h of sequence seq.
+// One work item: query tiles [q0, q0 + tpi * 128) of head h of sequence seq.
 struct Item {
   int seq, h, hk, seg0, len, q0, n_tiles_q, n_kv;
 };
@@ -150,9 +151,9 @@ __device__ __forceinline__ bool decode_item(int w, const Params &prm, int bk, It
   it.hk = it.h / (prm.H / prm.Hkv);
   it.seg0 = prm.cu[it.seq];
   it.len = prm.cu[it.seq + 1] - it.seg0;
-  it.q0 = pair * 2 * kBlockQ;
+  it.q0 = pair * prm.tpi * kBlockQ;
   if (it.q0 >= it.len) return false;
-  it.n_tiles_q = (it.len - it.q0 > kBlockQ) ? 2 : 1;
+  it.n_tiles_q = (prm.tpi == 2 && it.len - it.q0 > kBlockQ) ? 2 : 1;
   const int n_pre = prm.P > 0 ? (prm.P + bk - 1) / bk : 0;
   it.n_kv = n_pre + (it.len + bk - 1) / bk;
   return true;
@@ -1108,7 +1109,13 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
   prm.C = C;
   prm.Hkv = Hkv;
   prm.P = P;
-  prm.n_pairs = (s.max_seqlen + 2 * attn::kBlockQ - 1) / (2 * attn::kBlockQ);
+  // Items of one query tile when even those fit in one round over the SMs
+  // (short sequences: twice the CTAs at work, each tile's softmax without a
+  // second tile beside it); else pairs sharing each K/V tile.
+  const long long single_items =
+      (long long)((s.max_seqlen + attn::kBlockQ - 1) / attn::kBlockQ) * H * s.n_seqs;
+  prm.tpi = single_items <= num_sms ? 1 : 2;
+  prm.n_pairs = (s.max_seqlen + prm.tpi * attn::kBlockQ - 1) / (prm.tpi * attn::kBlockQ);
   prm.n_seqs = s.n_seqs;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.cu = s.cu_seqlens;
@@ -1127,7 +1134,8 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
   int grid = (persistent && n_items > num_sms) ? num_sms : n_items;
   attn::SkTable sk;
   sk.n = 0;
-  if (d == 72 && s.n_seqs == 1 && part && cnt && persistent && attn_split_enabled() &&
+  if (d == 72 && s.n_seqs == 1 && part && cnt && persistent && prm.tpi == 2 &&
+      attn_split_enabled() &&
       !build_split_table(s, H, prm.n_pairs, std::min(num_sms, attn::kMaxSkCtas), sk))
     sk.n = 0;
   if (sk.n) grid = sk.n;
