@@ -23,8 +23,8 @@
 //            K rows; head_dim 72: ones in V's column 72, the row sums), so
 //            the next item's first S overlaps the softmax epilogue
 //   4-11     softmax of query tile 0, 12-19 of query tile 1: two threads per
-//            query row, one per half of the key tile's score columns; the
-//            pair swaps partial row maxima through shared memory
+//            query row, one per half of the key tile's score columns; each
+//            also reads the other half's scores from TMEM for the row max
 // Per query tile t, TMEM holds S_t (fp32 scores of one key tile), P_t (bf16
 // probabilities, its own columns) and O_t.  Because P does not overwrite S,
 // the MMA warp issues S_t(j+1) = Q_t K_{j+1}^T as soon as the softmax threads
