@@ -112,6 +112,7 @@ static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 struct Params {
   int H, C, Hkv, P, n_pairs, n_seqs;
   int tpi;               // query tiles per item: 2, or 1 when the items would not fill the SMs
+  int snake;             // packed sequences: items by descending length, dealt out in a snake
   float scale_log2;      // softmax scale * log2(e)
   const int32_t *cu;
   const int32_t *pos;
@@ -159,6 +160,61 @@ __device__ __forceinline__ bool decode_item(int w, const Params &prm, int bk, It
   return true;
 }
 
+// Packed sequences of different lengths (snake schedule): the items are
+// listed by descending sequence length (a sequence's items pair-major, heads
+// inner) and dealt to the CTAs in a snake, round r going 0..G-1 for even r
+// and G-1..0 for odd r, so the long items spread evenly and the short ones
+// fill in behind them.  The CTA's warp 0 builds the order in shared
+// memory: ord[i] = i-th longest sequence, pre[i] = items before it.
+constexpr int kMaxSnakeSeqs = 64;
+struct SnakeTab {
+  int len[kMaxSnakeSeqs];
+  int ord[kMaxSnakeSeqs];
+  int pre[kMaxSnakeSeqs + 1];
+};
+
+// Warp 0: each lane ranks sequences lane and lane + 32 by length
+// (descending, ties by index), then lane 0 sums the items in that order.
+__device__ __forceinline__ void build_snake(const Params &prm, SnakeTab *tab, int lane) {
+  const int n = prm.n_seqs;
+  for (int i = lane; i < n; i += 32) tab->len[i] = prm.cu[i + 1] - prm.cu[i];
+  __syncwarp();
+  for (int i = lane; i < n; i += 32) {
+    const int li = tab->len[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const int lj = tab->len[j];
+      rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    tab->ord[rank] = i;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    tab->pre[0] = 0;
+    for (int i = 0; i < n; ++i)
+      tab->pre[i + 1] =
+          tab->pre[i] + (tab->len[tab->ord[i]] + 2 * kBlockQ - 1) / (2 * kBlockQ) * prm.H;
+  }
+}
+
+// Item w of the snake order (always a real item).
+__device__ __forceinline__ void decode_snake(int w, const Params &prm, const SnakeTab &tab, int bk,
+                                             Item &it) {
+  int i = 0;
+  while (tab.pre[i + 1] <= w) ++i;
+  const int local = w - tab.pre[i];
+  const int pair = local / prm.H;
+  it.seq = tab.ord[i];
+  it.h = local - pair * prm.H;
+  it.hk = it.h / (prm.H / prm.Hkv);
+  it.seg0 = prm.cu[it.seq];
+  it.len = tab.len[it.seq];
+  it.q0 = pair * 2 * kBlockQ;
+  it.n_tiles_q = (it.len - it.q0 > kBlockQ) ? 2 : 1;
+  const int n_pre = prm.P > 0 ? (prm.P + bk - 1) / bk : 0;
+  it.n_kv = n_pre + (it.len + bk - 1) / bk;
+}
+
 // A work unit: key tiles [j0, j1) of item w.
 struct Unit {
   Item it;
@@ -169,8 +225,18 @@ struct Unit {
 // k-th unit of this CTA: 0 = no more units, 1 = unit, 2 = nothing to do for
 // this k (an empty pair slot)
 __device__ __forceinline__ int get_unit(int k, const Params &prm, const SkTable &sk, int bk,
-                                        Unit &u) {
+                                        Unit &u, const SnakeTab *snake) {
   const int c = blockIdx.x;
+  if (prm.snake) {
+    const int G = gridDim.x;
+    u.w = k * G + ((k & 1) ? G - 1 - c : c);
+    if (u.w >= snake->pre[prm.n_seqs]) return 0;  // rounds only grow: no more items
+    decode_snake(u.w, prm, *snake, bk, u.it);
+    u.j0 = 0;
+    u.j1 = u.it.n_kv;
+    u.whole = true;
+    return 1;
+  }
   if (sk.n == 0) {
     u.w = c + k * gridDim.x;
     if (u.w >= prm.n_pairs * prm.H * prm.n_seqs) return 0;
@@ -426,6 +492,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   pdl_wait();
   const int n_pre = prm.P > 0 ? (prm.P + BK - 1) / BK : 0;
 
+  // the snake order's table sits in the row-sum exchange region, unused at
+  // head_dim 72 (the only persistent kernel that takes the snake schedule)
+  SnakeTab *snake = reinterpret_cast<SnakeTab *>(smem + CF::kXOff);
+  static_assert(sizeof(SnakeTab) <= 4096, "snake table");
+  if (warp == 0 && prm.snake) build_snake(prm, snake, lane);
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
@@ -487,7 +558,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       uint32_t issued = 0, issued_par = 0, q_issued = 0;
       for (int k = 0; ok; ++k) {
         Unit u;
-        const int gu = get_unit(k, prm, sk, BK, u);
+        const int gu = get_unit(k, prm, sk, BK, u, snake);
         if (gu == 0) break;
         if (gu == 2) continue;
         const Item &it = u.it;
@@ -598,7 +669,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       uint32_t act = 0;   // items in which this query tile was active
       for (int k = 0; ok; ++k) {
         Unit u;
-        const int gu = get_unit(k, prm, sk, BK, u);
+        const int gu = get_unit(k, prm, sk, BK, u, snake);
         if (gu == 0) break;
         if (gu == 2) continue;
         const Item &it = u.it;
@@ -658,7 +729,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       Unit u;
-      const int gu = get_unit(k, prm, sk, BK, u);
+      const int gu = get_unit(k, prm, sk, BK, u, snake);
       if (gu == 0) break;
       if (gu == 2) continue;
       const Item &it = u.it;
@@ -767,7 +838,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     uint32_t pd = 0;    // split units (tile 0: phases of part_done)
     for (int k = 0; ok; ++k) {
       Unit u;
-      const int gu = get_unit(k, prm, sk, BK, u);
+      const int gu = get_unit(k, prm, sk, BK, u, snake);
       if (gu == 0) break;
       if (gu == 2) continue;
       const Item &it = u.it;
@@ -1116,6 +1187,7 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
       (long long)((s.max_seqlen + attn::kBlockQ - 1) / attn::kBlockQ) * H * s.n_seqs;
   prm.tpi = single_items <= num_sms ? 1 : 2;
   prm.n_pairs = (s.max_seqlen + prm.tpi * attn::kBlockQ - 1) / (prm.tpi * attn::kBlockQ);
+  prm.snake = 0;  // set below for packed sequences on the persistent kernel
   prm.n_seqs = s.n_seqs;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.cu = s.cu_seqlens;
@@ -1139,6 +1211,10 @@ cudaError_t launch_attention_tc(const void *qkv, void *o, const SeqArgs &s, int 
       !build_split_table(s, H, prm.n_pairs, std::min(num_sms, attn::kMaxSkCtas), sk))
     sk.n = 0;
   if (sk.n) grid = sk.n;
+  // several sequences of (possibly) different lengths: the snake schedule
+  if (d == 72 && persistent && sk.n == 0 && prm.tpi == 2 && s.n_seqs > 1 &&
+      s.n_seqs <= attn::kMaxSnakeSeqs && n_items > grid)
+    prm.snake = 1;
   const bool rope = s.pos != nullptr;
   if (d == 72)
     return rope ? launch_hd<72, true>(maps, prm, grid, fr, sk, st)
