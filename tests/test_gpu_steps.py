@@ -222,6 +222,11 @@ ATTN_CASES = [
     (2, 128, [300, 90], 100, 1, False),
     (2, 128, [256, 129], 256, 2, True),
     (3, 72, [140, 77], 130, 3, True),
+    # 16 heads: pairs of query tiles; several lengths (and an empty image)
+    # take the longest-first snake schedule, 70 sequences the plain order
+    (16, 72, [700, 0, 300, 1300, 130, 1], 0, 0, False),
+    (16, 72, [int(v) for v in np.random.Generator(np.random.PCG64(7)).integers(1, 200, 70)], 0, 0,
+     False),
 ]
 
 
